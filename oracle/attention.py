@@ -1,0 +1,188 @@
+"""Plain, slow fp64 CPU oracle for exact softmax attention and its gradients.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this module:
+only the test-suite, the smoke check in ``__graft_entry__`` and the ``cpu_baseline``
+/ ``--impl reference`` legs of ``bench.py`` call it. It shares no code with the
+CUDA path (no kernels, headers, helpers or constants) and imports nothing from it.
+
+What it computes is the plain definition of attention, written out with the full
+N x N score matrix materialised per (batch, head), in float64:
+
+    S   = scale * Q K^T                         (then -inf where masked)
+    P   = softmax_rows(S)                       (max-subtracted)
+    lse = m + ln sum_j exp(S_ij - m)            (natural log, scale and mask included)
+    O   = P V
+
+The pages on which the method is described state that the tiled algorithm reaches
+this same result "with no approximation" ("FlashAttention-2: Faster Attention with
+Better Parallelism and Work Partitioning" review, Abstract; "... Proposed method",
+first bullet: output unchanged) and that it computes accurate attention ("Researchers
+at Stanford University Propose FlashAttention: Fast and Memory-Efficient Exact
+Attention with IO-Awareness", method paragraph). The oracle is therefore the
+definition itself; it deliberately does what the method avoids (store S and P).
+
+Masks:
+  * causal: key j is visible to query i iff j <= i (square problems only; the
+    review's "Proposed method" bullet on causal masking gives no formula, and every
+    workload here has N_q = N_k).
+  * block-sparse: a [ceil(N/T), ceil(N/T)] 0/1 tile mask with T = ``mask_block``
+    keeps S_ij iff mask[i // T][j // T] != 0 (the block-sparse paragraph of the
+    Stanford summary page; the granularity T = 128 is this library's choice).
+    Causal and block-sparse may be combined (logical AND).
+  * a row with no visible key has P = 0, O = 0 and lse = -inf (the pages are
+    silent; this is the only value consistent with lse = ln sum exp over an empty
+    set).
+
+Backward: the gradients of L = sum(O * dO) with respect to Q, K, V, from the
+materialised P (the Stanford summary page, method paragraph: the normalisation
+factor saved by the forward lets the backward recompute attention):
+
+    dV = P^T dO,  dP = dO V^T,  D_i = sum_j P_ij dP_ij  (= sum_c dO_ic O_ic),
+    dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+
+Parity status: every function below is pinned by tests/test_oracle.py against
+closed forms, invariants, brute-force finite differences and a library routine;
+none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "attn_scores_ref",
+    "attn_probs_ref",
+    "attn_fwd_ref",
+    "attn_fwd_rows_ref",
+    "attn_bwd_ref",
+]
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast of any real array (bf16/fp32 via torch or numpy) to float64."""
+    if hasattr(x, "detach"):  # a torch tensor; keep torch out of the arithmetic
+        x = x.detach().to("cpu")
+        if str(x.dtype) in ("torch.bfloat16", "torch.float16"):
+            x = x.float()
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _visible(n_q_rows: np.ndarray, n_k: int, causal: bool, block_mask, mask_block: int) -> np.ndarray:
+    """Boolean [len(rows), n_k] visibility for the given absolute query rows."""
+    rows = np.asarray(n_q_rows, dtype=np.int64)
+    cols = np.arange(n_k, dtype=np.int64)
+    vis = np.ones((rows.shape[0], n_k), dtype=bool)
+    if causal:
+        vis &= cols[None, :] <= rows[:, None]
+    if block_mask is not None:
+        bm = np.asarray(block_mask) != 0
+        vis &= bm[rows[:, None] // mask_block, cols[None, :] // mask_block]
+    return vis
+
+
+def attn_scores_ref(q, k, scale: float, causal: bool = False, block_mask=None,
+                    mask_block: int = 128, rows=None) -> np.ndarray:
+    """Masked, scaled scores S for one head: q [Nq, d], k [N, d] -> [Nq, N] fp64.
+
+    ``rows`` gives the absolute index of each query row (default 0..Nq-1); masked
+    entries are -inf.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    if rows is None:
+        rows = np.arange(q.shape[0])
+    s = float(scale) * (q @ k.T)
+    vis = _visible(rows, k.shape[0], causal, block_mask, mask_block)
+    return np.where(vis, s, -np.inf)
+
+
+def _softmax_rows(s: np.ndarray):
+    """Row softmax of a masked score matrix; returns (P, lse). Empty rows -> (0, -inf)."""
+    m = np.max(s, axis=1, keepdims=True)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    e = np.exp(s - m_safe)  # exp(-inf) = 0 for masked entries
+    z = np.sum(e, axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p = np.where(empty, 0.0, e / np.where(empty, 1.0, z))
+        lse = np.where(empty, -np.inf, m_safe + np.log(np.where(empty, 1.0, z)))
+    return p, lse[:, 0]
+
+
+def attn_probs_ref(q, k, scale: float, causal: bool = False, block_mask=None,
+                   mask_block: int = 128) -> np.ndarray:
+    """Attention probabilities P for one head ([N, d] inputs) -> [N, N] fp64."""
+    p, _ = _softmax_rows(attn_scores_ref(q, k, scale, causal, block_mask, mask_block))
+    return p
+
+
+def attn_fwd_ref(q, k, v, causal: bool = False, scale: float | None = None,
+                 block_mask=None, mask_block: int = 128):
+    """Forward for [B, H, N, d] inputs -> (O [B,H,N,d], lse [B,H,N]) in fp64.
+
+    One (b, h) at a time: S materialised, masked, softmaxed, multiplied by V.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, H, N, v.shape[-1]))
+    lse = np.zeros((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            s = attn_scores_ref(q[b, h], k[b, h], scale, causal, block_mask, mask_block)
+            p, l = _softmax_rows(s)
+            o[b, h] = p @ v[b, h]
+            lse[b, h] = l
+    return o, lse
+
+
+def attn_fwd_rows_ref(q_rows, rows, k, v, causal: bool, scale: float,
+                      block_mask=None, mask_block: int = 128):
+    """Forward for a sample of query rows of ONE head.
+
+    q_rows [R, d] are the queries at absolute positions ``rows`` (length R); k, v are
+    the head's full [N, d] keys and values. Returns (O [R, d], lse [R]). Used for
+    sampled checks at sizes where the full N x N matrix is too large to hold.
+    """
+    s = attn_scores_ref(q_rows, k, scale, causal, block_mask, mask_block, rows=rows)
+    p, lse = _softmax_rows(s)
+    return p @ _f64(v), lse
+
+
+def attn_bwd_ref(q, k, v, do, causal: bool = False, scale: float | None = None,
+                 block_mask=None, mask_block: int = 128):
+    """Gradients of L = sum(O * dO) for [B, H, N, d] inputs, in fp64.
+
+    Returns a dict with dq, dk, dv ([B,H,N,d]), D ([B,H,N], sum_j P dP), and the
+    forward's o and lse. D is computed both as sum_j P_ij dP_ij and as
+    sum_c dO_ic O_ic; the two must agree (asserted).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = {name: np.zeros_like(q) for name in ("dq", "dk")}
+    out["dv"] = np.zeros_like(v)
+    out["o"] = np.zeros_like(v)
+    out["lse"] = np.zeros((B, H, N))
+    out["D"] = np.zeros((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            s = attn_scores_ref(q[b, h], k[b, h], scale, causal, block_mask, mask_block)
+            p, lse = _softmax_rows(s)
+            o = p @ v[b, h]
+            dv = p.T @ do[b, h]
+            dp = do[b, h] @ v[b, h].T
+            D = np.sum(p * dp, axis=1)
+            D_alt = np.sum(do[b, h] * o, axis=1)
+            assert np.allclose(D, D_alt, rtol=1e-9, atol=1e-9 * (1.0 + np.max(np.abs(D_alt), initial=0.0)))
+            ds = p * (dp - D[:, None])
+            out["dq"][b, h] = scale * (ds @ k[b, h])
+            out["dk"][b, h] = scale * (ds.T @ q[b, h])
+            out["dv"][b, h] = dv
+            out["o"][b, h] = o
+            out["lse"][b, h] = lse
+            out["D"][b, h] = D
+    return out
+
