@@ -1,0 +1,207 @@
+"""Exact tiled attention on B200 (sm_100a): thin Python binding of libfa.so.
+
+Every function here only marshals torch tensors into the C ABI declared in
+``include/fa.h``; all arithmetic runs in the library's CUDA kernels. PyTorch is
+used for device memory and streams only. There is no fallback: if the library
+is missing or a tensor is not a CUDA tensor, the call raises.
+
+    o, lse = forward(q, k, v, causal=False, scale=None)
+    o, lse = forward_blocksparse(q, k, v, tile_mask, scale=None)
+    dq, dk, dv = backward(q, k, v, o, lse, do, causal=False, scale=None)
+    dq, dk, dv = backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None)
+
+Tensors are bf16 [B, H, N, d] contiguous on one CUDA device; lse is fp32 [B, H, N];
+tile_mask is uint8 [N/128, N/128] on the same device. N % 128 == 0, d in {64, 128}.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+__all__ = [
+    "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
+    "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa.h")
+
+STATUS = {
+    0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_ALIGNMENT",
+    4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA", 6: "FA_ERR_DEVICE_TIMEOUT",
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        super().__init__(f"{what}: {STATUS.get(self.status, self.status)}")
+
+
+def lib_path() -> str:
+    return os.environ.get("FA_LIB", os.path.join(_HERE, "libfa.so"))
+
+
+_lib = None
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "fa_status_string": ([_i], ctypes.c_char_p),
+    "fa_version": ([], _i),
+    "fa_fwd": ([_vp] * 5 + [_i] * 5 + [_f, _vp], _i),
+    "fa_fwd_blocksparse": ([_vp] * 6 + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_workspace_bytes": ([_i] * 4, _sz),
+    "fa_bwd": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_blocksparse": ([_vp] * 10 + [_sz, _vp, _i] + [_i] * 4 + [_f, _vp], _i),
+    "fa_device_status": ([_vp, ctypes.POINTER(_i)], _i),
+}
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise FAError(5, f"{path} is missing; build it with `python -m exact_tiled_attention_34_b200.build`")
+        handle = ctypes.CDLL(path)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def exported_names():
+    """Function names declared in include/fa.h."""
+    with open(_HEADER) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(fa_\w+)\s*\(", src, re.M)))
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise FAError(status, what)
+
+
+def _stream_ptr(dev):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check_qkv(*ts):
+    import torch
+    t0 = ts[0]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (no CPU path)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v, o, dO must be bfloat16")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, N, d]")
+        if t.shape != t0.shape or t.device != t0.device:
+            raise ValueError("q, k, v (and o, dO) must share shape and device")
+    if t0.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+
+
+def _scale(scale, d):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def forward(q, k, v, causal: bool = False, scale=None, out=None, lse=None):
+    """O = softmax(scale q k^T [causal]) v and the fp32 row log-sum-exp."""
+    import torch
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    with torch.cuda.device(q.device):
+        st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                          B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_fwd")
+    return o, l
+
+
+def _check_mask(tile_mask, q, mask_block):
+    import torch
+    if tile_mask.dtype != torch.uint8 or not tile_mask.is_contiguous() or tile_mask.device != q.device:
+        raise ValueError("tile_mask must be a contiguous uint8 tensor on the device of q")
+    nt = q.shape[2] // mask_block
+    if tuple(tile_mask.shape) != (nt, nt):
+        raise ValueError(f"tile_mask must be [{nt}, {nt}]")
+
+
+def forward_blocksparse(q, k, v, tile_mask, scale=None, mask_block: int = 128, out=None, lse=None):
+    """Block-sparse forward: attention restricted to the kept 128x128 tiles."""
+    import torch
+    _check_qkv(q, k, v)
+    _check_mask(tile_mask, q, mask_block)
+    B, H, N, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    with torch.cuda.device(q.device):
+        st = lib().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                      tile_mask.data_ptr(), mask_block, B, H, N, d, _scale(scale, d),
+                                      _stream_ptr(q.device))
+    _check(st, "fa_fwd_blocksparse")
+    return o, l
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def _bwd_prep(q, k, v, o, lse, do, workspace, grads):
+    import torch
+    _check_qkv(q, k, v, o, do)
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    need = bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    return workspace, grads
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None, grads=None):
+    """Gradients (dq, dk, dv) of sum(O * dO) given the forward's o and lse."""
+    import torch
+    workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
+    B, H, N, d = q.shape
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                          B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None, mask_block: int = 128, workspace=None,
+                         grads=None):
+    """Block-sparse backward (same mask as the forward)."""
+    import torch
+    _check_mask(tile_mask, q, mask_block)
+    workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
+    B, H, N, d = q.shape
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                      do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                      workspace.data_ptr(), workspace.numel(), tile_mask.data_ptr(), mask_block,
+                                      B, H, N, d, _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_bwd_blocksparse")
+    return dq, dk, dv
+
+
+def device_status(device=None):
+    """Synchronise the current stream and return (status, detail) of the device status word."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    detail = ctypes.c_int(0)
+    with torch.cuda.device(dev):
+        st = lib().fa_device_status(_stream_ptr(dev), ctypes.byref(detail))
+    return int(st), int(detail.value)

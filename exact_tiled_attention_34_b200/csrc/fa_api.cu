@@ -1,0 +1,228 @@
+// fa_api.cu - the C ABI of libfa.so (declared in include/fa.h): argument checks,
+// TMA tensor-map encoding, kernel selection and launch. No allocation on any call
+// path; every buffer is the caller's.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kTimeoutNs = 4000000000ull;  // 4 s per device-side wait
+
+// Library status word, one per device (module globals are per device).
+__device__ int g_fa_status[2];
+
+// ------------------------------------------------------------------ argument checks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_sizes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows > INT_MAX || static_cast<long long>(B) * H > INT_MAX / 2) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (p == nullptr) return FA_ERR_INVALID_ARG;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_ALIGNMENT;
+  return FA_OK;
+}
+
+fa_status check_scale(float scale) { return std::isfinite(scale) ? FA_OK : FA_ERR_INVALID_ARG; }
+
+// ------------------------------------------------------------------ per-device state
+
+struct DeviceState {
+  std::once_flag once;
+  int* status = nullptr;  // device address of g_fa_status
+  cudaError_t err = cudaSuccess;
+};
+DeviceState g_dev[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+fa_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+// Device address of the status word for the current device (set up once).
+fa_status device_status_ptr(int** out) {
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, [&] {
+    void* ptr = nullptr;
+    st.err = cudaGetSymbolAddress(&ptr, g_fa_status);
+    if (st.err == cudaSuccess) {
+      st.status = static_cast<int*>(ptr);
+      st.err = cudaMemset(st.status, 0, sizeof(int) * 2);
+    }
+  });
+  if (st.err != cudaSuccess || st.status == nullptr) return FA_ERR_CUDA;
+  *out = st.status;
+  return FA_OK;
+}
+
+fa_status encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? FA_OK : FA_ERR_CUDA;
+}
+
+// [BH, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 columns x
+// `box_rows` rows with 128-byte swizzle, matching the MMA operand layout.
+fa_status make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * d * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+fa_status set_smem(K kernel, int bytes, std::once_flag (&flags)[kMaxDevices], cudaError_t (&errs)[kMaxDevices]) {
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  std::call_once(flags[dev], [&] {
+    errs[dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+  return errs[dev] == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
+                     cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE>;
+  constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
+  if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  const unsigned grid = unsigned(p.n_qblocks) * unsigned(p.BH);
+  kernel<<<grid, fa::FwdCfg<D>::kThreads, smem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
+                     int B, int H, int N, int d, int causal, float scale, void* stream) {
+  fa_status s;
+  if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
+  if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if ((s = encoder()) != FA_OK) return s;
+  int* status;
+  if ((s = device_status_ptr(&status)) != FA_OK) return s;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if ((s = make_map(&mq, q, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, BH, N, d, 128)) != FA_OK) return s;
+  fa::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.tile_mask = mask;
+  p.status = status;
+  p.timeout_ns = kTimeoutNs;
+  p.N = N;
+  p.BH = BH;
+  p.n_tiles = N / 128;
+  p.n_qblocks = (p.n_tiles + 1) / 2;
+  p.c_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mask) {
+    return d == 64 ? launch_fwd<64, false, true>(mq, mk, mv, p, st) : launch_fwd<128, false, true>(mq, mk, mv, p, st);
+  }
+  if (causal) {
+    return d == 64 ? launch_fwd<64, true, false>(mq, mk, mv, p, st) : launch_fwd<128, true, false>(mq, mk, mv, p, st);
+  }
+  return d == 64 ? launch_fwd<64, false, false>(mq, mk, mv, p, st) : launch_fwd<128, false, false>(mq, mk, mv, p, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+int fa_version(void) { return 100; }
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 int causal, float scale, void* stream) {
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, N, d, causal != 0, scale, stream);
+}
+
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const uint8_t* tile_mask, int mask_block, int B, int H, int N, int d, float scale,
+                             void* stream) {
+  if (tile_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (mask_block != 128) return FA_ERR_UNSUPPORTED;
+  return fwd_common(q, k, v, o, lse, tile_mask, B, H, N, d, 0, scale, stream);
+}
+
+fa_status fa_device_status(void* stream, int* detail) {
+  int* status;
+  if (detail) *detail = 0;
+  if (device_status_ptr(&status) != FA_OK) return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpy(h, status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemset(status, 0, sizeof(h)) != cudaSuccess) return FA_ERR_CUDA;
+  if (detail) *detail = h[1];
+  return h[0] == 0 ? FA_OK : static_cast<fa_status>(h[0]);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------- backward (in progress)
+extern "C" {
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  const size_t rows = size_t(B) * H * N;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return up(rows * d * 4) + up(rows * 4);
+}
+fa_status fa_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*, void*,
+                 void*, size_t, int, int, int, int, int, float, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+fa_status fa_bwd_blocksparse(const void*, const void*, const void*, const void*, const float*, const void*, void*,
+                             void*, void*, void*, size_t, const uint8_t*, int, int, int, int, int, float, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+}

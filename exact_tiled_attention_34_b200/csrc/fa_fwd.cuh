@@ -1,0 +1,438 @@
+// fa_fwd.cuh - forward kernel: exact attention with online softmax on sm_100a.
+//
+// Method: "FlashAttention-2: Faster Attention with Better Parallelism and Work
+// Partitioning" (paper review), "Proposed method": online-softmax tiling, fewer
+// non-matmul FLOPs, parallelism over sequence length, work split between warps,
+// causal masking by skipping tiles; "Researchers at Stanford University Propose
+// FlashAttention ..." (summary), method paragraph: blocks of Q, K, V processed in
+// on-chip memory with the softmax reduced progressively, the normalisation factor
+// saved for the backward.
+//
+// One CTA owns a block of 2 x 128 query rows (two Q tiles) of one (batch, head) and
+// streams the 128-key K/V tiles it needs through a shared-memory ring:
+//   warp 0      TMA producer (one elected thread): Q once, then K_j, V_j per tile
+//   warp 1      MMA issuer (one thread) + TMEM allocator (whole warp)
+//   warps 4-7   softmax warpgroup for Q tile 0 (thread = query row = TMEM lane)
+//   warps 8-11  softmax warpgroup for Q tile 1
+// Tensor memory (512 columns): S0 | S1 | O0 | O1 (fp32), with the bf16 P_i written
+// over S_i (head dim 128) or into spare columns (head dim 64). The MMA warp
+// alternates between the two tiles so that the softmax of one tile overlaps the
+// matrix products of the other.
+//
+// Online softmax per row (base-2, scale folded into c = scale * log2 e):
+//   m' = max(m, c * max_j s_j); P_j = 2^(c s_j - m'); l = l 2^(m - m') + sum P_j;
+//   O = O 2^(m - m') + P V;  at the end O /= l, lse = (m + log2 l) ln 2.
+// The rescale of O in TMEM is skipped unless some row of the warp raised its max by
+// more than 8 (P then stays <= 2^8): the final O / l and lse use the same reference
+// max, so skipping is exact (a deferred normalisation).
+#pragma once
+
+#include "fa_ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  const uint8_t* tile_mask;  // [nT, nT] or nullptr
+  int* status;               // library status word (global)
+  unsigned long long timeout_ns;
+  int N;                     // sequence length (multiple of 128)
+  int BH;                    // B * H
+  int n_tiles;               // N / 128
+  int n_qblocks;             // ceil(n_tiles / 2)
+  float c_log2;              // scale * log2(e)
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kRows = 128;                   // rows per Q tile and per K/V tile
+  static constexpr int kColBlocks = D / 64;           // 128-byte column blocks per row
+  static constexpr int kBlockBytes = kRows * 128;     // one column block of a tile
+  static constexpr int kTileBytes = kRows * D * 2;    // one bf16 tile
+  static constexpr int kStages = (D == 64) ? 3 : 2;   // K/V ring depth
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
+  static constexpr int kThreads = 384;
+  // TMEM columns
+  __host__ __device__ static constexpr uint32_t tm_s(int i) { return i ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t tm_o(int i) { return 256u + (i ? uint32_t(D) : 0u); }
+  __host__ __device__ static constexpr uint32_t tm_p(int i) {
+    return D == 64 ? (i ? 448u : 384u) : tm_s(i);  // spare columns, or over S_i
+  }
+  static constexpr uint32_t kTmCols = 512;
+};
+
+// Barrier block in shared memory.
+template <int S>
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t k_full[S];
+  uint64_t v_full[S];
+  uint64_t kv_empty[S];
+  uint64_t s_full[2];
+  uint64_t p_ready[2];
+  uint64_t o_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Which of the CTA's two Q tiles need K/V tile j (bit 0: tile 0, bit 1: tile 1).
+template <bool CAUSAL, bool SPARSE>
+struct FwdSched {
+  int t0, t1;
+  bool valid1;
+  int n_tiles;
+  const uint8_t* mask;
+  __device__ __forceinline__ int last() const { return CAUSAL ? (valid1 ? t1 : t0) : n_tiles - 1; }
+  __device__ __forceinline__ uint32_t bits(int j) const {
+    bool k0 = CAUSAL ? (j <= t0) : true;
+    bool k1 = valid1 && (CAUSAL ? (j <= t1) : true);
+    if (SPARSE) {
+      k0 = k0 && (mask[size_t(t0) * n_tiles + j] != 0);
+      k1 = k1 && (mask[size_t(t1) * n_tiles + j] != 0);
+    }
+    return (k0 ? 1u : 0u) | (k1 ? 2u : 0u);
+  }
+  // Next j > j0 with a non-empty bit set (or -1).
+  __device__ __forceinline__ int next(int j0, uint32_t& b) const {
+    const int jl = last();
+    for (int j = j0 + 1; j <= jl; ++j) {
+      b = bits(j);
+      if (b) return j;
+    }
+    b = 0;
+    return -1;
+  }
+};
+
+// Wait-site codes reported through the status word (detail field).
+enum FwdSite : int {
+  kSiteFwdQ = 101, kSiteFwdKvEmpty, kSiteFwdKFull, kSiteFwdVFull, kSiteFwdPReady, kSiteFwdSFull,
+  kSiteFwdOFull, kSiteFwdDrain
+};
+
+// One softmax step for the calling thread's row: s[0..127] are the raw scores of
+// the current K/V tile; m is the running (base-2, scaled) reference max. Writes the
+// bf16 probabilities into TMEM at tp (64 columns of packed pairs), returns the two
+// partial row sums, the factor alpha = 2^(m - m_use) for the old O and l, and the new
+// reference max m_use. The rescale decision is warp-uniform (see the file header).
+// DIAG: the tile on the causal diagonal; column t is visible iff t <= r.
+template <bool DIAG>
+__device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, float m, uint32_t tp, float& sum0,
+                                            float& sum1, float& alpha, float& m_use) {
+  float mx;
+  if (c >= 0.f) {
+    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int t = 0; t < 128; ++t) a[t & 3] = fmaxf(a[t & 3], (DIAG && t > r) ? -INFINITY : s[t]);
+    mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * c;
+  } else {
+    float a[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+#pragma unroll
+    for (int t = 0; t < 128; ++t) a[t & 3] = fminf(a[t & 3], (DIAG && t > r) ? INFINITY : s[t]);
+    mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * c;
+  }
+  const float m_new = fmaxf(m, mx);
+  const bool rescale = __any_sync(0xffffffffu, m_new > m + 8.f);
+  m_use = rescale ? m_new : m;
+  const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+  alpha = ex2(m - m_sub);  // 0 on the first tile (m = -inf), 1 when the max is kept
+  sum0 = 0.f;
+  sum1 = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const int c0 = h * 64 + 2 * t;
+      float p0 = ex2(fmaf(s[c0], c, -m_sub));
+      float p1 = ex2(fmaf(s[c0 + 1], c, -m_sub));
+      if (DIAG) {
+        p0 = (c0 > r) ? 0.f : p0;
+        p1 = (c0 + 1 > r) ? 0.f : p1;
+      }
+      sum0 += p0;
+      sum1 += p1;
+      pk[t] = pack_bf16(p0, p1);
+    }
+    tmem_st32(tp + h * 32, pk);
+  }
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+__global__ void __launch_bounds__(384, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Cfg = FwdCfg<D>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
+  FwdBars<S>* bars = reinterpret_cast<FwdBars<S>*>(smem + Cfg::kOffBar);
+  uint8_t* sQ = smem + Cfg::kOffQ;
+  uint8_t* sK = smem + Cfg::kOffK;
+  uint8_t* sV = smem + Cfg::kOffV;
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  // Longest causal blocks first: linear block id -> (query block, batch*head).
+  const int lin = blockIdx.x;
+  const int qb = p.n_qblocks - 1 - lin / p.BH;
+  const int bh = lin % p.BH;
+
+  FwdSched<CAUSAL, SPARSE> sch;
+  sch.t0 = 2 * qb;
+  sch.t1 = 2 * qb + 1;
+  sch.valid1 = sch.t1 < p.n_tiles;
+  sch.n_tiles = p.n_tiles;
+  sch.mask = p.tile_mask;
+
+  WaitCtl wc{&bars->abort, p.status, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_ready[i], 128);
+      mbar_init(&bars->o_full[i], 1);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, Cfg::kTmCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint64_t keep = policy_evict_last();
+      mbar_arrive_expect_tx(&bars->q_full, Cfg::kTileBytes * (sch.valid1 ? 2 : 1));
+      for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+        tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, sch.t0 * 128, bh);
+      if (sch.valid1)
+        for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+          tma_load_3d(sQ + Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64,
+                      sch.t1 * 128, bh);
+      int it = 0;
+      uint32_t b;
+      for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b), ++it) {
+        const int st = it % S;
+        const int n = it / S;
+        if (n > 0 && !mbar_wait(&bars->kv_empty[st], (n - 1) & 1, wc, kSiteFwdKvEmpty)) break;
+        uint8_t* dk = sK + st * Cfg::kTileBytes;
+        uint8_t* dv = sV + st * Cfg::kTileBytes;
+        mbar_arrive_expect_tx(&bars->k_full[st], Cfg::kTileBytes);
+        for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+          tma_load_3d_hint(dk + cb * Cfg::kBlockBytes, &tm_k, &bars->k_full[st], cb * 64, j * 128, bh, keep);
+        mbar_arrive_expect_tx(&bars->v_full[st], Cfg::kTileBytes);
+        for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+          tma_load_3d_hint(dv + cb * Cfg::kBlockBytes, &tm_v, &bars->v_full[st], cb * 64, j * 128, bh, keep);
+      }
+      // On abort, wait (bounded) for this thread's own copies still in flight.
+      if (bars->abort) {
+        mbar_wait_drain(&bars->q_full, 0, wc, kSiteFwdDrain);
+        for (int i = (it > S ? it - S : 0); i < it; ++i) {
+          mbar_wait_drain(&bars->k_full[i % S], (i / S) & 1, wc, kSiteFwdDrain);
+          mbar_wait_drain(&bars->v_full[i % S], (i / S) & 1, wc, kSiteFwdDrain);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);  // S = Q K^T, both K-major
+      constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // O += P V, V is N-major
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      auto issue_s = [&](int i, int st) {
+        const uint32_t qa = sQa + i * Cfg::kTileBytes;
+        const uint32_t ka = sKa + st * Cfg::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * Cfg::kBlockBytes + (k & 3) * 32;
+          mma_ss(tmem + Cfg::tm_s(i), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS,
+                 k > 0);
+        }
+      };
+      auto issue_pv = [&](int i, int st, bool acc) {
+        const uint32_t va = sVa + st * Cfg::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k) {
+          mma_ts(tmem + Cfg::tm_o(i), tmem + Cfg::tm_p(i) + k * 8,
+                 sdesc_sw128(va + k * 16 * 128, Cfg::kBlockBytes, 1024), idO, (acc || k > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, wc, kSiteFwdQ);
+      tc_fence_after();
+      uint32_t issued = 0;
+      int cnt[2] = {0, 0};
+      int it = 0;
+      uint32_t b = 0, bn = 0;
+      int j = ok ? sch.next(-1, b) : -1;
+      while (j >= 0) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        const int jn = sch.next(j, bn);
+        const int stn = (it + 1) % S;
+        const uint32_t phn = ((it + 1) / S) & 1;
+        const uint32_t need = b & ~issued;
+        if (need) {
+          if (!mbar_wait(&bars->k_full[st], ph, wc, kSiteFwdKFull)) { ok = false; break; }
+          tc_fence_after();
+          for (int i = 0; i < 2; ++i)
+            if (need & (1u << i)) {
+              issue_s(i, st);
+              mma_commit(&bars->s_full[i]);
+            }
+        }
+        if (!mbar_wait(&bars->v_full[st], ph, wc, kSiteFwdVFull)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t next_issued = 0;
+        for (int i = 0; i < 2; ++i) {
+          if (!(b & (1u << i))) continue;
+          if (!mbar_wait(&bars->p_ready[i], cnt[i] & 1, wc, kSiteFwdPReady)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(i, st, cnt[i] > 0);
+          ++cnt[i];
+          if (jn >= 0 && (bn & (1u << i))) {
+            if (!mbar_wait(&bars->k_full[stn], phn, wc, kSiteFwdKFull)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(i, stn);
+            mma_commit(&bars->s_full[i]);
+            next_issued |= 1u << i;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bars->kv_empty[st]);
+        issued = next_issued;
+        b = bn;
+        j = jn;
+        ++it;
+      }
+      if (ok) {
+        mma_commit(&bars->o_full[0]);
+        mma_commit(&bars->o_full[1]);
+      }
+      // Every MMA issued by this thread must finish before TMEM is released.
+      mma_commit(&bars->mma_done);
+      mbar_wait_drain(&bars->mma_done, 0, wc, kSiteFwdDrain);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int i = (warp - 4) >> 2;  // Q tile of this warpgroup
+    const int quarter = warp & 3;   // TMEM lane quarter
+    const int r = quarter * 32 + lane;
+    const int tile = i == 0 ? sch.t0 : sch.t1;
+    const bool active = (i == 0) || sch.valid1;
+    const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
+    const float c = p.c_log2;
+    float m = -INFINITY, l = 0.f;
+    int cnt = 0;
+    bool ok = true;
+    if (active) {
+      uint32_t b;
+      for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b)) {
+        if (!(b & (1u << i))) continue;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], cnt & 1, wc, kSiteFwdSFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t raw[32];
+          tmem_ld32(trow + Cfg::tm_s(i) + q4 * 32, raw);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) s[q4 * 32 + t] = __uint_as_float(raw[t]);
+        }
+        tmem_wait_ld();
+        float sum0, sum1, alpha, m_use;
+        if (CAUSAL && j == tile)
+          softmax_row<true>(s, r, c, m, trow + Cfg::tm_p(i), sum0, sum1, alpha, m_use);
+        else
+          softmax_row<false>(s, r, c, m, trow + Cfg::tm_p(i), sum0, sum1, alpha, m_use);
+        const bool rescale = m_use != m;
+        l = l * alpha + (sum0 + sum1);
+        if (__any_sync(0xffffffffu, rescale) && cnt > 0) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t ov[32];
+            tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * alpha);
+            tmem_st32(trow + Cfg::tm_o(i) + cc * 32, ov);
+          }
+        }
+        m = m_use;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready[i]);
+        ++cnt;
+      }
+      // ---------------------------------------------------------- epilogue
+      const size_t row = size_t(bh) * p.N + size_t(tile) * 128 + r;
+      __nv_bfloat16* orow = p.o + row * D;
+      if (ok && cnt > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[i], 0, wc, kSiteFwdOFull));
+        if (ok) {
+          tc_fence_after();
+          const float inv_l = 1.f / l;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t ov[32];
+            tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, ov);
+            tmem_wait_ld();
+            uint4 pk[4];
+            uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              pw[t] = pack_bf16(__uint_as_float(ov[2 * t]) * inv_l, __uint_as_float(ov[2 * t + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) dst[t] = pk[t];
+          }
+          p.lse[row] = (m + __log2f(l)) * 0.69314718055994531f;
+        }
+      } else if (ok) {
+        // No visible key for this row (only possible with a block mask).
+        uint4 z = make_uint4(0, 0, 0, 0);
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t) dst[t] = z;
+        p.lse[row] = -INFINITY;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,144 @@
+/*
+ * fa.h - C ABI of the exact tiled attention library (libfa.so), sm_100a.
+ *
+ * The library computes exact softmax attention
+ *
+ *     O = softmax(scale * Q K^T [+ causal mask | block mask]) V
+ *
+ * tile by tile with an online softmax, so the N x N score matrix never reaches
+ * device memory, and the gradients of a scalar loss with respect to Q, K and V
+ * by recomputing the attention tiles from the saved per-row log-sum-exp.
+ *
+ * Sources of the operations (pages on the method):
+ *  - "FlashAttention-2: Faster Attention with Better Parallelism and Work
+ *    Partitioning" (paper review), Abstract and "Proposed method": exact result,
+ *    online-softmax tiling, parallelism over sequence length as well as batch and
+ *    heads, causal masking by skipping blocks.
+ *  - "Researchers at Stanford University Propose FlashAttention: Fast and
+ *    Memory-Efficient Exact Attention with IO-Awareness" (summary), method
+ *    paragraphs: inputs split into blocks with the softmax reduced progressively;
+ *    the forward's softmax normalisation factor saved so that the backward
+ *    recomputes attention on chip; block-sparse attention as a variant.
+ *
+ * Common conventions for every call
+ *  - Tensors q, k, v, o, dO, dq, dk, dv: bfloat16, shape [B, H, N, d], contiguous,
+ *    d innermost; element (b, h, n, c) at offset ((b*H + h)*N + n)*d + c.
+ *  - lse: float32 [B, H, N]; lse[b,h,i] = ln sum_j exp(scale * q_i . k_j) over the
+ *    keys visible to row i (natural log, scale and mask included); -INFINITY for
+ *    a row that sees no key (possible only with a block mask).
+ *  - All pointers are DEVICE pointers on the current device, except where noted.
+ *    Every base pointer must be 16-byte aligned.
+ *  - Supported sizes: B, H, N >= 1; N % 128 == 0; d in {64, 128}. B*H*N must fit
+ *    in int32.
+ *  - Causal: key j is visible to query i iff j <= i (top-left aligned; N_q = N_k).
+ *  - Block mask (tile_mask): uint8 [N/128, N/128] device array, row-major,
+ *    1 = tile kept, 0 = tile skipped, shared by every (b, h). Within a kept tile
+ *    every element is visible (the mask is not combined with causal).
+ *  - Ownership: the caller owns every buffer. The library allocates and frees no
+ *    device memory on these paths; scratch is caller-provided ("workspace").
+ *  - Asynchrony: each call only enqueues work on `stream` (a cudaStream_t, or
+ *    NULL for the legacy default stream) and returns; no implicit synchronisation.
+ *    Inputs must stay unmodified, and outputs unread, until the stream reaches
+ *    that point.
+ *  - Errors: arguments are checked synchronously before anything is enqueued; on
+ *    a non-FA_OK return nothing has been written. A launch failure reported by the
+ *    CUDA runtime returns FA_ERR_CUDA. Kernels never trap: a device-side wait that
+ *    exceeds its time limit makes the kernel record FA_ERR_DEVICE_TIMEOUT in a
+ *    library status word and return early; read it with fa_device_status().
+ *  - Thread safety: calls may be made from several host threads on different
+ *    streams.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, non-finite scale */
+  FA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, N % 128 != 0, mask_block != 128 */
+  FA_ERR_ALIGNMENT = 3,       /* a base pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,       /* workspace too small */
+  FA_ERR_CUDA = 5,            /* the CUDA runtime or driver reported an error */
+  FA_ERR_DEVICE_TIMEOUT = 6   /* a kernel gave up waiting (see fa_device_status) */
+} fa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Forward (the review's "Proposed method": online-softmax tiling, sequence-length
+ * parallelism; the summary's saved normalisation factor).
+ *   q, k, v : [B,H,N,d] bf16 inputs.
+ *   o       : [B,H,N,d] bf16 output, O = P V rounded to nearest-even.
+ *   lse     : [B,H,N] fp32 output (see conventions).
+ *   causal  : 0 = full attention, 1 = causal mask.
+ *   scale   : softmax scale (usually 1/sqrt(d)); any finite value.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Block-sparse forward (the summary's block-sparse paragraph): as fa_fwd without
+ * the causal flag, restricted to the kept tiles of `tile_mask`. Skipped tiles
+ * cost neither loads nor matrix products. mask_block must be 128.
+ */
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const uint8_t* tile_mask, int mask_block,
+                             int B, int H, int N, int d, float scale, void* stream);
+
+/*
+ * Bytes of device scratch that fa_bwd / fa_bwd_blocksparse need for these sizes:
+ * an fp32 [B,H,N,d] dQ accumulator plus the fp32 [B,H,N] row terms
+ * D_i = sum_c dO_ic O_ic, each rounded up to 256 bytes. Returns 0 for
+ * non-positive sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward (the summary's method paragraph: attention recomputed on chip from
+ * the saved normalisation factor). Gradients of L = sum(O * dO):
+ *   dv = P^T dO, dS = P * (dO V^T - D), dq = scale dS K, dk = scale dS^T Q.
+ *   q, k, v, o, lse : the forward's inputs and outputs (o and lse from fa_fwd
+ *                     with the same causal flag and scale).
+ *   dO              : [B,H,N,d] bf16 upstream gradient.
+ *   dq, dk, dv      : [B,H,N,d] bf16 outputs.
+ *   workspace       : device scratch of at least fa_bwd_workspace_bytes(B,H,N,d)
+ *                     bytes, 256-byte aligned; its contents on entry do not
+ *                     matter; it must not be shared with a concurrent call.
+ * dq is accumulated with fp32 atomic adds across key tiles, so its summation
+ * order (and last bits) may differ from run to run; dk and dv are deterministic.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes,
+                 int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/* Block-sparse backward: fa_bwd restricted to the kept tiles of `tile_mask`. */
+fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                             void* workspace, size_t workspace_bytes,
+                             const uint8_t* tile_mask, int mask_block,
+                             int B, int H, int N, int d, float scale, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the library's device status
+ * word for the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel since
+ * the last call gave up on a wait. *detail (if non-NULL, host pointer) receives
+ * a kernel-specific code naming the wait that expired (0 if none).
+ */
+fa_status fa_device_status(void* stream, int* detail);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,93 @@
+"""CPU tests of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments synchronously without touching a GPU."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+import torch
+
+import exact_tiled_attention_34_b200 as fa
+
+OK, INVALID, UNSUPPORTED, ALIGN, WORKSPACE, CUDA = 0, 1, 2, 3, 4, 5
+
+
+@pytest.fixture(scope="module")
+def L():
+    from exact_tiled_attention_34_b200 import build
+    build.build()
+    return fa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = fa.exported_names()
+    assert {"fa_fwd", "fa_bwd", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_bwd_workspace_bytes",
+            "fa_status_string", "fa_device_status", "fa_version"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True,
+                         check=True).stdout
+    defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in defined]
+    assert not missing, missing
+    for n in names:
+        assert getattr(L, n) is not None
+
+
+def test_status_strings(L):
+    for code, name in fa.STATUS.items():
+        assert L.fa_status_string(code).decode() == name
+    assert L.fa_status_string(99).decode() == "FA_ERR_UNKNOWN"
+    assert L.fa_version() >= 100
+
+
+A = 1 << 20  # fake, 16-byte aligned "device" addresses: never dereferenced by these checks
+
+
+def _fwd(L, q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
+    return L.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, None)
+
+
+def test_fwd_argument_checks(L):
+    assert _fwd(L, q=None) == INVALID
+    assert _fwd(L, lse=None) == INVALID
+    assert _fwd(L, k=A + 8) == ALIGN
+    assert _fwd(L, o=A + 2) == ALIGN
+    assert _fwd(L, B=0) == INVALID
+    assert _fwd(L, H=-1) == INVALID
+    assert _fwd(L, N=0) == INVALID
+    assert _fwd(L, d=32) == UNSUPPORTED
+    assert _fwd(L, d=96) == UNSUPPORTED
+    assert _fwd(L, N=130) == UNSUPPORTED
+    assert _fwd(L, B=1 << 16, H=1 << 16, N=128) == UNSUPPORTED  # B*H*N beyond int32
+    assert _fwd(L, scale=float("nan")) == INVALID
+    assert _fwd(L, scale=float("inf")) == INVALID
+
+
+def test_blocksparse_argument_checks(L):
+    f = L.fa_fwd_blocksparse
+    assert f(A, A, A, A, A, None, 128, 1, 1, 128, 64, 0.1, None) == INVALID
+    assert f(A, A, A, A, A, A, 64, 1, 1, 128, 64, 0.1, None) == UNSUPPORTED
+    assert f(A, A, A, A, A, A, 128, 1, 1, 128, 48, 0.1, None) == UNSUPPORTED
+
+
+def test_workspace_bytes(L):
+    up = lambda x: (x + 255) // 256 * 256
+    for (B, H, N, d) in ((1, 1, 128, 64), (8, 16, 2048, 64), (2, 16, 8192, 128), (3, 5, 384, 128)):
+        rows = B * H * N
+        assert L.fa_bwd_workspace_bytes(B, H, N, d) == up(rows * d * 4) + up(rows * 4)
+    assert L.fa_bwd_workspace_bytes(0, 1, 128, 64) == 0
+    assert L.fa_bwd_workspace_bytes(1, 1, -128, 64) == 0
+
+
+def test_binding_rejects_cpu_tensors():
+    q = torch.zeros((1, 1, 128, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q)
+    with pytest.raises(ValueError):
+        fa.backward(q, q, q, q, torch.zeros((1, 1, 128)), q)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(fa, "_lib", None)
+    monkeypatch.setenv("FA_LIB", str(tmp_path / "nope.so"))
+    with pytest.raises(fa.FAError):
+        fa.lib()

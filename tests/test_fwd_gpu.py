@@ -1,0 +1,161 @@
+"""GPU parity of the forward kernel (through the C ABI) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_tiled_attention_34_b200 as fa
+import oracle
+from exact_tiled_attention_34_b200.inputs import make_qkv, make_tile_mask, sweep_shape
+from tests.parity import assert_fwd_close, f64, sample_rows, sampled_fwd_check, tol_o_sharp
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(t, dev):
+    return {k: x.to(dev) for k, x in t.items()}
+
+
+def _full_check(B, H, N, d, causal, dev, scale=None, seed=0, mask=None, tol_o=None):
+    t = _dev(make_qkv(B, H, N, d, seed=seed, with_do=False), dev)
+    sc = 1.0 / math.sqrt(d) if scale is None else scale
+    if mask is None:
+        o, lse = fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc)
+    else:
+        o, lse = fa.forward_blocksparse(t["q"], t["k"], t["v"], mask.to(dev), scale=sc)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attn_fwd_ref(t["q"], t["k"], t["v"], causal, sc,
+                                       None if mask is None else mask.numpy(), 128)
+    assert_fwd_close(o, lse, o_ref, l_ref, f"B{B} H{H} N{N} d{d} causal={causal} scale={sc}", tol_o=tol_o)
+    assert fa.device_status() == (0, 0)
+    return t, o, lse
+
+
+def test_pr1(cuda_device):
+    """B=1, H=2, N=128, d=64, non-causal, seed 0."""
+    _full_check(1, 2, 128, 64, False, cuda_device)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 384, 512])
+def test_small_shapes(cuda_device, N, causal, d):
+    """Several tiles, an odd tile count (second Q tile of the last block absent)."""
+    _full_check(2, 3, N, d, causal, cuda_device, seed=N + d)
+
+
+@pytest.mark.parametrize("scale", [0.3, 1.0, -0.4, 0.0])
+def test_scales(cuda_device, scale):
+    """Any finite scale, including negative and zero (uniform attention).
+
+    Far from 1/sqrt(d) the softmax is peaked and |O| approaches max|V|, where the
+    bf16 rounding of P and of O each contribute up to 2^-9 |V|; the bound used here
+    is tol_o_sharp(V) (the spec'd 1e-2 holds for the workload scales).
+    """
+    for (H, d, causal, seed) in ((2, 64, True, 7), (1, 128, False, 8)):
+        t = make_qkv(1, H, 256, d, seed=seed, with_do=False)
+        _full_check(1, H, 256, d, causal, cuda_device, scale=scale, seed=seed, tol_o=tol_o_sharp(t["v"]))
+
+
+def test_causal_row0_exact(cuda_device):
+    """Causal: row 0 of every head sees only key 0, so O_0 = V_0 exactly."""
+    t, o, lse = _full_check(2, 2, 256, 128, True, cuda_device, seed=9)
+    assert torch.equal(o[:, :, 0], t["v"][:, :, 0])
+    ref = (t["q"][:, :, 0].double() * t["k"][:, :, 0].double()).sum(-1) / math.sqrt(128)
+    assert float((lse[:, :, 0].double() - ref).abs().max()) < 1e-3
+
+
+def test_equal_keys_give_mean_of_v(cuda_device):
+    """All keys equal: O is the mean of V (non-causal) / cumulative mean (causal)."""
+    B, H, N, d = 1, 2, 384, 64
+    t = _dev(make_qkv(B, H, N, d, seed=11, with_do=False), cuda_device)
+    k = t["k"][:, :, :1].expand(B, H, N, d).contiguous()
+    for causal in (False, True):
+        o, lse = fa.forward(t["q"], k, t["v"], causal=causal)
+        v = f64(t["v"])
+        ref = np.cumsum(v, axis=2) / np.arange(1, N + 1)[None, None, :, None] if causal else \
+            np.broadcast_to(v.mean(axis=2, keepdims=True), v.shape)
+        assert float(np.max(np.abs(f64(o) - ref))) <= 1e-2
+
+
+def test_deterministic(cuda_device):
+    t = _dev(make_qkv(2, 4, 1024, 128, seed=12, with_do=False), cuda_device)
+    a = fa.forward(t["q"], t["k"], t["v"], causal=True)
+    b = fa.forward(t["q"], t["k"], t["v"], causal=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_blocksparse_small(cuda_device, d):
+    N = 640
+    nt = N // 128
+    mask = make_tile_mask(nt, seed=3, density=0.4)
+    mask[2, :] = 0  # a tile row with nothing kept: O = 0, lse = -inf there
+    _, o, lse = _full_check(2, 2, N, d, False, cuda_device, seed=13, mask=mask)
+    assert torch.all(o[:, :, 256:384] == 0)
+    assert torch.all(torch.isneginf(lse[:, :, 256:384]))
+
+
+def test_blocksparse_all_ones_equals_dense(cuda_device):
+    t = _dev(make_qkv(1, 3, 768, 64, seed=14, with_do=False), cuda_device)
+    ones = torch.ones((6, 6), dtype=torch.uint8, device=cuda_device)
+    a = fa.forward(t["q"], t["k"], t["v"])
+    b = fa.forward_blocksparse(t["q"], t["k"], t["v"], ones)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_blocksparse_diagonal_equals_causal_free_blocks(cuda_device):
+    """Diagonal-only mask = independent attention inside each 128-token block."""
+    B, H, N, d = 1, 2, 512, 128
+    t = _dev(make_qkv(B, H, N, d, seed=15, with_do=False), cuda_device)
+    eye = torch.eye(4, dtype=torch.uint8, device=cuda_device)
+    o, lse = fa.forward_blocksparse(t["q"], t["k"], t["v"], eye)
+    for blk in range(4):
+        sl = slice(blk * 128, (blk + 1) * 128)
+        q, k, v = (t[n][:, :, sl].contiguous() for n in ("q", "k", "v"))
+        ob, lb = fa.forward(q, k, v)
+        assert float((o[:, :, sl].float() - ob.float()).abs().max()) <= 1e-2
+        assert float((lse[:, :, sl] - lb).abs().max()) <= 1e-3
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _sampled(B, H, N, d, causal, dev, mask=None, do_scale=1.0):
+    t = _dev(make_qkv(B, H, N, d, seed=0, with_do=False), dev)
+    sc = 1.0 / math.sqrt(d)
+    if mask is None:
+        o, lse = fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc)
+    else:
+        o, lse = fa.forward_blocksparse(t["q"], t["k"], t["v"], mask.to(dev), scale=sc)
+    torch.cuda.synchronize()
+    assert fa.device_status() == (0, 0)
+    heads = sorted({(0, 0), (B - 1, H - 1), (B // 2, H // 2)})
+    rows = sample_rows(N)
+    o_c, lse_c = o.cpu(), lse.cpu()
+    t_c = {k: x.cpu() for k, x in t.items()}
+    return sampled_fwd_check(t_c["q"], t_c["k"], t_c["v"], o_c, lse_c, causal, sc, heads, rows,
+                             None if mask is None else mask, f"B{B} H{H} N{N} d{d} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_b8h16n2048d64(cuda_device, causal):
+    _sampled(8, 16, 2048, 64, causal, cuda_device)
+
+
+def test_b2h16n8192d128_causal(cuda_device):
+    _sampled(2, 16, 8192, 128, True, cuda_device)
+
+
+def test_b1h16n16384d64_sparse(cuda_device):
+    mask = make_tile_mask(128, seed=0, density=0.25)
+    assert int(mask.sum()) == 4180
+    _sampled(1, 16, 16384, 64, False, cuda_device, mask=mask)
+
+
+@pytest.mark.parametrize("N", [512, 1024, 4096, 16384])
+@pytest.mark.parametrize("d", [64, 128])
+def test_sweep_points(cuda_device, N, d):
+    B, H = sweep_shape(N, d)
+    for causal in (False, True):
+        _sampled(B, H, N, d, causal, cuda_device)
