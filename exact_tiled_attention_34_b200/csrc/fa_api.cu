@@ -163,6 +163,101 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   return d == 64 ? launch_fwd<64, false, false>(mq, mk, mv, p, st) : launch_fwd<128, false, false>(mq, mk, mv, p, st);
 }
 
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t bwd_ws_bytes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  const size_t rows = size_t(B) * H * N;
+  return round256(rows * d * 4) + round256(rows * 4);
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const CUtensorMap& mdo, const fa::BwdParams& p, cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  auto kernel = fa::fa_bwd_kernel<D, CAUSAL, SPARSE>;
+  constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
+  if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
+  kernel<<<grid, 384, smem, stream>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int B, int H,
+                     int N, int d, int causal, float scale, void* stream) {
+  fa_status s;
+  if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv, ws})) != FA_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FA_ERR_ALIGNMENT;
+  if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if (ws_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
+  if ((s = encoder()) != FA_OK) return s;
+  int* status;
+  if ((s = device_status_ptr(&status)) != FA_OK) return s;
+  const int BH = B * H;
+  const size_t rows = size_t(BH) * N;
+  float* dqacc = static_cast<float*>(ws);
+  float* Drow = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round256(rows * d * 4));
+  CUtensorMap mq, mk, mv, mdo;
+  if ((s = make_map(&mq, q, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mdo, dO, BH, N, d, 128)) != FA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // 1) D = rowsum(dO * O), dQacc = 0
+  {
+    const long long threads = static_cast<long long>(rows) * (d / 8);
+    const unsigned grid = unsigned((threads + 255) / 256);
+    if (d == 64)
+      fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                      static_cast<const __nv_bfloat16*>(dO), Drow, dqacc,
+                                                      static_cast<long long>(rows));
+    else
+      fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                       static_cast<const __nv_bfloat16*>(dO), Drow, dqacc,
+                                                       static_cast<long long>(rows));
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  // 2) dK, dV and the dQ accumulation
+  fa::BwdParams p;
+  p.lse = lse;
+  p.Drow = Drow;
+  p.dqacc = dqacc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.tile_mask = mask;
+  p.status = status;
+  p.timeout_ns = kTimeoutNs;
+  p.N = N;
+  p.BH = BH;
+  p.n_tiles = N / 128;
+  p.scale = scale;
+  if (mask)
+    s = d == 64 ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, st)
+                : launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, st);
+  else if (causal)
+    s = d == 64 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, st)
+                : launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, st);
+  else
+    s = d == 64 ? launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, st)
+                : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, st);
+  if (s != FA_OK) return s;
+  // 3) dq = bf16(scale * dQacc)
+  {
+    const long long n4 = static_cast<long long>(rows) * d / 4;
+    const long long want = (n4 + 255) / 256;
+    const unsigned grid = unsigned(want < 148LL * 16 ? want : 148LL * 16);
+    fa::fa_bwd_dq_convert_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dqacc),
+                                                       static_cast<uint2*>(dq), scale, n4);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -209,20 +304,26 @@ fa_status fa_device_status(void* stream, int* detail) {
 
 }  // extern "C"
 
-// ---------------------------------------------------------------------------- backward (in progress)
+
 extern "C" {
-size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
-  const size_t rows = size_t(B) * H * N;
-  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return up(rows * d * 4) + up(rows * 4);
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) { return bwd_ws_bytes(B, H, N, d); }
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                 int causal, float scale, void* stream) {
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d, causal != 0,
+                    scale, stream);
 }
-fa_status fa_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*, void*,
-                 void*, size_t, int, int, int, int, int, float, void*) {
-  return FA_ERR_UNSUPPORTED;
+
+fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                             const uint8_t* tile_mask, int mask_block, int B, int H, int N, int d, float scale,
+                             void* stream) {
+  if (tile_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (mask_block != 128) return FA_ERR_UNSUPPORTED;
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, B, H, N, d, 0, scale,
+                    stream);
 }
-fa_status fa_bwd_blocksparse(const void*, const void*, const void*, const void*, const float*, const void*, void*,
-                             void*, void*, void*, size_t, const uint8_t*, int, int, int, int, int, float, void*) {
-  return FA_ERR_UNSUPPORTED;
-}
-}
+
+}  // extern "C"

@@ -5,6 +5,7 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
 """
 from .attention import (  # noqa: F401
     attn_bwd_ref,
+    attn_dq_rows_ref,
     attn_fwd_ref,
     attn_fwd_rows_ref,
     attn_probs_ref,

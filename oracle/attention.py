@@ -54,6 +54,7 @@ __all__ = [
     "attn_fwd_ref",
     "attn_fwd_rows_ref",
     "attn_bwd_ref",
+    "attn_dq_rows_ref",
 ]
 
 
@@ -186,3 +187,20 @@ def attn_bwd_ref(q, k, v, do, causal: bool = False, scale: float | None = None,
             out["D"][b, h] = D
     return out
 
+
+
+def attn_dq_rows_ref(q_rows, rows, k, v, do_rows, causal: bool, scale: float,
+                     block_mask=None, mask_block: int = 128) -> np.ndarray:
+    """dQ for a sample of query rows of ONE head (same definition as attn_bwd_ref).
+
+    Row i needs only its own scores: P_i = softmax(S_i), dP_i = dO_i V^T,
+    D_i = sum_j P_ij dP_ij, dS_i = P_i * (dP_i - D_i), dQ_i = scale dS_i K.
+    q_rows, do_rows [R, d] at absolute positions ``rows``; k, v the head's [N, d].
+    """
+    k, v, do_rows = _f64(k), _f64(v), _f64(do_rows)
+    s = attn_scores_ref(q_rows, k, scale, causal, block_mask, mask_block, rows=rows)
+    p, _ = _softmax_rows(s)
+    dp = do_rows @ v.T
+    D = np.sum(p * dp, axis=1)
+    ds = p * (dp - D[:, None])
+    return scale * (ds @ k)

@@ -269,6 +269,18 @@ def pin_gradient_invariants(mod):
         assert np.allclose(g["dv"].sum(axis=2), do.sum(axis=2), atol=1e-11)
 
 
+def pin_dq_rows_match_full(mod):
+    """The sampled-row dQ equals the corresponding rows of the full backward."""
+    N, T = 16, 4
+    q, k, v, do = (_rand((1, 1, N, 4), s) for s in (57, 58, 59, 60))
+    mask = _tiny_mask(N, T, seed=61)
+    rows = np.array([0, 2, 5, 8, 15])
+    for causal, m in ((False, None), (True, None), (False, mask)):
+        g = mod.attn_bwd_ref(q, k, v, do, causal, 0.7, m, T)
+        dq = mod.attn_dq_rows_ref(q[0, 0, rows], rows, k[0, 0], v[0, 0], do[0, 0, rows], causal, 0.7, m, T)
+        assert np.allclose(dq, g["dq"][0, 0, rows], atol=1e-12)
+
+
 FORWARD_PINS = [
     pin_probs_rows_sum_to_one,
     pin_equal_keys_mean_of_v,
@@ -288,5 +300,6 @@ BACKWARD_PINS = [
     pin_finite_differences,
     pin_D_two_ways,
     pin_gradient_invariants,
+    pin_dq_rows_match_full,
 ]
 ALL_PINS = FORWARD_PINS + BACKWARD_PINS
