@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Throughput of exact tiled attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = the whole hot path over one batch of synthetic input: for every
+variant of the workload (default: B=8, H=16, N=2048, d=64, non-causal and causal)
+the forward kernel, then the backward's three launches (D pre-pass, main
+kernel, dQ conversion). Metric: algorithmic TFLOPs/s, counting the forward as
+4 B H N^2 d (halved for causal, times the kept-tile fraction for block-sparse)
+and the backward as 2.5x the forward.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device
+synchronise; every step is timed with CUDA events on the launching stream, and
+L2 is flushed (256 MiB write) before each timed step, outside the step's events.
+Multi-GPU (torchrun): every rank runs the same workload on its own inputs (weak
+scaling, no data-path collective); the reported time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (plain definition, materialised
+scores) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd / fwd+bwd TFLOPs/s and % of B200 dense BF16 peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+# ---------------------------------------------------------------- workloads
+
+def workload(name: str):
+    """(B, H, N, d, variants) where a variant is (label, causal, sparse_density or None)."""
+    from exact_tiled_attention_34_b200.inputs import WORKLOADS, sweep_shape
+    if name.startswith("sweep_"):
+        # sweep_N4096_d128_causal / sweep_N4096_d128
+        parts = name.split("_")
+        N = int(parts[1][1:])
+        d = int(parts[2][1:])
+        B, H = sweep_shape(N, d)
+        causal = len(parts) > 3 and parts[3] == "causal"
+        return dict(B=B, H=H, N=N, d=d, variants=[("causal" if causal else "noncausal", causal, None)],
+                    do_scale=0.5)
+    w = WORKLOADS[name]
+    variants = []
+    if "sparse_density" in w:
+        variants.append(("blocksparse", False, w["sparse_density"]))
+    else:
+        for c in w["causal"]:
+            variants.append(("causal" if c else "noncausal", c, None))
+    return dict(B=w["B"], H=w["H"], N=w["N"], d=w["d"], variants=variants, do_scale=1.0)
+
+
+def fwd_flops(B, H, N, d, causal, density=1.0):
+    f = 4.0 * B * H * N * N * d
+    if causal:
+        f *= 0.5
+    return f * density
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_tiled_attention_34_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, wl_name: str):
+    """Per-launch DRAM bytes of `kernel` on `wl_name` from a committed ncu summary,
+    or None if there is none or the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{wl_name}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for ln in f:
+            if ":" in ln and not ln.startswith("#"):
+                k, v = ln.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+_HOST_INPUTS = {}
+
+
+def cpu_oracle_sample(wl, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle's forward+backward head by head (all variants of the
+    workload per head) until ~budget_s seconds have passed. Returns (TFLOPs/s, desc, s)."""
+    import oracle
+    from exact_tiled_attention_34_b200.inputs import make_qkv, make_tile_mask
+    B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
+    key = (B, H, N, d, seed, wl["do_scale"])
+    if key not in _HOST_INPUTS:
+        _HOST_INPUTS[key] = make_qkv(B, H, N, d, seed=seed, do_scale=wl["do_scale"])
+    t = _HOST_INPUTS[key]
+    sc = 1.0 / math.sqrt(d)
+    masks = {}
+    flops, heads, el = 0.0, 0, 0.0
+    for b in range(B):
+        for h in range(H):
+            x = {k: v[b:b + 1, h:h + 1] for k, v in t.items()}
+            for (label, causal, dens) in wl["variants"]:
+                m = None
+                if dens is not None:
+                    if dens not in masks:
+                        masks[dens] = make_tile_mask(N // 128, seed=seed, density=dens).numpy()
+                    m = masks[dens]
+                kept = 1.0 if m is None else float(m.sum()) / m.size
+                t0 = time.perf_counter()
+                oracle.attn_bwd_ref(x["q"], x["k"], x["v"], x["do"], causal, sc, m, 128)
+                el += time.perf_counter() - t0
+                flops += 3.5 * fwd_flops(1, 1, N, d, causal, kept)
+            heads += 1
+            if el >= budget_s:
+                break
+        if el >= budget_s:
+            break
+    desc = (f"{heads} of {B * H} (batch, head) pairs, fwd+bwd of every variant "
+            f"({', '.join(v[0] for v in wl['variants'])}), fp64 NumPy, {el:.1f} s")
+    return flops / el / 1e12, desc, el
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, wl_name, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    budget = 1.0  # seconds of oracle work per step
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, budget)
+    vals, times = [], []
+    for _ in range(args.steps):
+        v, desc, el = cpu_oracle_sample(wl, budget)
+        vals.append(v)
+        times.append(el)
+    value = statistics.mean(vals)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPs/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * statistics.mean(times), 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded inputs)",
+        "config": {"workload": wl_name, "B": wl["B"], "H": wl["H"], "N": wl["N"], "d": wl["d"],
+                   "variants": [v[0] for v in wl["variants"]]},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPs/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, wl_name, wl):
+    import torch
+    import torch.distributed as dist
+
+    import exact_tiled_attention_34_b200 as fa
+    from exact_tiled_attention_34_b200.inputs import make_qkv, make_tile_mask
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    fa.lib()
+
+    B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
+    sc = 1.0 / math.sqrt(d)
+    host = make_qkv(B, H, N, d, seed=rank, do_scale=wl["do_scale"])
+    t = {k: v.to(dev) for k, v in host.items()}
+    masks = {}
+    for (_, _, dens) in wl["variants"]:
+        if dens is not None:
+            masks[dens] = make_tile_mask(N // 128, seed=0, density=dens).to(dev)
+    ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    outs = {}
+    for (label, _, _) in wl["variants"]:
+        outs[label] = dict(o=torch.empty_like(t["q"]), lse=torch.empty((B, H, N), dtype=torch.float32, device=dev),
+                           dq=torch.empty_like(t["q"]), dk=torch.empty_like(t["q"]), dv=torch.empty_like(t["q"]))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    step_flops = 0.0
+    kinds = {}
+    for (label, causal, dens) in wl["variants"]:
+        kept = 1.0 if dens is None else float(masks[dens].float().mean())
+        f = fwd_flops(B, H, N, d, causal, kept)
+        kinds[label] = dict(causal=causal, mask=None if dens is None else masks[dens], fwd=f, bwd=2.5 * f)
+        step_flops += 3.5 * f
+
+    def one_step(ev=None):
+        # ev: dict label -> list of 5 events [start, after fwd, after pre, after main, after convert]
+        for (label, causal, _) in wl["variants"]:
+            k = kinds[label]
+            x = outs[label]
+            e = None if ev is None else ev[label]
+            if e:
+                e[0].record(stream)
+            if k["mask"] is None:
+                fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc, out=x["o"], lse=x["lse"])
+            else:
+                fa.forward_blocksparse(t["q"], t["k"], t["v"], k["mask"], scale=sc, out=x["o"], lse=x["lse"])
+            if e:
+                e[1].record(stream)
+            fa.bwd_preprocess(x["o"], t["do"], ws)
+            if e:
+                e[2].record(stream)
+            fa.bwd_main(t["q"], t["k"], t["v"], x["lse"], t["do"], x["dk"], x["dv"], ws, causal=causal, scale=sc,
+                        tile_mask=k["mask"])
+            if e:
+                e[3].record(stream)
+            fa.bwd_dq_convert(ws, x["dq"], scale=sc)
+            if e:
+                e[4].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(dev)
+    st, dt = fa.device_status(dev)
+    if st != 0:
+        raise SystemExit(f"device status {st} (site {dt}) after warm-up")
+
+    evs = [{label: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for (label, _, _) in wl["variants"]}
+           for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        flush.zero_()
+        one_step(evs[s])
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    st, dt = fa.device_status(dev)
+    if st != 0:
+        raise SystemExit(f"device status {st} (site {dt}) in the timed region")
+
+    # per-kernel and per-step device times (ms)
+    per = {label: dict(fwd=0.0, pre=0.0, main=0.0, conv=0.0) for (label, _, _) in wl["variants"]}
+    step_ms = []
+    for s in range(args.steps):
+        tot = 0.0
+        for (label, _, _) in wl["variants"]:
+            e = evs[s][label]
+            a = [e[i].elapsed_time(e[i + 1]) for i in range(4)]
+            per[label]["fwd"] += a[0]
+            per[label]["pre"] += a[1]
+            per[label]["main"] += a[2]
+            per[label]["conv"] += a[3]
+            tot += sum(a)
+        step_ms.append(tot)
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    K = args.steps
+    value = world * step_flops * K / (total_ms * 1e-3) / 1e12
+
+    pk, pk_kind = peaks()
+    sustained = clk is not None and clk["sm_mhz"] < 0.9 * clk.get("sm_max_mhz", 1965.0)
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    peak_label = ("sustained" if sustained else "burst") + f" bf16, {pk_kind}"
+
+    breakdown = {}
+    main_flops, main_ms = 0.0, 0.0
+    for (label, _, _) in wl["variants"]:
+        k = kinds[label]
+        p = {kk: v / K for kk, v in per[label].items()}
+        bwd_ms = p["pre"] + p["main"] + p["conv"]
+        breakdown[label] = {
+            "fwd_ms": round(p["fwd"], 4), "bwd_ms": round(bwd_ms, 4),
+            "bwd_main_ms": round(p["main"], 4), "bwd_pre_ms": round(p["pre"], 4), "bwd_convert_ms": round(p["conv"], 4),
+            "fwd_tflops": round(k["fwd"] / (p["fwd"] * 1e-3) / 1e12, 2),
+            "bwd_tflops": round(k["bwd"] / (bwd_ms * 1e-3) / 1e12, 2),
+            "fwd_bwd_tflops": round(3.5 * k["fwd"] / ((p["fwd"] + bwd_ms) * 1e-3) / 1e12, 2),
+            "fwd_pct_peak": round(100 * k["fwd"] / (p["fwd"] * 1e-3) / 1e12 / peak, 1),
+            "bwd_pct_peak": round(100 * k["bwd"] / (bwd_ms * 1e-3) / 1e12 / peak, 1),
+        }
+        main_flops += k["bwd"]
+        main_ms += p["main"]
+    achieved = main_flops / (main_ms * 1e-3) / 1e12
+    roofline = {"kernel": "fa_bwd_kernel (backward main)", "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peak, "peak_kind": peak_label, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": profiled_traffic("fa_bwd_kernel", wl_name)}
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    e2e_steps = max(3, min(K, 10))
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    res_host = {label: {n: torch.empty(outs[label][n].shape, dtype=outs[label][n].dtype).pin_memory()
+                        for n in ("o", "lse", "dq", "dk", "dv")} for (label, _, _) in wl["variants"]}
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = sum(v.numel() * v.element_size() for r in res_host.values() for v in r.values())
+
+    def e2e_step():
+        x = {k: v.to(dev, non_blocking=True) for k, v in pin.items()}
+        for (label, causal, _) in wl["variants"]:
+            k = kinds[label]
+            if k["mask"] is None:
+                o, lse = fa.forward(x["q"], x["k"], x["v"], causal=causal, scale=sc)
+                g = fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, scale=sc, workspace=ws)
+            else:
+                o, lse = fa.forward_blocksparse(x["q"], x["k"], x["v"], k["mask"], scale=sc)
+                g = fa.backward_blocksparse(x["q"], x["k"], x["v"], o, lse, x["do"], k["mask"], scale=sc,
+                                            workspace=ws)
+            for n, v in zip(("o", "lse", "dq", "dk", "dv"), (o, lse) + tuple(g)):
+                res_host[label][n].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOPs/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs rounded to bf16; per-rank seeds)",
+        "config": {"workload": wl_name, "B": B, "H": H, "N": N, "d": d,
+                   "variants": [v[0] for v in wl["variants"]],
+                   "step": "per variant: forward, backward pre-pass, backward main, dQ convert",
+                   "l2": "flushed before every timed step (256 MiB write, outside the step events)",
+                   "parallelism": f"replicas x{world} (independent (batch, head) shards, no collective)"},
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "peak_tflops": peak, "peak_kind": peak_label,
+        "breakdown": breakdown,
+        "roofline": roofline,
+        "gpu_launches": 4 * len(wl["variants"]) * K,
+        "wall_s_timed_region": round(wall, 4),
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPs/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "api": "exact_tiled_attention_34_b200.forward/backward (C ABI), pinned host buffers"},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, el = cpu_oracle_sample(wl, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOPs/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="b8h16n2048d64")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, args.workload, wl)
+    return run_ours(args, args.workload, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

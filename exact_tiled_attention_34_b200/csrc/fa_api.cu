@@ -185,77 +185,114 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                     void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int B, int H,
-                     int N, int d, int causal, float scale, void* stream) {
+struct BwdArgs {
+  int BH;
+  size_t rows;
+  float* dqacc;
+  float* Drow;
+};
+
+// Checks shared by the backward stages; fills the workspace views.
+fa_status bwd_check(void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a) {
   fa_status s;
-  if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv, ws})) != FA_OK) return s;
+  if (ws == nullptr) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FA_ERR_ALIGNMENT;
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
-  if ((s = check_scale(scale)) != FA_OK) return s;
   if (ws_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
+  a->BH = B * H;
+  a->rows = size_t(a->BH) * N;
+  a->dqacc = static_cast<float*>(ws);
+  a->Drow = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round256(a->rows * d * 4));
+  return FA_OK;
+}
+
+fa_status bwd_pre(const void* o, const void* dO, void* ws, size_t ws_bytes, int B, int H, int N, int d,
+                  void* stream) {
+  fa_status s;
+  if ((s = check_ptrs({o, dO})) != FA_OK) return s;
+  BwdArgs a;
+  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long threads = static_cast<long long>(a.rows) * (d / 8);
+  const unsigned grid = unsigned((threads + 255) / 256);
+  const auto* ob = static_cast<const __nv_bfloat16*>(o);
+  const auto* db = static_cast<const __nv_bfloat16*>(dO);
+  if (d == 64)
+    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, a.Drow, a.dqacc, static_cast<long long>(a.rows));
+  else
+    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, a.Drow, a.dqacc, static_cast<long long>(a.rows));
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
+                   void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H, int N,
+                   int d, int causal, float scale, void* stream) {
+  fa_status s;
+  if ((s = check_ptrs({q, k, v, lse, dO, dk, dv})) != FA_OK) return s;
+  if (mask != nullptr && (mask_block != 128 || causal)) return FA_ERR_UNSUPPORTED;
+  BwdArgs a;
+  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
   int* status;
   if ((s = device_status_ptr(&status)) != FA_OK) return s;
-  const int BH = B * H;
-  const size_t rows = size_t(BH) * N;
-  float* dqacc = static_cast<float*>(ws);
-  float* Drow = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round256(rows * d * 4));
   CUtensorMap mq, mk, mv, mdo;
-  if ((s = make_map(&mq, q, BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mk, k, BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mv, v, BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mdo, dO, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mq, q, a.BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, a.BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, a.BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mdo, dO, a.BH, N, d, 128)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  // 1) D = rowsum(dO * O), dQacc = 0
-  {
-    const long long threads = static_cast<long long>(rows) * (d / 8);
-    const unsigned grid = unsigned((threads + 255) / 256);
-    if (d == 64)
-      fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                      static_cast<const __nv_bfloat16*>(dO), Drow, dqacc,
-                                                      static_cast<long long>(rows));
-    else
-      fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                       static_cast<const __nv_bfloat16*>(dO), Drow, dqacc,
-                                                       static_cast<long long>(rows));
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  }
-  // 2) dK, dV and the dQ accumulation
   fa::BwdParams p;
   p.lse = lse;
-  p.Drow = Drow;
-  p.dqacc = dqacc;
+  p.Drow = a.Drow;
+  p.dqacc = a.dqacc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.tile_mask = mask;
   p.status = status;
   p.timeout_ns = kTimeoutNs;
   p.N = N;
-  p.BH = BH;
+  p.BH = a.BH;
   p.n_tiles = N / 128;
   p.scale = scale;
   if (mask)
-    s = d == 64 ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, st)
-                : launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, st);
-  else if (causal)
-    s = d == 64 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, st)
-                : launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, st);
-  else
-    s = d == 64 ? launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, st)
-                : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, st);
-  if (s != FA_OK) return s;
-  // 3) dq = bf16(scale * dQacc)
-  {
-    const long long n4 = static_cast<long long>(rows) * d / 4;
-    const long long want = (n4 + 255) / 256;
-    const unsigned grid = unsigned(want < 148LL * 16 ? want : 148LL * 16);
-    fa::fa_bwd_dq_convert_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dqacc),
-                                                       static_cast<uint2*>(dq), scale, n4);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  }
-  return FA_OK;
+    return d == 64 ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, st)
+                   : launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, st);
+  if (causal)
+    return d == 64 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, st)
+                   : launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, st);
+  return d == 64 ? launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, st)
+                 : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, st);
+}
+
+fa_status bwd_convert(const void* ws, size_t ws_bytes, void* dq, int B, int H, int N, int d, float scale,
+                      void* stream) {
+  fa_status s;
+  if ((s = check_ptrs({dq})) != FA_OK) return s;
+  BwdArgs a;
+  if ((s = bwd_check(const_cast<void*>(ws), ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  const long long n4 = static_cast<long long>(a.rows) * d / 4;
+  const long long want = (n4 + 255) / 256;
+  const unsigned grid = unsigned(want < 148LL * 16 ? want : 148LL * 16);
+  fa::fa_bwd_dq_convert_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float4*>(a.dqacc), static_cast<uint2*>(dq), scale, n4);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int B, int H,
+                     int N, int d, int causal, float scale, void* stream) {
+  fa_status s;
+  // Validate everything before the first launch so that an error writes nothing.
+  if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv})) != FA_OK) return s;
+  BwdArgs a;
+  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if ((s = bwd_pre(o, dO, ws, ws_bytes, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = bwd_main(q, k, v, lse, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, d, causal, scale, stream)) != FA_OK)
+    return s;
+  return bwd_convert(ws, ws_bytes, dq, B, H, N, d, scale, stream);
 }
 
 }  // namespace
@@ -314,6 +351,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int causal, float scale, void* stream) {
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d, causal != 0,
                     scale, stream);
+}
+
+fa_status fa_bwd_preprocess(const void* o, const void* dO, void* workspace, size_t workspace_bytes, int B, int H,
+                            int N, int d, void* stream) {
+  return bwd_pre(o, dO, workspace, workspace_bytes, B, H, N, d, stream);
+}
+
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
+                      void* dv, void* workspace, size_t workspace_bytes, const uint8_t* tile_mask, int mask_block,
+                      int B, int H, int N, int d, int causal, float scale, void* stream) {
+  return bwd_main(q, k, v, lse, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N, d,
+                  causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void* dq, int B, int H, int N, int d,
+                            float scale, void* stream) {
+  return bwd_convert(workspace, workspace_bytes, dq, B, H, N, d, scale, stream);
 }
 
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -127,6 +127,29 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
                              int B, int H, int N, int d, float scale, void* stream);
 
 /*
+ * The three launches that make up fa_bwd / fa_bwd_blocksparse, for callers that
+ * schedule or time them separately. On one stream,
+ *   fa_bwd_preprocess; fa_bwd_main; fa_bwd_dq_convert
+ * is exactly fa_bwd (tile_mask = NULL) or fa_bwd_blocksparse (tile_mask set).
+ * Arguments have the meanings given for fa_bwd; the workspace must be the same
+ * buffer for all three.
+ *   fa_bwd_preprocess : D_i = sum_c dO_ic O_ic into the workspace, and the fp32
+ *                       dQ accumulator in the workspace set to zero.
+ *   fa_bwd_main       : dk, dv, and dQ products added into the accumulator.
+ *                       tile_mask may be NULL (then `causal` applies) or a block
+ *                       mask (then causal must be 0 and mask_block 128).
+ *   fa_bwd_dq_convert : dq = bf16(scale * accumulator).
+ */
+fa_status fa_bwd_preprocess(const void* o, const void* dO, void* workspace, size_t workspace_bytes,
+                            int B, int H, int N, int d, void* stream);
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO,
+                      void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                      const uint8_t* tile_mask, int mask_block,
+                      int B, int H, int N, int d, int causal, float scale, void* stream);
+fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void* dq,
+                            int B, int H, int N, int d, float scale, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the library's device status
  * word for the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel since
  * the last call gave up on a wait. *detail (if non-NULL, host pointer) receives
