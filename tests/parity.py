@@ -24,7 +24,8 @@ def max_abs(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     both_ninf = np.isneginf(a) & np.isneginf(b)
-    d = np.where(both_ninf, 0.0, np.abs(a - b))
+    with np.errstate(invalid="ignore"):
+        d = np.where(both_ninf, 0.0, np.abs(a - b))
     return float(np.max(d)) if d.size else 0.0
 
 
