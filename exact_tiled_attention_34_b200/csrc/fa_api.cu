@@ -381,3 +381,60 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------- no-allocation backward
+// Scratch for fa_bwd_noalloc: a fixed array compiled into the library, so callers
+// that may not allocate device memory can still run the backward. Every device
+// that loads the library holds it until exit. In host code `g_noalloc_scratch`
+// only names the symbol; its device address comes from cudaGetSymbolAddress,
+// looked up once per device in noalloc_scratch() below.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocState {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoallocState g_noalloc[kMaxDevices];
+
+// Device address of the scratch array on the current device (first call: lookup).
+fa_status noalloc_scratch(void** out) {
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  NoallocState& st = g_noalloc[dev];
+  std::call_once(st.once, [&] {
+    void* ptr = nullptr;
+    st.err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    st.ptr = (st.err == cudaSuccess) ? ptr : nullptr;
+  });
+  if (st.err != cudaSuccess || st.ptr == nullptr) return FA_ERR_CUDA;
+  *out = st.ptr;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                    const void* dO, void* dq, void* dk, void* dv, const uint8_t* tile_mask,
+                                    int mask_block, int B, int H, int N, int d, int causal, float scale,
+                                    void* stream) {
+  fa_status s;
+  if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv})) != FA_OK) return s;
+  if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if (tile_mask != nullptr && (mask_block != 128 || causal)) return FA_ERR_UNSUPPORTED;
+  const size_t need = bwd_ws_bytes(B, H, N, d);
+  if (need > size_t(FA_BWD_NOALLOC_SCRATCH_BYTES)) return FA_ERR_WORKSPACE;
+  void* scratch;
+  if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
+  // The pre-pass zeroes the dQ accumulator and rewrites D, so whatever an earlier
+  // call left in the array does not matter.
+  const size_t bytes = size_t(FA_BWD_NOALLOC_SCRATCH_BYTES);
+  if ((s = bwd_pre(o, dO, scratch, bytes, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = bwd_main(q, k, v, lse, dO, dk, dv, scratch, bytes, tile_mask, mask_block, B, H, N, d, causal, scale,
+                    stream)) != FA_OK)
+    return s;
+  return bwd_convert(scratch, bytes, dq, B, H, N, d, scale, stream);
+}

@@ -150,6 +150,36 @@ fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void*
                             int B, int H, int N, int d, float scale, void* stream);
 
 /*
+ * Backward without caller-provided scratch (no counterpart on the pages: this is
+ * an interface convenience, not part of the method).
+ *
+ * For callers that cannot allocate device memory when they call the backward: a
+ * plugin whose host application owns all device memory and hands it only the
+ * input and output buffers, or a latency-critical loop that must not pay the
+ * implicit device synchronisation of cudaMalloc/cudaFree. Same arguments and
+ * results as fa_bwd / fa_bwd_blocksparse (tile_mask NULL or a 128-granular block
+ * mask with causal = 0), but the fp32 scratch (dQ accumulator and D rows) lives in
+ * one array compiled into the library: FA_BWD_NOALLOC_SCRATCH_BYTES bytes of device
+ * memory on every GPU that loads the library, held until the process exits.
+ *  - Sizes: needs fa_bwd_workspace_bytes(B,H,N,d) <= FA_BWD_NOALLOC_SCRATCH_BYTES
+ *    (e.g. B*H*N <= 129,024 rows at d = 64, <= 65,024 at d = 128); larger sizes
+ *    return FA_ERR_WORKSPACE and enqueue nothing.
+ *  - Allocation: none. No cudaMalloc, cudaFree or allocating library call.
+ *  - Set-up: the first call on a device (with that device current) looks up the
+ *    array's device address once; make that first call before any stream
+ *    capture on that device.
+ *  - Sharing: every call on a device uses the same array and leaves its contents
+ *    behind; each call re-initialises what it reads. Calls whose work overlaps on
+ *    the GPU (different streams, or several threads) race on the array: serialise
+ *    them (e.g. one stream).
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv,
+                         const uint8_t* tile_mask, int mask_block,
+                         int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the library's device status
  * word for the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel since
  * the last call gave up on a wait. *detail (if non-NULL, host pointer) receives
