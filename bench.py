@@ -474,6 +474,91 @@ def run_ours(args, wl_name, wl):
     return 0
 
 
+# ---------------------------------------------------------------- table of workloads
+
+def run_table(args):
+    """Per-workload forward / backward device times (not the contract line): one JSON line
+    per (workload, variant), median of --steps timed repetitions, L2 flushed before each."""
+    import torch
+
+    import exact_tiled_attention_34_b200 as fa
+    from exact_tiled_attention_34_b200.inputs import SWEEP_D, SWEEP_N, make_qkv, make_tile_mask
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse"]
+    names += [f"sweep_N{N}_d{d}{c}" for d in SWEEP_D for N in SWEEP_N for c in ("", "_causal")]
+    if args.only:
+        names = [n for n in names if any(o in n for o in args.only.split(","))]
+    pk, pk_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for name in names:
+        wl = workload(name)
+        B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
+        sc = 1.0 / math.sqrt(d)
+        t = {k: v.to(dev) for k, v in make_qkv(B, H, N, d, seed=0, do_scale=wl["do_scale"]).items()}
+        ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(t["q"])
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dq, dk, dv = (torch.empty_like(t["q"]) for _ in range(3))
+        for (label, causal, dens) in wl["variants"]:
+            mask = None if dens is None else make_tile_mask(N // 128, seed=0, density=dens).to(dev)
+            kept = 1.0 if mask is None else float(mask.float().mean())
+            F = fwd_flops(B, H, N, d, causal, kept)
+
+            def fwd():
+                if mask is None:
+                    fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc, out=o, lse=lse)
+                else:
+                    fa.forward_blocksparse(t["q"], t["k"], t["v"], mask, scale=sc, out=o, lse=lse)
+
+            def pre():
+                fa.bwd_preprocess(o, t["do"], ws)
+
+            def main():
+                fa.bwd_main(t["q"], t["k"], t["v"], lse, t["do"], dk, dv, ws, causal=causal, scale=sc,
+                            tile_mask=mask)
+
+            def conv():
+                fa.bwd_dq_convert(ws, dq, scale=sc)
+
+            def timed(fns):
+                ms = []
+                for r in range(args.warmup + args.steps):
+                    flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    for f in fns:
+                        f()
+                    e1.record(stream)
+                    torch.cuda.synchronize(dev)
+                    if r >= args.warmup:
+                        ms.append(e0.elapsed_time(e1))
+                return statistics.median(ms)
+
+            t_f = timed([fwd])
+            row = {"workload": name, "variant": label, "B": B, "H": H, "N": N, "d": d, "kept": round(kept, 4),
+                   "fwd_ms": round(t_f, 4), "fwd_tflops": round(F / t_f / 1e9, 1),
+                   "fwd_pct_peak": round(100 * F / t_f / 1e9 / pk["bf16_tflops"], 1)}
+            if name != "pr1":
+                pre()
+                t_m = timed([main])
+                t_b = timed([pre, main, conv])
+                row.update({"bwd_ms": round(t_b, 4), "bwd_main_ms": round(t_m, 4),
+                            "bwd_tflops": round(2.5 * F / t_b / 1e9, 1),
+                            "bwd_main_tflops": round(2.5 * F / t_m / 1e9, 1),
+                            "bwd_pct_peak": round(100 * 2.5 * F / t_b / 1e9 / pk["bf16_tflops"], 1),
+                            "fwd_bwd_tflops": round(3.5 * F / (t_f + t_b) / 1e9, 1)})
+            st, site = fa.device_status(dev)
+            row["status"] = st
+            row["peak"] = f'{pk["bf16_tflops"]} ({pk_kind}, burst)'
+            print(json.dumps(row), flush=True)
+        del t, ws, o, lse, dq, dk, dv
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,9 +568,13 @@ def main():
     ap.add_argument("--workload", default="b8h16n2048d64")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table", action="store_true", help="per-workload fwd/bwd times (JSON lines), not the contract line")
+    ap.add_argument("--only", default="", help="with --table: comma-separated substrings of workload names")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.table:
+        return run_table(args)
     wl = workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, args.workload, wl)

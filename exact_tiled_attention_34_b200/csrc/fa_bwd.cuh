@@ -196,9 +196,11 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   const int warp = warp_id();
   const int lane = lane_id();
+  // Head-major order (the key tiles of one head run together and share its Q/dO
+  // tiles through L2), small j first within a head (most query tiles when causal).
   const int lin = blockIdx.x;
-  const int j = lin / p.BH;  // key tile: small j first (most query tiles when causal)
-  const int bh = lin % p.BH;
+  const int bh = lin / p.n_tiles;
+  const int j = lin % p.n_tiles;
   BwdSched<CAUSAL, SPARSE> sch{j, p.n_tiles, p.tile_mask};
   WaitCtl wc{&bars->abort, p.status, p.timeout_ns};
 

@@ -180,10 +180,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int warp = warp_id();
   const int lane = lane_id();
 
-  // Longest causal blocks first: linear block id -> (query block, batch*head).
+  // Head-major order (the query blocks of one head run together and share its K/V
+  // tiles through L2), longest causal blocks first within a head.
   const int lin = blockIdx.x;
-  const int qb = p.n_qblocks - 1 - lin / p.BH;
-  const int bh = lin % p.BH;
+  const int bh = lin / p.n_qblocks;
+  const int qb = p.n_qblocks - 1 - lin % p.n_qblocks;
 
   FwdSched<CAUSAL, SPARSE> sch;
   sch.t0 = 2 * qb;
