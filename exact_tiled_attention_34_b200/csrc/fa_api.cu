@@ -180,8 +180,19 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   auto kernel = fa::fa_bwd_kernel<D, CAUSAL, SPARSE>;
   constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  // The kernel re-divides its register pool between warpgroups; that is only valid
+  // if it was built with exactly the register count the split assumes.
+  static int regs[kMaxDevices];
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  if (regs[dev] == 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+    regs[dev] = attr.numRegs;
+  }
+  if (regs[dev] != fa::kBwdLaunchRegs) return FA_ERR_UNSUPPORTED;
   const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
-  kernel<<<grid, 384, smem, stream>>>(mq, mk, mv, mdo, p);
+  kernel<<<grid, 512, smem, stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -22,13 +22,16 @@
 // with vector atomics (order of the additions not fixed); dK and dV stay in TMEM
 // until the end. A final kernel converts the fp32 dQ accumulator to bf16.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner,
-// warps 4-7 "compute" (thread = key row: P^T, dS^T, epilogue for dK/dV),
-// warps 8-11 "dQ" (thread = query row: TMEM -> atomics).
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner,
+// warps 4-11 two "compute" warpgroups (thread = key row; warpgroup h takes query
+// columns [64h, 64h+64): P^T, dS^T; epilogue dK (h = 0) / dV (h = 1)),
+// warps 12-15 "dQ" (thread = query row: TMEM -> atomics).
 // TMEM columns, head dim 64:  dK 0 | dV 64 | S^T 128 | dP^T 256 | dQ 384
-//               head dim 128: dK 0 | dV 128 | S^T 256 | dP^T 384; dQ_i is split in
-// two 64-column halves placed over the S^T / dP^T columns that P^T / dS^T (bf16,
-// 64 columns each) leave free, so the next S^T waits until dQ_i has been read.
+//               head dim 128: dK 0 | dV 128 | S^T 256 | dP^T 384; dQ_i is formed in
+// two 64-column parts, one after the other, in the dP^T columns that dS^T (bf16,
+// 64 columns) leaves free. The next S^T is issued right after dV (it overwrites
+// P^T, which dV has read: products execute in issue order); the next dP^T waits
+// until the last dQ part has been read out.
 #pragma once
 
 #include "fa_ptx.cuh"
@@ -140,13 +143,27 @@ struct BwdBars {
   uint64_t dq_empty;
   uint64_t acc_done;
   uint64_t mma_done;
+  uint64_t rd_s;   // both compute warpgroups have read S^T of this tile
+  uint64_t rd_dp;  // ... and dP^T
   uint32_t tmem_base;
   int abort;
 };
 
+// Register split of the 512-thread backward block launched with 128 registers per
+// thread (65,536 in all): producer/MMA warpgroup 80, the two compute warpgroups 160
+// each, the dQ warpgroup 112 -> 128 * (80 + 160 + 160 + 112) = 65,536. The two
+// decreases happen first thing and are never undone; the compute warpgroups' single
+// increase needs exactly what they release.
+constexpr int kBwdLaunchRegs = 128;
+constexpr int kBwdRegsCtl = 80;
+constexpr int kBwdRegsCompute = 160;
+constexpr int kBwdRegsDq = 112;
+static_assert(128 * (kBwdRegsCtl + 2 * kBwdRegsCompute + kBwdRegsDq) <= 512 * kBwdLaunchRegs,
+              "register split exceeds the block's register pool");
+
 enum BwdSite : int {
   kSiteBwdKV = 201, kSiteBwdTEmpty, kSiteBwdTFull, kSiteBwdPReady, kSiteBwdDsReady, kSiteBwdDqEmpty,
-  kSiteBwdSFull, kSiteBwdDpFull, kSiteBwdDqFull, kSiteBwdAcc, kSiteBwdDrain, kSiteBwdAlign
+  kSiteBwdSFull, kSiteBwdDpFull, kSiteBwdDqFull, kSiteBwdAcc, kSiteBwdDrain, kSiteBwdAlign, kSiteBwdRead
 };
 
 // Query tiles that see key tile j.
@@ -171,11 +188,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 template <int D, bool CAUSAL, bool SPARSE>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdParams p) {
   using Cfg = BwdCfg<D>;
+  constexpr int kDqParts = Cfg::kAlias ? 2 : 1;  // dQ_i products (and read-outs) per query tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_off = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((base_off + 1023u) & ~1023u) - base_off);
@@ -212,12 +230,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_ready, 128);
-    mbar_init(&bars->ds_ready, 128);
+    mbar_init(&bars->p_ready, 256);
+    mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, 128);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->rd_s, 256);
+    mbar_init(&bars->rd_dp, 256);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -230,9 +250,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   constexpr uint32_t kTileTx = 2 * Cfg::kTileBytes + 2 * 512;
-
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    regs_dec<kBwdRegsCtl>();
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -266,12 +286,16 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           mbar_wait_drain(&bars->t_full[x & 1], (x >> 1) & 1, wc, kSiteBwdDrain);
       }
     }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    regs_dec<kBwdRegsCtl>();
     if (lane == 0) {
       constexpr uint32_t idT = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idG = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM, B N-major)
-      constexpr uint32_t idQ = idesc_bf16_f32(128, Cfg::kAlias ? 64 : D, 1, 1);  // dQ (A M-major, B N-major)
+      constexpr uint32_t idQ = idesc_bf16_f32(128, 64, 1, 1);   // dQ (part): A M-major, B N-major
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
                      aDS = smem_u32(sDS);
       // X[tm] = A[128 x D] * B[128 x D]^T with both operands K-major (A: key rows, B: query rows)
@@ -289,24 +313,14 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           mma_ts(tmem + tm, tmem + a_tm + k * 8, sdesc_sw128(b + k * 2048, Cfg::kBlockBytes, 1024), idG,
                  (acc || k > 0) ? 1u : 0u);
       };
-      // dQ_i = dS[q x kv] * K_j[kv x D]: A = dS stored M-major, B = K_j N-major
-      auto issue_dq = [&]() {
-        if (Cfg::kAlias) {
+      // 64 columns [64h, 64h+64) of dQ_i = dS[q x kv] * K_j[kv x D] into TMEM column tm
+      auto issue_dq = [&](uint32_t tm, int h) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t tm = h == 0 ? Cfg::kTmS + 64 : Cfg::kTmDP + 64;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              mma_ss(tmem + tm, sdesc_sw128(aDS + k * 2048, Cfg::kBlockBytes, 1024),
-                     sdesc_sw128(aK + h * Cfg::kBlockBytes + k * 2048, Cfg::kBlockBytes, 1024), idQ, k > 0);
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + Cfg::kTmDQ, sdesc_sw128(aDS + k * 2048, Cfg::kBlockBytes, 1024),
-                   sdesc_sw128(aK + k * 2048, Cfg::kBlockBytes, 1024), idQ, k > 0);
-        }
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + tm, sdesc_sw128(aDS + k * 2048, Cfg::kBlockBytes, 1024),
+                 sdesc_sw128(aK + h * Cfg::kBlockBytes + k * 2048, Cfg::kBlockBytes, 1024), idQ, k > 0);
       };
+      constexpr uint32_t kTmDqPart = Cfg::kAlias ? Cfg::kTmDP + 64 : Cfg::kTmDQ;
       bool ok = mbar_wait(&bars->kv_full, 0, wc, kSiteBwdKV);
       tc_fence_after();
       int i = ok ? sch.first() : -1;
@@ -328,34 +342,37 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int in = sch.next(i);
         const int stn = (it + 1) & 1;
         const uint32_t phn = ((it + 1) >> 1) & 1;
-        // dV += P^T dO_i
+        // dV += P^T dO_i, then at once S^T for the next query tile (it overwrites P^T
+        // only after this dV product has read it: products run in issue order).
         if (!mbar_wait(&bars->p_ready, it & 1, wc, kSiteBwdPReady)) { ok = false; break; }
         tc_fence_after();
         issue_g(Cfg::kTmDV, Cfg::kTmS, aDO + st * Cfg::kTileBytes, it > 0);
-        // Without aliasing, the next S^T can start now (P^T has been issued for reading).
-        if (!Cfg::kAlias && in >= 0) {
+        if (in >= 0) {
           if (!mbar_wait(&bars->t_full[stn], phn, wc, kSiteBwdTFull)) { ok = false; break; }
           tc_fence_after();
           issue_t(Cfg::kTmS, aK, aQ + stn * Cfg::kTileBytes);
           mma_commit(&bars->s_full);
         }
-        // dK += dS^T Q_i ; dQ_i = dS K_j
+        // dK += dS^T Q_i ; dQ_i = dS K_j (in kDqParts column parts of 64)
         if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteBwdDsReady)) { ok = false; break; }
         tc_fence_after();
         issue_g(Cfg::kTmDK, Cfg::kTmDP, aQ + st * Cfg::kTileBytes, it > 0);
-        if (it > 0 && !mbar_wait(&bars->dq_empty, (it - 1) & 1, wc, kSiteBwdDqEmpty)) { ok = false; break; }
-        tc_fence_after();
-        issue_dq();
-        mma_commit(&bars->dq_full);
+        for (int h = 0; h < kDqParts && ok; ++h) {
+          const int hc = it * kDqParts + h;  // dQ product counter
+          if (hc > 0 && !mbar_wait(&bars->dq_empty, (hc - 1) & 1, wc, kSiteBwdDqEmpty)) { ok = false; break; }
+          tc_fence_after();
+          issue_dq(kTmDqPart, h);
+          mma_commit(&bars->dq_full);
+        }
+        if (!ok) break;
         mma_commit(&bars->t_empty[st]);
         if (in >= 0) {
+          // dP^T for the next tile overwrites dS^T (read by dK above, in issue order)
+          // and, at head dim 128, the dQ part columns: wait until they are read out.
           if (Cfg::kAlias) {
-            // dQ_i occupies half of the S^T / dP^T columns: wait until it has been read.
-            if (!mbar_wait(&bars->dq_empty, it & 1, wc, kSiteBwdDqEmpty)) { ok = false; break; }
-            if (!mbar_wait(&bars->t_full[stn], phn, wc, kSiteBwdTFull)) { ok = false; break; }
+            const int hc = it * kDqParts + kDqParts - 1;
+            if (!mbar_wait(&bars->dq_empty, hc & 1, wc, kSiteBwdDqEmpty)) { ok = false; break; }
             tc_fence_after();
-            issue_t(Cfg::kTmS, aK, aQ + stn * Cfg::kTileBytes);
-            mma_commit(&bars->s_full);
           }
           issue_t(Cfg::kTmDP, aV, aDO + stn * Cfg::kTileBytes);
           mma_commit(&bars->dp_full);
@@ -367,8 +384,20 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mma_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, wc, kSiteBwdDrain);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ compute warpgroup
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmCols);
+  } else if (warp < 4) {
+    // idle warps of the first warpgroup: they take part in its register hand-over
+    regs_dec<kBwdRegsCtl>();
+    __syncthreads();
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ compute warpgroups
+    regs_inc<kBwdRegsCompute>();
+    // Warpgroup h (0 or 1) handles query columns [64h, 64h + 64) of the key rows.
+    const int h = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row within tile j
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
@@ -387,38 +416,39 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      const float* lse = sL + st * 128;
-      const float* Dr = sDr + st * 128;
+      const float* lse = sL + st * 128 + h * 64;
+      const float* Dr = sDr + st * 128 + h * 64;
       const bool diag = CAUSAL && (i == j);  // query c visible to key r iff c >= r
-      // ---- P^T row r (query columns c = 0..127), packed bf16 pairs
-      uint32_t pk[64];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t raw[32];
-        tmem_ld32(trow + Cfg::kTmS + q4 * 32, raw);
+      // ---- P^T row r, query columns 64h + (0..63), packed bf16 pairs
+      uint32_t pk[32];
+      {
+        uint32_t raw[64];
+        tmem_ld32(trow + Cfg::kTmS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]));
+        tmem_ld32(trow + Cfg::kTmS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[32]));
         tmem_wait_ld();
+        // The packed P^T of query q goes to column q / 2: warpgroup 1 writes columns
+        // 32..63, which hold scores warpgroup 0 reads. Both finish reading first.
+        mbar_arrive(&bars->rd_s);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_s, it & 1, wc, kSiteBwdRead))) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-        for (int t4 = 0; t4 < 8; ++t4) {
-          const int c0 = q4 * 32 + 4 * t4;
+        for (int t4 = 0; t4 < 16; ++t4) {
+          const int c0 = 4 * t4;
           const float4 l4 = *reinterpret_cast<const float4*>(lse + c0);
           float pv[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float lu = u == 0 ? l4.x : u == 1 ? l4.y : u == 2 ? l4.z : l4.w;
-            pv[u] = ex2(fmaf(__uint_as_float(raw[4 * t4 + u]), sc, -lu) * kLog2e);
-            if (diag) pv[u] = (c0 + u < r) ? 0.f : pv[u];
+            pv[u] = ex2(fmaf(__uint_as_float(raw[c0 + u]), sc, -lu) * kLog2e);
+            if (diag) pv[u] = (h * 64 + c0 + u < r) ? 0.f : pv[u];
           }
-          pk[q4 * 16 + 2 * t4] = pack_bf16(pv[0], pv[1]);
-          pk[q4 * 16 + 2 * t4 + 1] = pack_bf16(pv[2], pv[3]);
+          pk[2 * t4] = pack_bf16(pv[0], pv[1]);
+          pk[2 * t4 + 1] = pack_bf16(pv[2], pv[3]);
         }
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) w[t] = pk[h * 32 + t];
-        tmem_st32(trow + Cfg::kTmS + h * 32, w);
-      }
+      tmem_st32(trow + Cfg::kTmS + h * 32, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_ready);
@@ -427,32 +457,39 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         ok = false;
         break;
       }
-      // The previous dQ MMA reads the shared dS buffer: wait for it to finish.
-      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, (it - 1) & 1, wc, kSiteBwdDqFull))) {
+      // The previous tile's dQ products read the shared dS buffer: wait for the last.
+      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, (it * kDqParts - 1) & 1, wc,
+                                                       kSiteBwdDqFull))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      uint32_t dpr[64];
+      tmem_ld32(trow + Cfg::kTmDP + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]));
+      tmem_ld32(trow + Cfg::kTmDP + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]));
+      tmem_wait_ld();
+      // dS^T (packed) overwrites dP^T columns that the other warpgroup reads.
+      mbar_arrive(&bars->rd_dp);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
+        ok = false;
+        break;
+      }
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t raw[32];
-        tmem_ld32(trow + Cfg::kTmDP + q4 * 32, raw);
-        tmem_wait_ld();
+      for (int q2 = 0; q2 < 2; ++q2) {
         uint32_t ds[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-          const int c0 = q4 * 32 + 2 * t;
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[q4 * 16 + t]));
+          const int c0 = q2 * 32 + 2 * t;
+          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[q2 * 16 + t]));
           const float2 dd = *reinterpret_cast<const float2*>(Dr + c0);
-          ds[t] = pack_bf16(pp.x * (__uint_as_float(raw[2 * t]) - dd.x), pp.y * (__uint_as_float(raw[2 * t + 1]) - dd.y));
+          ds[t] = pack_bf16(pp.x * (__uint_as_float(dpr[c0]) - dd.x), pp.y * (__uint_as_float(dpr[c0 + 1]) - dd.y));
         }
-        tmem_st16(trow + Cfg::kTmDP + q4 * 16, ds);
-        // Shared memory, M-major 128-byte swizzle: [q block of 64][key row][64 q].
+        tmem_st16(trow + Cfg::kTmDP + h * 32 + q2 * 16, ds);
+        // Shared memory, M-major 128-byte swizzle: [q block h][key row][64 q].
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          const int cq = q4 * 4 + ch;  // 16-byte chunk index along q (8 values)
-          const int mb = cq >> 3;
-          uint8_t* dst = sDS + mb * Cfg::kBlockBytes + r * 128 + (((cq & 7) ^ (r & 7)) << 4);
+          const int cq = q2 * 4 + ch;  // 16-byte chunk index (8 q values) within the block
+          uint8_t* dst = sDS + h * Cfg::kBlockBytes + r * 128 + ((cq ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(dst) = make_uint4(ds[4 * ch], ds[4 * ch + 1], ds[4 * ch + 2], ds[4 * ch + 3]);
         }
       }
@@ -461,93 +498,80 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(&bars->ds_ready);
     }
-    // ---------------------------------------------------------- epilogue: dK, dV
+    // ---------------------------------------------------------- epilogue: dK (h = 0), dV (h = 1)
     const size_t row = size_t(bh) * p.N + size_t(j) * 128 + r;
     if (ok) {
       const bool any = it > 0;
       if (any) ok = __all_sync(0xffffffffu, mbar_wait(&bars->acc_done, 0, wc, kSiteBwdAcc));
       if (ok) {
         tc_fence_after();
+        __nv_bfloat16* dst = (h == 0 ? p.dk : p.dv) + row * D;
+        const float mul = h == 0 ? sc : 1.f;
+        const uint32_t col = h == 0 ? Cfg::kTmDK : Cfg::kTmDV;
 #pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          __nv_bfloat16* dst = (which == 0 ? p.dk : p.dv) + row * D;
-          const float mul = which == 0 ? sc : 1.f;
-          const uint32_t col = which == 0 ? Cfg::kTmDK : Cfg::kTmDV;
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          if (any) {
+            tmem_ld32(trow + col + cc * 32, v);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t v[32];
-            if (any) {
-              tmem_ld32(trow + col + cc * 32, v);
-              tmem_wait_ld();
-            } else {
-#pragma unroll
-              for (int t = 0; t < 32; ++t) v[t] = 0u;
-            }
-            uint4 o4[4];
-            uint32_t* w = reinterpret_cast<uint32_t*>(o4);
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-              w[t] = pack_bf16(__uint_as_float(v[2 * t]) * mul, __uint_as_float(v[2 * t + 1]) * mul);
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) d4[t] = o4[t];
+            for (int t = 0; t < 32; ++t) v[t] = 0u;
           }
+          uint4 o4[4];
+          uint32_t* w = reinterpret_cast<uint32_t*>(o4);
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            w[t] = pack_bf16(__uint_as_float(v[2 * t]) * mul, __uint_as_float(v[2 * t + 1]) * mul);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) d4[t] = o4[t];
         }
       }
     }
-  } else if (warp >= 8) {
+    tc_fence_before();
+    __syncthreads();
+  } else {
     // ------------------------------------------------------------ dQ warpgroup
+    regs_dec<kBwdRegsDq>();
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row within tile i
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
+    constexpr uint32_t kTmDqPart = Cfg::kAlias ? Cfg::kTmDP + 64 : Cfg::kTmDQ;
     int it = 0;
-    for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, it & 1, wc, kSiteBwdDqFull))) break;
-      tc_fence_after();
+    bool ok = true;
+    for (int i = sch.first(); i >= 0 && ok; i = sch.next(i), ++it) {
       float4* dst = reinterpret_cast<float4*>(p.dqacc + (size_t(bh) * p.N + size_t(i) * 128 + r) * D);
-      uint32_t v[D];
-      if (Cfg::kAlias) {
-        uint32_t a[32], b[32], c[32], d[32];
-        tmem_ld32(trow + Cfg::kTmS + 64, a);
-        tmem_ld32(trow + Cfg::kTmS + 96, b);
-        tmem_ld32(trow + Cfg::kTmDP + 64, c);
-        tmem_ld32(trow + Cfg::kTmDP + 96, d);
-        tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          v[t] = a[t];
-          v[32 + t] = b[t];
-          v[64 + t] = c[t];
-          v[96 + t] = d[t];
+      for (int h = 0; h < kDqParts; ++h) {
+        const int hc = it * kDqParts + h;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, hc & 1, wc, kSiteBwdDqFull))) {
+          ok = false;
+          break;
         }
-      } else {
+        tc_fence_after();
         uint32_t a[32], b[32];
-        tmem_ld32(trow + Cfg::kTmDQ, a);
-        tmem_ld32(trow + Cfg::kTmDQ + 32, b);
+        tmem_ld32(trow + kTmDqPart, a);
+        tmem_ld32(trow + kTmDqPart + 32, b);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->dq_empty);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          v[t] = a[t];
-          v[32 + t] = b[t];
-        }
+        for (int t = 0; t < 8; ++t)
+          atomicAdd(dst + h * 16 + t, make_float4(__uint_as_float(a[4 * t]), __uint_as_float(a[4 * t + 1]),
+                                                  __uint_as_float(a[4 * t + 2]), __uint_as_float(a[4 * t + 3])));
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          atomicAdd(dst + h * 16 + 8 + t, make_float4(__uint_as_float(b[4 * t]), __uint_as_float(b[4 * t + 1]),
+                                                      __uint_as_float(b[4 * t + 2]), __uint_as_float(b[4 * t + 3])));
       }
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
-#pragma unroll
-      for (int t = 0; t < D / 4; ++t)
-        atomicAdd(dst + t, make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
-                                       __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
     }
+    tc_fence_before();
+    __syncthreads();
   }
-
-  // ---------------------------------------------------------------- teardown
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, Cfg::kTmCols);
-  }
+  // Teardown: every role ends with its own CTA barrier (there is no common tail,
+  // so the warpgroups keep their register budgets to the end); warp 1 then frees
+  // TMEM. Only the compute warpgroups ever raise their budget, and only once, by
+  // exactly what the other two warpgroups released: no increase can be starved.
 }
 
 }  // namespace fa

@@ -66,7 +66,7 @@ struct WaitCtl {
   uint64_t timeout_ns;   // per-wait limit
 };
 
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int site,
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int site,
                                             bool honour_abort) {
   const uint64_t t0 = global_ns();
   while (true) {
@@ -266,6 +266,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// Per-warpgroup register budget (all warps of the warpgroup execute the same one).
+// The increases must fit in what the decreases of other warpgroups release: the
+// pool is the launch register count times the block size.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------------ math helpers
