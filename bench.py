@@ -300,7 +300,7 @@ def run_ours(args, wl_name, wl):
         step_flops += 3.5 * f
 
     def one_step(ev=None):
-        # ev: dict label -> list of 5 events [start, after fwd, after pre, after main, after convert]
+        # ev: dict label -> 5 events [start, after fwd, after pre, after dK/dV, after dQ]
         for (label, causal, _) in wl["variants"]:
             k = kinds[label]
             x = outs[label]
@@ -313,14 +313,14 @@ def run_ours(args, wl_name, wl):
                 fa.forward_blocksparse(t["q"], t["k"], t["v"], k["mask"], scale=sc, out=x["o"], lse=x["lse"])
             if e:
                 e[1].record(stream)
-            fa.bwd_preprocess(x["o"], t["do"], ws)
+            fa.bwd_preprocess(x["o"], t["do"], x["lse"], ws)
             if e:
                 e[2].record(stream)
-            fa.bwd_main(t["q"], t["k"], t["v"], x["lse"], t["do"], x["dk"], x["dv"], ws, causal=causal, scale=sc,
+            fa.bwd_dkdv(t["q"], t["k"], t["v"], t["do"], x["dk"], x["dv"], ws, causal=causal, scale=sc,
                         tile_mask=k["mask"])
             if e:
                 e[3].record(stream)
-            fa.bwd_dq_convert(ws, x["dq"], scale=sc)
+            fa.bwd_dq(t["q"], t["k"], t["v"], t["do"], x["dq"], ws, causal=causal, scale=sc, tile_mask=k["mask"])
             if e:
                 e[4].record(stream)
 
@@ -353,7 +353,7 @@ def run_ours(args, wl_name, wl):
         raise SystemExit(f"device status {st} (site {dt}) in the timed region")
 
     # per-kernel and per-step device times (ms)
-    per = {label: dict(fwd=0.0, pre=0.0, main=0.0, conv=0.0) for (label, _, _) in wl["variants"]}
+    per = {label: dict(fwd=0.0, pre=0.0, dkdv=0.0, dq=0.0) for (label, _, _) in wl["variants"]}
     step_ms = []
     for s in range(args.steps):
         tot = 0.0
@@ -362,8 +362,8 @@ def run_ours(args, wl_name, wl):
             a = [e[i].elapsed_time(e[i + 1]) for i in range(4)]
             per[label]["fwd"] += a[0]
             per[label]["pre"] += a[1]
-            per[label]["main"] += a[2]
-            per[label]["conv"] += a[3]
+            per[label]["dkdv"] += a[2]
+            per[label]["dq"] += a[3]
             tot += sum(a)
         step_ms.append(tot)
     total_ms = sum(step_ms)
@@ -380,26 +380,27 @@ def run_ours(args, wl_name, wl):
     peak_label = ("sustained" if sustained else "burst") + f" bf16, {pk_kind}"
 
     breakdown = {}
-    main_flops, main_ms = 0.0, 0.0
+    dkdv_flops, dkdv_ms = 0.0, 0.0
     for (label, _, _) in wl["variants"]:
         k = kinds[label]
         p = {kk: v / K for kk, v in per[label].items()}
-        bwd_ms = p["pre"] + p["main"] + p["conv"]
+        bwd_ms = p["pre"] + p["dkdv"] + p["dq"]
         breakdown[label] = {
             "fwd_ms": round(p["fwd"], 4), "bwd_ms": round(bwd_ms, 4),
-            "bwd_main_ms": round(p["main"], 4), "bwd_pre_ms": round(p["pre"], 4), "bwd_convert_ms": round(p["conv"], 4),
+            "bwd_pre_ms": round(p["pre"], 4), "bwd_dkdv_ms": round(p["dkdv"], 4), "bwd_dq_ms": round(p["dq"], 4),
             "fwd_tflops": round(k["fwd"] / (p["fwd"] * 1e-3) / 1e12, 2),
             "bwd_tflops": round(k["bwd"] / (bwd_ms * 1e-3) / 1e12, 2),
             "fwd_bwd_tflops": round(3.5 * k["fwd"] / ((p["fwd"] + bwd_ms) * 1e-3) / 1e12, 2),
             "fwd_pct_peak": round(100 * k["fwd"] / (p["fwd"] * 1e-3) / 1e12 / peak, 1),
             "bwd_pct_peak": round(100 * k["bwd"] / (bwd_ms * 1e-3) / 1e12 / peak, 1),
         }
-        main_flops += k["bwd"]
-        main_ms += p["main"]
-    achieved = main_flops / (main_ms * 1e-3) / 1e12
-    roofline = {"kernel": "fa_bwd_kernel (backward main)", "bound": "tensor", "achieved": round(achieved, 2),
-                "peak": peak, "peak_kind": peak_label, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": profiled_traffic("fa_bwd_kernel", wl_name)}
+        # dK/dV kernel: S^T, dP^T, dV, dK = four N x N x d products = 2x the forward count
+        dkdv_flops += 2.0 * k["fwd"]
+        dkdv_ms += p["dkdv"]
+    achieved = dkdv_flops / (dkdv_ms * 1e-3) / 1e12
+    roofline = {"kernel": "fa_bwd_dkdv_kernel (backward dK/dV, 4 products per tile pair)", "bound": "tensor",
+                "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_label, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("fa_bwd_dkdv_kernel", wl_name)}
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e_steps = max(3, min(K, 10))
@@ -448,7 +449,7 @@ def run_ours(args, wl_name, wl):
         "data": "synthetic (seeded N(0,1) inputs rounded to bf16; per-rank seeds)",
         "config": {"workload": wl_name, "B": B, "H": H, "N": N, "d": d,
                    "variants": [v[0] for v in wl["variants"]],
-                   "step": "per variant: forward, backward pre-pass, backward main, dQ convert",
+                   "step": "per variant: forward, backward pre-pass, backward dK/dV, backward dQ",
                    "l2": "flushed before every timed step (256 MiB write, outside the step events)",
                    "parallelism": f"replicas x{world} (independent (batch, head) shards, no collective)"},
         "pct_of_peak": round(100 * value / world / peak, 2),
@@ -514,14 +515,13 @@ def run_table(args):
                     fa.forward_blocksparse(t["q"], t["k"], t["v"], mask, scale=sc, out=o, lse=lse)
 
             def pre():
-                fa.bwd_preprocess(o, t["do"], ws)
+                fa.bwd_preprocess(o, t["do"], lse, ws)
 
-            def main():
-                fa.bwd_main(t["q"], t["k"], t["v"], lse, t["do"], dk, dv, ws, causal=causal, scale=sc,
-                            tile_mask=mask)
+            def dkdv():
+                fa.bwd_dkdv(t["q"], t["k"], t["v"], t["do"], dk, dv, ws, causal=causal, scale=sc, tile_mask=mask)
 
-            def conv():
-                fa.bwd_dq_convert(ws, dq, scale=sc)
+            def dqk():
+                fa.bwd_dq(t["q"], t["k"], t["v"], t["do"], dq, ws, causal=causal, scale=sc, tile_mask=mask)
 
             def timed(fns):
                 ms = []
@@ -543,11 +543,13 @@ def run_table(args):
                    "fwd_pct_peak": round(100 * F / t_f / 1e9 / pk["bf16_tflops"], 1)}
             if name != "pr1":
                 pre()
-                t_m = timed([main])
-                t_b = timed([pre, main, conv])
-                row.update({"bwd_ms": round(t_b, 4), "bwd_main_ms": round(t_m, 4),
+                t_kv = timed([dkdv])
+                t_q = timed([dqk])
+                t_b = timed([pre, dkdv, dqk])
+                row.update({"bwd_ms": round(t_b, 4), "bwd_dkdv_ms": round(t_kv, 4), "bwd_dq_ms": round(t_q, 4),
                             "bwd_tflops": round(2.5 * F / t_b / 1e9, 1),
-                            "bwd_main_tflops": round(2.5 * F / t_m / 1e9, 1),
+                            "dkdv_tflops": round(2.0 * F / t_kv / 1e9, 1),
+                            "dq_exec_tflops": round(1.5 * F / t_q / 1e9, 1),
                             "bwd_pct_peak": round(100 * 2.5 * F / t_b / 1e9 / pk["bf16_tflops"], 1),
                             "fwd_bwd_tflops": round(3.5 * F / (t_f + t_b) / 1e9, 1)})
             st, site = fa.device_status(dev)

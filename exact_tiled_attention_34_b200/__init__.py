@@ -22,8 +22,8 @@ import re
 
 __all__ = [
     "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
-    "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_main",
-    "bwd_dq_convert",
+    "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_dkdv",
+    "bwd_dq",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -56,9 +56,9 @@ _SIGS = {
     "fa_bwd": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_blocksparse": ([_vp] * 10 + [_sz, _vp, _i] + [_i] * 4 + [_f, _vp], _i),
     "fa_device_status": ([_vp, ctypes.POINTER(_i)], _i),
-    "fa_bwd_preprocess": ([_vp] * 3 + [_sz] + [_i] * 4 + [_vp], _i),
-    "fa_bwd_main": ([_vp] * 8 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
-    "fa_bwd_dq_convert": ([_vp, _sz, _vp] + [_i] * 4 + [_f, _vp], _i),
+    "fa_bwd_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
+    "fa_bwd_dkdv": ([_vp] * 7 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_dq": ([_vp] * 6 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
 }
 
 
@@ -214,30 +214,32 @@ def device_status(device=None):
 # ---------------------------------------------------------------- staged backward
 # The three launches of ``backward`` as separate calls (same workspace for all three).
 
-def bwd_preprocess(o, do, workspace):
+def bwd_preprocess(o, do, lse, workspace):
     import torch
     B, H, N, d = o.shape
     with torch.cuda.device(o.device):
-        st = lib().fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                                     B, H, N, d, _stream_ptr(o.device))
+        st = lib().fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel(), B, H, N, d, _stream_ptr(o.device))
     _check(st, "fa_bwd_preprocess")
 
 
-def bwd_main(q, k, v, lse, do, dk, dv, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
+def bwd_dkdv(q, k, v, do, dk, dv, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
     import torch
     B, H, N, d = q.shape
     with torch.cuda.device(q.device):
-        st = lib().fa_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                               dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        st = lib().fa_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                None if tile_mask is None else tile_mask.data_ptr(), mask_block,
                                B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
-    _check(st, "fa_bwd_main")
+    _check(st, "fa_bwd_dkdv")
 
 
-def bwd_dq_convert(workspace, dq, scale=None):
+def bwd_dq(q, k, v, do, dq, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
     import torch
-    B, H, N, d = dq.shape
-    with torch.cuda.device(dq.device):
-        st = lib().fa_bwd_dq_convert(workspace.data_ptr(), workspace.numel(), dq.data_ptr(), B, H, N, d,
-                                     _scale(scale, d), _stream_ptr(dq.device))
-    _check(st, "fa_bwd_dq_convert")
+    B, H, N, d = q.shape
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_dq(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dq.data_ptr(),
+                             workspace.data_ptr(), workspace.numel(),
+                             None if tile_mask is None else tile_mask.data_ptr(), mask_block,
+                             B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_bwd_dq")

@@ -166,23 +166,22 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace: fp32 D rows [BH*N], then fp32 lse*log2(e) rows [BH*N], each 256-aligned.
 size_t bwd_ws_bytes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
   const size_t rows = size_t(B) * H * N;
-  return round256(rows * d * 4) + round256(rows * 4);
+  return 2 * round256(rows * 4);
 }
 
-template <int D, bool CAUSAL, bool SPARSE>
-fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          const CUtensorMap& mdo, const fa::BwdParams& p, cudaStream_t stream) {
-  static std::once_flag flags[kMaxDevices];
-  static cudaError_t errs[kMaxDevices];
-  auto kernel = fa::fa_bwd_kernel<D, CAUSAL, SPARSE>;
-  constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
+// Launch one of the two 384-thread backward kernels. They re-divide their register
+// pool between warpgroups; refuse to launch if the build gave them fewer registers
+// per thread than that split needs.
+template <typename K>
+fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk,
+                            const CUtensorMap& mv, const CUtensorMap& mdo, const fa::BwdParams& p,
+                            cudaStream_t stream, std::once_flag (&flags)[kMaxDevices],
+                            cudaError_t (&errs)[kMaxDevices], int (&regs)[kMaxDevices]) {
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
-  // The kernel re-divides its register pool between warpgroups; that is only valid
-  // if it was built with exactly the register count the split assumes.
-  static int regs[kMaxDevices];
   int dev;
   if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
   if (regs[dev] == 0) {
@@ -190,21 +189,40 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
     if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
     regs[dev] = attr.numRegs;
   }
-  if (regs[dev] != fa::kBwdLaunchRegs) return FA_ERR_UNSUPPORTED;
-  const unsigned grid = unsigned(p.n_tiles) * unsigned(p.BH);
-  kernel<<<grid, 512, smem, stream>>>(mq, mk, mv, mdo, p);
+  if (regs[dev] * fa::kBwdThreads < fa::kBwdRegsNeeded) return FA_ERR_UNSUPPORTED;
+  kernel<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+fa_status launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                      const fa::BwdParams& p, cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  static int regs[kMaxDevices];
+  return launch_bwd_kernel(fa::fa_bwd_dkdv_kernel<D, CAUSAL, SPARSE>, fa::BwdCfg<D>::kSmemBytes,
+                           unsigned(p.n_tiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+fa_status launch_dq(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                    const fa::BwdParams& p, cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  static int regs[kMaxDevices];
+  return launch_bwd_kernel(fa::fa_bwd_dq_kernel<D, CAUSAL, SPARSE>, fa::BwdCfg<D>::kQSmemBytes,
+                           unsigned(p.n_tiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
 }
 
 struct BwdArgs {
   int BH;
   size_t rows;
-  float* dqacc;
   float* Drow;
+  float* lse2;
 };
 
 // Checks shared by the backward stages; fills the workspace views.
-fa_status bwd_check(void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a) {
+fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a) {
   fa_status s;
   if (ws == nullptr) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FA_ERR_ALIGNMENT;
@@ -212,15 +230,15 @@ fa_status bwd_check(void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdAr
   if (ws_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
   a->BH = B * H;
   a->rows = size_t(a->BH) * N;
-  a->dqacc = static_cast<float*>(ws);
-  a->Drow = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round256(a->rows * d * 4));
+  a->Drow = static_cast<float*>(const_cast<void*>(ws));
+  a->lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(const_cast<void*>(ws)) + round256(a->rows * 4));
   return FA_OK;
 }
 
-fa_status bwd_pre(const void* o, const void* dO, void* ws, size_t ws_bytes, int B, int H, int N, int d,
-                  void* stream) {
+fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, size_t ws_bytes, int B, int H, int N,
+                  int d, void* stream) {
   fa_status s;
-  if ((s = check_ptrs({o, dO})) != FA_OK) return s;
+  if ((s = check_ptrs({o, dO, lse})) != FA_OK) return s;
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -229,17 +247,21 @@ fa_status bwd_pre(const void* o, const void* dO, void* ws, size_t ws_bytes, int 
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   if (d == 64)
-    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, a.Drow, a.dqacc, static_cast<long long>(a.rows));
+    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, static_cast<long long>(a.rows));
   else
-    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, a.Drow, a.dqacc, static_cast<long long>(a.rows));
+    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, static_cast<long long>(a.rows));
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
-                   void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H, int N,
-                   int d, int causal, float scale, void* stream) {
+enum class BwdStage { kDkdv, kDq };
+
+// dK/dV (stage kDkdv: dk, dv written) or dQ (stage kDq: dq written).
+fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v, const void* dO, void* out0,
+                    void* out1, const void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H,
+                    int N, int d, int causal, float scale, void* stream) {
   fa_status s;
-  if ((s = check_ptrs({q, k, v, lse, dO, dk, dv})) != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, dO, out0})) != FA_OK) return s;
+  if (stage == BwdStage::kDkdv && (s = check_ptrs({out1})) != FA_OK) return s;
   if (mask != nullptr && (mask_block != 128 || causal)) return FA_ERR_UNSUPPORTED;
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
@@ -254,11 +276,11 @@ fa_status bwd_main(const void* q, const void* k, const void* v, const float* lse
   if ((s = make_map(&mdo, dO, a.BH, N, d, 128)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fa::BwdParams p;
-  p.lse = lse;
+  p.lse2 = a.lse2;
   p.Drow = a.Drow;
-  p.dqacc = a.dqacc;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq = stage == BwdStage::kDq ? static_cast<__nv_bfloat16*>(out0) : nullptr;
+  p.dk = stage == BwdStage::kDkdv ? static_cast<__nv_bfloat16*>(out0) : nullptr;
+  p.dv = stage == BwdStage::kDkdv ? static_cast<__nv_bfloat16*>(out1) : nullptr;
   p.tile_mask = mask;
   p.status = status;
   p.timeout_ns = kTimeoutNs;
@@ -266,29 +288,20 @@ fa_status bwd_main(const void* q, const void* k, const void* v, const float* lse
   p.BH = a.BH;
   p.n_tiles = N / 128;
   p.scale = scale;
-  if (mask)
-    return d == 64 ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, st)
-                   : launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, st);
-  if (causal)
-    return d == 64 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, st)
-                   : launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, st);
-  return d == 64 ? launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, st)
-                 : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, st);
-}
-
-fa_status bwd_convert(const void* ws, size_t ws_bytes, void* dq, int B, int H, int N, int d, float scale,
-                      void* stream) {
-  fa_status s;
-  if ((s = check_ptrs({dq})) != FA_OK) return s;
-  BwdArgs a;
-  if ((s = bwd_check(const_cast<void*>(ws), ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
-  if ((s = check_scale(scale)) != FA_OK) return s;
-  const long long n4 = static_cast<long long>(a.rows) * d / 4;
-  const long long want = (n4 + 255) / 256;
-  const unsigned grid = unsigned(want < 148LL * 16 ? want : 148LL * 16);
-  fa::fa_bwd_dq_convert_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const float4*>(a.dqacc), static_cast<uint2*>(dq), scale, n4);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+#define FA_BWD_DISPATCH(LAUNCH)                                                                  \
+  if (mask)                                                                                      \
+    return d == 64 ? LAUNCH<64, false, true>(mq, mk, mv, mdo, p, st)                             \
+                   : LAUNCH<128, false, true>(mq, mk, mv, mdo, p, st);                           \
+  if (causal)                                                                                    \
+    return d == 64 ? LAUNCH<64, true, false>(mq, mk, mv, mdo, p, st)                             \
+                   : LAUNCH<128, true, false>(mq, mk, mv, mdo, p, st);                           \
+  return d == 64 ? LAUNCH<64, false, false>(mq, mk, mv, mdo, p, st)                              \
+                 : LAUNCH<128, false, false>(mq, mk, mv, mdo, p, st);
+  if (stage == BwdStage::kDkdv) {
+    FA_BWD_DISPATCH(launch_dkdv)
+  }
+  FA_BWD_DISPATCH(launch_dq)
+#undef FA_BWD_DISPATCH
 }
 
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -300,10 +313,12 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
   if ((s = check_scale(scale)) != FA_OK) return s;
-  if ((s = bwd_pre(o, dO, ws, ws_bytes, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = bwd_main(q, k, v, lse, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, d, causal, scale, stream)) != FA_OK)
+  if ((s = bwd_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, d, causal, scale,
+                     stream)) != FA_OK)
     return s;
-  return bwd_convert(ws, ws_bytes, dq, B, H, N, d, scale, stream);
+  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, ws, ws_bytes, mask, 128, B, H, N, d, causal, scale,
+                   stream);
 }
 
 }  // namespace
@@ -364,21 +379,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                     scale, stream);
 }
 
-fa_status fa_bwd_preprocess(const void* o, const void* dO, void* workspace, size_t workspace_bytes, int B, int H,
-                            int N, int d, void* stream) {
-  return bwd_pre(o, dO, workspace, workspace_bytes, B, H, N, d, stream);
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace,
+                            size_t workspace_bytes, int B, int H, int N, int d, void* stream) {
+  return bwd_pre(o, dO, lse, workspace, workspace_bytes, B, H, N, d, stream);
 }
 
-fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
-                      void* dv, void* workspace, size_t workspace_bytes, const uint8_t* tile_mask, int mask_block,
-                      int B, int H, int N, int d, int causal, float scale, void* stream) {
-  return bwd_main(q, k, v, lse, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N, d,
-                  causal != 0, scale, stream);
+fa_status fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                      const void* workspace, size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B,
+                      int H, int N, int d, int causal, float scale, void* stream) {
+  return bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N,
+                   d, causal != 0, scale, stream);
 }
 
-fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void* dq, int B, int H, int N, int d,
-                            float scale, void* stream) {
-  return bwd_convert(workspace, workspace_bytes, dq, B, H, N, d, scale, stream);
+fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, const void* workspace,
+                    size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B, int H, int N, int d,
+                    int causal, float scale, void* stream) {
+  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, workspace, workspace_bytes, tile_mask, mask_block, B, H,
+                   N, d, causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -440,12 +457,13 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
   if (need > size_t(FA_BWD_NOALLOC_SCRATCH_BYTES)) return FA_ERR_WORKSPACE;
   void* scratch;
   if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
-  // The pre-pass zeroes the dQ accumulator and rewrites D, so whatever an earlier
-  // call left in the array does not matter.
+  // The pre-pass rewrites every row the other two launches read, so whatever an
+  // earlier call left in the array does not matter.
   const size_t bytes = size_t(FA_BWD_NOALLOC_SCRATCH_BYTES);
-  if ((s = bwd_pre(o, dO, scratch, bytes, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = bwd_main(q, k, v, lse, dO, dk, dv, scratch, bytes, tile_mask, mask_block, B, H, N, d, causal, scale,
-                    stream)) != FA_OK)
+  if ((s = bwd_pre(o, dO, lse, scratch, bytes, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, scratch, bytes, tile_mask, mask_block, B, H, N, d,
+                     causal, scale, stream)) != FA_OK)
     return s;
-  return bwd_convert(scratch, bytes, dq, B, H, N, d, scale, stream);
+  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, scratch, bytes, tile_mask, mask_block, B, H, N, d, causal,
+                   scale, stream);
 }

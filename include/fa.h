@@ -94,9 +94,8 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
 
 /*
  * Bytes of device scratch that fa_bwd / fa_bwd_blocksparse need for these sizes:
- * an fp32 [B,H,N,d] dQ accumulator plus the fp32 [B,H,N] row terms
- * D_i = sum_c dO_ic O_ic, each rounded up to 256 bytes. Returns 0 for
- * non-positive sizes.
+ * two fp32 [B,H,N] row arrays (D_i = sum_c dO_ic O_ic, and lse_i * log2 e), each
+ * rounded up to 256 bytes. Returns 0 for non-positive sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -111,8 +110,9 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *   workspace       : device scratch of at least fa_bwd_workspace_bytes(B,H,N,d)
  *                     bytes, 256-byte aligned; its contents on entry do not
  *                     matter; it must not be shared with a concurrent call.
- * dq is accumulated with fp32 atomic adds across key tiles, so its summation
- * order (and last bits) may differ from run to run; dk and dv are deterministic.
+ * All three gradients are deterministic (no atomics): dk and dv come from one pass
+ * over the query tiles per key tile, dq from one pass over the key tiles per query
+ * tile (which recomputes the scores and dP it needs).
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dO, void* dq, void* dk, void* dv,
@@ -129,25 +129,26 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
 /*
  * The three launches that make up fa_bwd / fa_bwd_blocksparse, for callers that
  * schedule or time them separately. On one stream,
- *   fa_bwd_preprocess; fa_bwd_main; fa_bwd_dq_convert
+ *   fa_bwd_preprocess; fa_bwd_dkdv; fa_bwd_dq
  * is exactly fa_bwd (tile_mask = NULL) or fa_bwd_blocksparse (tile_mask set).
  * Arguments have the meanings given for fa_bwd; the workspace must be the same
- * buffer for all three.
- *   fa_bwd_preprocess : D_i = sum_c dO_ic O_ic into the workspace, and the fp32
- *                       dQ accumulator in the workspace set to zero.
- *   fa_bwd_main       : dk, dv, and dQ products added into the accumulator.
- *                       tile_mask may be NULL (then `causal` applies) or a block
- *                       mask (then causal must be 0 and mask_block 128).
- *   fa_bwd_dq_convert : dq = bf16(scale * accumulator).
+ * buffer for all three. fa_bwd_dkdv and fa_bwd_dq only read the workspace and may
+ * run in either order (or concurrently) after fa_bwd_preprocess.
+ *   fa_bwd_preprocess : D_i = sum_c dO_ic O_ic and lse_i log2(e) into the workspace.
+ *   fa_bwd_dkdv       : dk and dv. tile_mask may be NULL (then `causal` applies)
+ *                       or a block mask (then causal must be 0, mask_block 128).
+ *   fa_bwd_dq         : dq (same mask rules).
  */
-fa_status fa_bwd_preprocess(const void* o, const void* dO, void* workspace, size_t workspace_bytes,
-                            int B, int H, int N, int d, void* stream);
-fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO,
-                      void* dk, void* dv, void* workspace, size_t workspace_bytes,
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace,
+                            size_t workspace_bytes, int B, int H, int N, int d, void* stream);
+fa_status fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                      const void* workspace, size_t workspace_bytes,
                       const uint8_t* tile_mask, int mask_block,
                       int B, int H, int N, int d, int causal, float scale, void* stream);
-fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void* dq,
-                            int B, int H, int N, int d, float scale, void* stream);
+fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq,
+                    const void* workspace, size_t workspace_bytes,
+                    const uint8_t* tile_mask, int mask_block,
+                    int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
  * Backward without caller-provided scratch (no counterpart on the pages: this is
@@ -158,12 +159,12 @@ fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void*
  * input and output buffers, or a latency-critical loop that must not pay the
  * implicit device synchronisation of cudaMalloc/cudaFree. Same arguments and
  * results as fa_bwd / fa_bwd_blocksparse (tile_mask NULL or a 128-granular block
- * mask with causal = 0), but the fp32 scratch (dQ accumulator and D rows) lives in
- * one array compiled into the library: FA_BWD_NOALLOC_SCRATCH_BYTES bytes of device
+ * mask with causal = 0), but the fp32 scratch (two per-row arrays) lives in one
+ * array compiled into the library: FA_BWD_NOALLOC_SCRATCH_BYTES bytes of device
  * memory on every GPU that loads the library, held until the process exits.
- *  - Sizes: needs fa_bwd_workspace_bytes(B,H,N,d) <= FA_BWD_NOALLOC_SCRATCH_BYTES
- *    (e.g. B*H*N <= 129,024 rows at d = 64, <= 65,024 at d = 128); larger sizes
- *    return FA_ERR_WORKSPACE and enqueue nothing.
+ *  - Sizes: needs fa_bwd_workspace_bytes(B,H,N,d) <= FA_BWD_NOALLOC_SCRATCH_BYTES,
+ *    i.e. B*H*N <= 1,048,576 rows (any d); larger sizes return FA_ERR_WORKSPACE
+ *    and enqueue nothing.
  *  - Allocation: none. No cudaMalloc, cudaFree or allocating library call.
  *  - Set-up: the first call on a device (with that device current) looks up the
  *    array's device address once; make that first call before any stream
@@ -173,7 +174,7 @@ fa_status fa_bwd_dq_convert(const void* workspace, size_t workspace_bytes, void*
  *    the GPU (different streams, or several threads) race on the array: serialise
  *    them (e.g. one stream).
  */
-#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                          const void* dO, void* dq, void* dk, void* dv,
                          const uint8_t* tile_mask, int mask_block,

@@ -15,7 +15,7 @@ import exact_tiled_attention_34_b200 as fa
 from exact_tiled_attention_34_b200.inputs import make_qkv, make_tile_mask
 from tests.parity import assert_grad_close, f64
 
-SCRATCH_BYTES = 32 * 1024 * 1024  # FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h
+SCRATCH_BYTES = 8 * 1024 * 1024  # FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h
 
 
 def _noalloc_fn():
@@ -40,10 +40,11 @@ def _call(fn, t, o, lse, grads, mask, causal, scale):
 def test_oversized_request_is_rejected_without_touching_the_gpu():
     fn = _noalloc_fn()
     a = 1 << 20  # aligned stand-in addresses; the size check comes first
-    # d = 64: 129,024 rows fit, 129,152 do not; d = 128: 65,024 fit, 65,152 do not.
-    assert fa.lib().fa_bwd_workspace_bytes(1, 1, 129152, 64) > SCRATCH_BYTES
-    assert fn(a, a, a, a, a, a, a, a, a, None, 128, 1, 1, 129152, 64, 0, 0.125, None) == 4
-    assert fn(a, a, a, a, a, a, a, a, a, None, 128, 1, 1, 65152, 128, 1, 0.125, None) == 4
+    # B*H*N = 1,048,576 rows fit (any d); 1,048,704 do not.
+    assert fa.lib().fa_bwd_workspace_bytes(1, 16, 65536, 64) <= SCRATCH_BYTES
+    assert fa.lib().fa_bwd_workspace_bytes(1, 1, 1048704, 64) > SCRATCH_BYTES
+    assert fn(a, a, a, a, a, a, a, a, a, None, 128, 1, 1, 1048704, 64, 0, 0.125, None) == 4
+    assert fn(a, a, a, a, a, a, a, a, a, None, 128, 3, 1, 349568, 128, 1, 0.125, None) == 4
     assert fn(None, a, a, a, a, a, a, a, a, None, 128, 1, 1, 128, 64, 0, 0.125, None) == 1
     assert fn(a, a, a, a, a, a, a, a, a, a, 64, 1, 1, 128, 64, 0, 0.125, None) == 2
 
