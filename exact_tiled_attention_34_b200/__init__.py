@@ -59,6 +59,7 @@ _SIGS = {
     "fa_bwd_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
     "fa_bwd_dkdv": ([_vp] * 7 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_dq": ([_vp] * 6 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
+    "fa_debug_exp2": ([_vp, _vp, _i, _i, _vp], _i),
 }
 
 
@@ -243,3 +244,16 @@ def bwd_dq(q, k, v, do, dq, workspace, causal=False, scale=None, tile_mask=None,
                              None if tile_mask is None else tile_mask.data_ptr(), mask_block,
                              B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
     _check(st, "fa_bwd_dq")
+
+
+def debug_exp2(x, mode: int):
+    """2^x on the device through one of the kernels' two exponential paths
+    (0: special-function unit, 1: the library's polynomial). x: fp32 CUDA tensor."""
+    import torch
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        st = lib().fa_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), mode, _stream_ptr(x.device))
+    _check(st, "fa_debug_exp2")
+    return y

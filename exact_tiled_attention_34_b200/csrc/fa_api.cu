@@ -120,9 +120,20 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                      cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
+  static int regs[kMaxDevices];
   auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE>;
   constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  // The kernel re-divides its register pool between warpgroups: refuse to launch a
+  // build that gave it fewer registers per thread than the split needs.
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  if (regs[dev] == 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+    regs[dev] = attr.numRegs;
+  }
+  if (regs[dev] * fa::FwdCfg<D>::kThreads < fa::kFwdRegsNeeded) return FA_ERR_UNSUPPORTED;
   const unsigned grid = unsigned(p.n_qblocks) * unsigned(p.BH);
   kernel<<<grid, fa::FwdCfg<D>::kThreads, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -321,9 +332,28 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
                    stream);
 }
 
+__global__ void fa_debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int mode) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  const uint64_t v = fa::f2(a, b);
+  const float2 r = fa::f2_split(mode == 1 ? fa::ex2_poly_x2(v) : fa::ex2_mufu_x2(v));
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
+
 }  // namespace
 
 extern "C" {
+
+fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, void* stream) {
+  if (n < 0 || (mode != 0 && mode != 1)) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (x == nullptr || y == nullptr) return FA_ERR_INVALID_ARG;
+  const int pairs = (n + 1) / 2;
+  fa_debug_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 const char* fa_status_string(fa_status s) {
   switch (s) {

@@ -11,7 +11,7 @@
 // (P enters dV and dS rounded to bf16, as it enters the tensor-core products.)
 //
 // Three launches, all deterministic (no atomics):
-//  1. fa_bwd_pre_kernel: D and lse * log2(e) into the workspace.
+//  1. fa_bwd_pre_kernel: D and -lse * log2(e) into the workspace.
 //  2. fa_bwd_dkdv_kernel: one CTA per (128-key tile j, batch*head), looping over the
 //     query tiles i that see tile j (causal: i >= j; block-sparse: mask[i][j] = 1).
 //     The transposed products put key rows on TMEM lanes:
@@ -39,7 +39,8 @@ namespace fa {
 
 // ---------------------------------------------------------------- pre-processing
 
-// D[row] = sum_c dO[row, c] O[row, c] and lse2[row] = lse[row] log2(e) (fp32).
+// D[row] = sum_c dO[row, c] O[row, c] and nl2[row] = -lse[row] log2(e) (fp32), so
+// that the exponent of the recomputed P is one fused multiply-add: s c + nl2.
 // D / 8 threads per row, 16 bytes each.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
@@ -69,14 +70,14 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   for (int w = TPR / 2; w > 0; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
   if (valid && part == 0) {
     Drow[row] = s;
-    lse2[row] = lse[row] * 1.4426950408889634f;
+    lse2[row] = -lse[row] * 1.4426950408889634f;
   }
 }
 
 // ---------------------------------------------------------------- common
 
 struct BwdParams {
-  const float* lse2;    // [BH, N] lse * log2(e)
+  const float* lse2;    // [BH, N] -lse * log2(e)
   const float* Drow;    // [BH, N]
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
@@ -429,19 +430,19 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           ok = false;
           break;
         }
+        const uint64_t c2v = f2(c2, c2);
 #pragma unroll
-        for (int t4 = 0; t4 < 16; ++t4) {
-          const int c0 = 4 * t4;
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0);
-          float pv[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float lu = u == 0 ? l4.x : u == 1 ? l4.y : u == 2 ? l4.z : l4.w;
-            pv[u] = ex2(fmaf(__uint_as_float(raw[c0 + u]), c2, -lu));
-            if (diag) pv[u] = (h * 64 + c0 + u < r) ? 0.f : pv[u];
+        for (int t = 0; t < 32; ++t) {
+          const int c0 = 2 * t;
+          const float2 nl = *reinterpret_cast<const float2*>(lse2 + c0);  // -lse log2 e
+          uint64_t pv = ex2_split_x2(f2_fma(f2(__uint_as_float(raw[c0]), __uint_as_float(raw[c0 + 1])), c2v,
+                                            f2(nl.x, nl.y)), t);
+          if (diag) {
+            const float2 v = f2_split(pv);
+            pv = f2((h * 64 + c0 < r) ? 0.f : v.x, (h * 64 + c0 + 1 < r) ? 0.f : v.y);
           }
-          pk[2 * t4] = pack_bf16(pv[0], pv[1]);
-          pk[2 * t4 + 1] = pack_bf16(pv[2], pv[3]);
+          const float2 v = f2_split(pv);
+          pk[t] = pack_bf16(v.x, v.y);
         }
       }
       tmem_st32(trow + Cfg::kTmS + h * 32, pk);
@@ -466,10 +467,11 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         uint32_t ds[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[t]));
+          const float2 pp = unpack_bf16(pk[t]);
           const float2 dd = *reinterpret_cast<const float2*>(Dr + 2 * t);
-          ds[t] = pack_bf16(pp.x * (__uint_as_float(dpr[2 * t]) - dd.x),
-                            pp.y * (__uint_as_float(dpr[2 * t + 1]) - dd.y));
+          const uint64_t diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), f2(dd.x, dd.y));
+          const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
+          ds[t] = pack_bf16(v.x, v.y);
         }
         tmem_st32(trow + Cfg::kTmDP + h * 32, ds);
       }
@@ -682,15 +684,17 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->s_read);
+        const uint64_t c2v = f2(c2, c2), nl2 = f2(l2, l2);  // l2 = -lse log2 e
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          float p0 = ex2(fmaf(__uint_as_float(raw[2 * t]), c2, -l2));
-          float p1 = ex2(fmaf(__uint_as_float(raw[2 * t + 1]), c2, -l2));
+          uint64_t pv = ex2_split_x2(
+              f2_fma(f2(__uint_as_float(raw[2 * t]), __uint_as_float(raw[2 * t + 1])), c2v, nl2), t);
           if (diag) {
-            p0 = (h * 64 + 2 * t > r) ? 0.f : p0;
-            p1 = (h * 64 + 2 * t + 1 > r) ? 0.f : p1;
+            const float2 v = f2_split(pv);
+            pv = f2((h * 64 + 2 * t > r) ? 0.f : v.x, (h * 64 + 2 * t + 1 > r) ? 0.f : v.y);
           }
-          pk[t] = pack_bf16(p0, p1);
+          const float2 v = f2_split(pv);
+          pk[t] = pack_bf16(v.x, v.y);
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, wc, kSiteBwdDpFull))) {
@@ -707,11 +711,14 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           ok = false;
           break;
         }
+        const uint64_t dv2 = f2(Dv, Dv);
         uint32_t ds[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[t]));
-          ds[t] = pack_bf16(pp.x * (__uint_as_float(dpr[2 * t]) - Dv), pp.y * (__uint_as_float(dpr[2 * t + 1]) - Dv));
+          const float2 pp = unpack_bf16(pk[t]);
+          const uint64_t diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), dv2);
+          const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
+          ds[t] = pack_bf16(v.x, v.y);
         }
         tmem_st32(trow + Cfg::kQTmDP + h * 32, ds);
       }

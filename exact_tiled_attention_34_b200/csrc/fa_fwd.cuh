@@ -118,51 +118,69 @@ enum FwdSite : int {
 
 // One softmax step for the calling thread's row: s[0..127] are the raw scores of
 // the current K/V tile; m is the running (base-2, scaled) reference max. Writes the
-// bf16 probabilities into TMEM at tp (64 columns of packed pairs), returns the two
-// partial row sums, the factor alpha = 2^(m - m_use) for the old O and l, and the new
+// bf16 probabilities into TMEM at tp (64 columns of packed pairs), returns the row
+// sum of this tile, the factor alpha = 2^(m - m_use) for the old O and l, and the new
 // reference max m_use. The rescale decision is warp-uniform (see the file header).
+// Pairs of columns go through packed f32x2 arithmetic; the exponentials are split
+// between the special-function unit and a polynomial on the FMA pipe.
 // DIAG: the tile on the causal diagonal; column t is visible iff t <= r.
 template <bool DIAG>
-__device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, float m, uint32_t tp, float& sum0,
-                                            float& sum1, float& alpha, float& m_use) {
+__device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, float m, uint32_t tp, float& sum,
+                                            float& alpha, float& m_use) {
   float mx;
   if (c >= 0.f) {
-    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < 128; ++t) a[t & 3] = fmaxf(a[t & 3], (DIAG && t > r) ? -INFINITY : s[t]);
-    mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * c;
+    for (int t = 0; t < 128; t += 4) {
+      a0 = max3f(a0, (DIAG && t > r) ? -INFINITY : s[t], (DIAG && t + 1 > r) ? -INFINITY : s[t + 1]);
+      a1 = max3f(a1, (DIAG && t + 2 > r) ? -INFINITY : s[t + 2], (DIAG && t + 3 > r) ? -INFINITY : s[t + 3]);
+    }
+    mx = fmaxf(a0, a1) * c;
   } else {
-    float a[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+    float a0 = INFINITY, a1 = INFINITY;
 #pragma unroll
-    for (int t = 0; t < 128; ++t) a[t & 3] = fminf(a[t & 3], (DIAG && t > r) ? INFINITY : s[t]);
-    mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * c;
+    for (int t = 0; t < 128; t += 4) {
+      a0 = min3f(a0, (DIAG && t > r) ? INFINITY : s[t], (DIAG && t + 1 > r) ? INFINITY : s[t + 1]);
+      a1 = min3f(a1, (DIAG && t + 2 > r) ? INFINITY : s[t + 2], (DIAG && t + 3 > r) ? INFINITY : s[t + 3]);
+    }
+    mx = fminf(a0, a1) * c;
   }
   const float m_new = fmaxf(m, mx);
   const bool rescale = __any_sync(0xffffffffu, m_new > m + 8.f);
   m_use = rescale ? m_new : m;
   const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
   alpha = ex2(m - m_sub);  // 0 on the first tile (m = -inf), 1 when the max is kept
-  sum0 = 0.f;
-  sum1 = 0.f;
+  const uint64_t c2 = f2(c, c), nm2 = f2(-m_sub, -m_sub);
+  uint64_t acc = f2(0.f, 0.f);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t pk[32];
 #pragma unroll
     for (int t = 0; t < 32; ++t) {
       const int c0 = h * 64 + 2 * t;
-      float p0 = ex2(fmaf(s[c0], c, -m_sub));
-      float p1 = ex2(fmaf(s[c0 + 1], c, -m_sub));
+      const uint64_t x = f2_fma(f2(s[c0], s[c0 + 1]), c2, nm2);
+      uint64_t pv = ex2_split_x2(x, t);
       if (DIAG) {
-        p0 = (c0 > r) ? 0.f : p0;
-        p1 = (c0 + 1 > r) ? 0.f : p1;
+        const float2 v = f2_split(pv);
+        pv = f2((c0 > r) ? 0.f : v.x, (c0 + 1 > r) ? 0.f : v.y);
       }
-      sum0 += p0;
-      sum1 += p1;
-      pk[t] = pack_bf16(p0, p1);
+      acc = f2_add(acc, pv);
+      const float2 v = f2_split(pv);
+      pk[t] = pack_bf16(v.x, v.y);
     }
     tmem_st32(tp + h * 32, pk);
   }
+  const float2 a = f2_split(acc);
+  sum = a.x + a.y;
 }
+
+// Register split of the 384-thread forward block (launched with 168 per thread,
+// 64,512 in all): the producer/MMA warpgroup drops to 80, the two softmax
+// warpgroups rise to 200 -> 128 * (80 + 2 * 200) = 61,440. Only the softmax
+// warpgroups increase, once, by less than the first warpgroup releases.
+constexpr int kFwdRegsCtl = 80;
+constexpr int kFwdRegsSoftmax = 200;
+constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 
 template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(384, 1)
@@ -222,6 +240,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    regs_dec<kFwdRegsCtl>();
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -258,8 +277,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
     }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    regs_dec<kFwdRegsCtl>();
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);  // S = Q K^T, both K-major
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // O += P V, V is N-major
@@ -337,8 +360,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mma_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, wc, kSiteFwdDrain);
     }
-  } else if (warp >= 4) {
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmCols);
+  } else if (warp < 4) {
+    // idle warps of the first warpgroup: they take part in its register hand-over
+    regs_dec<kFwdRegsCtl>();
+    __syncthreads();
+  } else {
     // ------------------------------------------------------------ softmax warpgroups
+    regs_inc<kFwdRegsSoftmax>();
     const int i = (warp - 4) >> 2;  // Q tile of this warpgroup
     const int quarter = warp & 3;   // TMEM lane quarter
     const int r = quarter * 32 + lane;
@@ -367,13 +400,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           for (int t = 0; t < 32; ++t) s[q4 * 32 + t] = __uint_as_float(raw[t]);
         }
         tmem_wait_ld();
-        float sum0, sum1, alpha, m_use;
+        float sum, alpha, m_use;
         if (CAUSAL && j == tile)
-          softmax_row<true>(s, r, c, m, trow + Cfg::tm_p(i), sum0, sum1, alpha, m_use);
+          softmax_row<true>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
         else
-          softmax_row<false>(s, r, c, m, trow + Cfg::tm_p(i), sum0, sum1, alpha, m_use);
+          softmax_row<false>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
         const bool rescale = m_use != m;
-        l = l * alpha + (sum0 + sum1);
+        l = l * alpha + sum;
         if (__any_sync(0xffffffffu, rescale) && cnt > 0) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -424,16 +457,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         p.lse[row] = -INFINITY;
       }
     }
+    tc_fence_before();
+    __syncthreads();
   }
-
-  // ---------------------------------------------------------------- teardown
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, Cfg::kTmCols);
-  }
+  // Every role ends with its own CTA barrier (no common tail, so each warpgroup
+  // keeps its register budget to the end); warp 1 then frees TMEM.
 }
 
 }  // namespace fa

@@ -293,4 +293,91 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float2 unpack_bf16(uint32_t v) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+}
+
+// ---- packed pairs of fp32 (one f32x2 instruction works on both halves; low half first)
+
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Three-input maximum / minimum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of values without the special-function unit, so that part of a
+// tile's exponentials can run on the FMA and integer pipes next to the MUFU ones.
+// x = n + f with n = round(x) (adding 1.5 * 2^23 rounds to an integer in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f ~ 1 + f (c1 + f (c2 + f c3)), a cubic
+// fitted here to minimise the relative error on [-1/2, 1/2] with the constant term
+// fixed at 1 (csrc/fit_exp2_poly.py: max relative error 1.02e-4, 2^0 exact); 2^n is
+// then added into the exponent field. Inputs below -126 are clamped (result about
+// 1e-38), so the exponent never underflows; inputs must stay below 2^22.
+__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x) {
+  constexpr float kC1 = 6.932800412e-01f, kC2 = 2.422109395e-01f, kC3 = 5.502312258e-02f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float2 xv = f2_split(x);
+  const uint64_t xc = f2(fmaxf(xv.x, -126.f), fmaxf(xv.y, -126.f));
+  const uint64_t rnd = f2(kRound, kRound);
+  const uint64_t t = f2_add(xc, rnd);            // round(x) in the low mantissa bits
+  const uint64_t f = f2_sub(xc, f2_sub(t, rnd));  // x - round(x)
+  uint64_t p = f2_fma(f, f2(kC3, kC3), f2(kC2, kC2));
+  p = f2_fma(p, f, f2(kC1, kC1));
+  p = f2_fma(p, f, f2(1.f, 1.f));
+  const float2 pv = f2_split(p), tv = f2_split(t);
+  const uint32_t y0 = __float_as_uint(pv.x) + (__float_as_uint(tv.x) << 23);
+  const uint32_t y1 = __float_as_uint(pv.y) + (__float_as_uint(tv.y) << 23);
+  return f2(__uint_as_float(y0), __uint_as_float(y1));
+}
+
+// 2^x for a pair on the special-function unit.
+__device__ __forceinline__ uint64_t ex2_mufu_x2(uint64_t x) {
+  const float2 v = f2_split(x);
+  return f2(ex2(v.x), ex2(v.y));
+}
+
+// Which column pairs use the polynomial: pairs t with (t mod 8) < kPolyPer8. Called
+// from fully unrolled loops, so the choice is made at compile time.
+constexpr int kPolyPer8 = 3;
+__device__ __forceinline__ uint64_t ex2_split_x2(uint64_t x, int t) {
+  return ((t & 7) < kPolyPer8) ? ex2_poly_x2(x) : ex2_mufu_x2(x);
+}
+
 }  // namespace fa

@@ -188,6 +188,16 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  */
 fa_status fa_device_status(void* stream, int* detail);
 
+/*
+ * Diagnostic: y[i] = 2^x[i] for i < n, evaluated on the device by one of the two
+ * exponential paths the kernels split every score tile between. mode 0: the
+ * special-function unit (ex2.approx); mode 1: the library's own polynomial
+ * (round-to-nearest range reduction, cubic fitted on [-1/2, 1/2], max relative
+ * error about 1e-4; inputs below -126 give about 1e-38). x and y are device
+ * arrays of n floats, n >= 0; asynchronous on `stream` like every call here.
+ */
+fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int fa_version(void);
 
