@@ -63,6 +63,32 @@ def workload(name: str):
     return dict(B=w["B"], H=w["H"], N=w["N"], d=w["d"], variants=variants, do_scale=1.0)
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+# Every (batch, head) is independent, so ranks run the workload on their own inputs
+# (weak scaling) and share nothing on the data path; the process group only carries
+# barriers and the max-over-ranks reduction of the measured device time.
+
+def rank_seed(rank: int) -> int:
+    """Input seed of a rank: each rank processes its own shard of the job."""
+    return rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (the value itself when alone)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOPs/s: all ranks' algorithmic FLOPs over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def fwd_flops(B, H, N, d, causal, density=1.0):
     f = 4.0 * B * H * N * N * d
     if causal:
@@ -277,7 +303,7 @@ def run_ours(args, wl_name, wl):
 
     B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
     sc = 1.0 / math.sqrt(d)
-    host = make_qkv(B, H, N, d, seed=rank, do_scale=wl["do_scale"])
+    host = make_qkv(B, H, N, d, seed=rank_seed(rank), do_scale=wl["do_scale"])
     t = {k: v.to(dev) for k, v in host.items()}
     masks = {}
     for (_, _, dens) in wl["variants"]:
@@ -366,13 +392,9 @@ def run_ours(args, wl_name, wl):
             per[label]["dq"] += a[3]
             tot += sum(a)
         step_ms.append(tot)
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     K = args.steps
-    value = world * step_flops * K / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, step_flops, K, total_ms)
 
     pk, pk_kind = peaks()
     sustained = clk is not None and clk["sm_mhz"] < 0.9 * clk.get("sm_max_mhz", 1965.0)
@@ -435,12 +457,8 @@ def run_ours(args, wl_name, wl):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = job_throughput(world, step_flops, e2e_steps, e2e_ms)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOPs/s", "n_gpus": world, "steps": K,

@@ -134,7 +134,10 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     regs[dev] = attr.numRegs;
   }
   if (regs[dev] * fa::FwdCfg<D>::kThreads < fa::kFwdRegsNeeded) return FA_ERR_UNSUPPORTED;
-  const unsigned grid = unsigned(p.n_qblocks) * unsigned(p.BH);
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return FA_ERR_CUDA;
+  const unsigned grid = unsigned(p.n_items < sms ? p.n_items : sms);  // persistent: one CTA per SM
   kernel<<<grid, fa::FwdCfg<D>::kThreads, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -163,6 +166,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.BH = BH;
   p.n_tiles = N / 128;
   p.n_qblocks = (p.n_tiles + 1) / 2;
+  p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mask) {

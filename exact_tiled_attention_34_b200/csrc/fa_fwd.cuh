@@ -8,8 +8,11 @@
 // on-chip memory with the softmax reduced progressively, the normalisation factor
 // saved for the backward.
 //
-// One CTA owns a block of 2 x 128 query rows (two Q tiles) of one (batch, head) and
-// streams the 128-key K/V tiles it needs through a shared-memory ring:
+// The kernel is persistent: one CTA per SM walks a static list of work items, each a
+// block of 2 x 128 query rows (two Q tiles) of one (batch, head), streaming the
+// 128-key K/V tiles the block needs through a shared-memory ring that runs on
+// across items (as do the barrier phases), so that the next item's Q load and first
+// S products overlap the previous item's last products and epilogue:
 //   warp 0      TMA producer (one elected thread): Q once, then K_j, V_j per tile
 //   warp 1      MMA issuer (one thread) + TMEM allocator (whole warp)
 //   warps 4-7   softmax warpgroup for Q tile 0 (thread = query row = TMEM lane)
@@ -41,6 +44,7 @@ struct FwdParams {
   int BH;                    // B * H
   int n_tiles;               // N / 128
   int n_qblocks;             // ceil(n_tiles / 2)
+  int n_items;               // n_qblocks * BH work items (query block, batch*head)
   float c_log2;              // scale * log2(e)
 };
 
@@ -76,10 +80,36 @@ struct FwdBars {
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t o_full[2];
+  uint64_t o_empty[2];   // the softmax warpgroup has read O_i (the next item may overwrite it)
+  uint64_t q_empty;      // the item's S products are done with the Q tiles
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
 };
+
+// Persistent schedule: the k-th work item of this CTA, or false when it has none.
+// Rounds of gridDim.x items are dealt to the CTAs alternately forwards and backwards.
+// Item order: with all items equal (no causal mask) head-major, so the query blocks
+// of one head run together and share its K/V tiles through L2; with the causal mask
+// the cost of a block grows with its index, so items go longest first across all
+// heads (block-major), which with the alternating deal balances the CTAs' work.
+struct FwdItem {
+  int bh, qb;
+};
+template <bool CAUSAL>
+__device__ __forceinline__ bool fwd_item(int n_items, int n_qblocks, int BH, int k, FwdItem& it) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const long long pos = static_cast<long long>(k) * G + ((k & 1) ? (G - 1 - c) : c);
+  if (pos >= n_items) return false;
+  if (CAUSAL) {
+    it.qb = n_qblocks - 1 - static_cast<int>(pos / BH);
+    it.bh = static_cast<int>(pos % BH);
+  } else {
+    it.bh = static_cast<int>(pos / n_qblocks);
+    it.qb = n_qblocks - 1 - static_cast<int>(pos % n_qblocks);
+  }
+  return true;
+}
 
 // Which of the CTA's two Q tiles need K/V tile j (bit 0: tile 0, bit 1: tile 1).
 template <bool CAUSAL, bool SPARSE>
@@ -113,7 +143,7 @@ struct FwdSched {
 // Wait-site codes reported through the status word (detail field).
 enum FwdSite : int {
   kSiteFwdQ = 101, kSiteFwdKvEmpty, kSiteFwdKFull, kSiteFwdVFull, kSiteFwdPReady, kSiteFwdSFull,
-  kSiteFwdOFull, kSiteFwdDrain
+  kSiteFwdOFull, kSiteFwdDrain, kSiteFwdQEmpty, kSiteFwdOEmpty
 };
 
 // One softmax step for the calling thread's row: s[0..127] are the raw scores of
@@ -124,7 +154,7 @@ enum FwdSite : int {
 // Pairs of columns go through packed f32x2 arithmetic; the exponentials are split
 // between the special-function unit and a polynomial on the FMA pipe.
 // DIAG: the tile on the causal diagonal; column t is visible iff t <= r.
-template <bool DIAG>
+template <bool DIAG, int POLY8>
 __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, float m, uint32_t tp, float& sum,
                                             float& alpha, float& m_use) {
   float mx;
@@ -159,7 +189,7 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, flo
     for (int t = 0; t < 32; ++t) {
       const int c0 = h * 64 + 2 * t;
       const uint64_t x = f2_fma(f2(s[c0], s[c0 + 1]), c2, nm2);
-      uint64_t pv = ex2_split_x2(x, t);
+      uint64_t pv = ex2_split_x2<POLY8>(x, t);
       if (DIAG) {
         const float2 v = f2_split(pv);
         pv = f2((c0 > r) ? 0.f : v.x, (c0 + 1 > r) ? 0.f : v.y);
@@ -197,24 +227,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   const int warp = warp_id();
   const int lane = lane_id();
-
-  // Head-major order (the query blocks of one head run together and share its K/V
-  // tiles through L2), longest causal blocks first within a head.
-  const int lin = blockIdx.x;
-  const int bh = lin / p.n_qblocks;
-  const int qb = p.n_qblocks - 1 - lin % p.n_qblocks;
-
-  FwdSched<CAUSAL, SPARSE> sch;
-  sch.t0 = 2 * qb;
-  sch.t1 = 2 * qb + 1;
-  sch.valid1 = sch.t1 < p.n_tiles;
-  sch.n_tiles = p.n_tiles;
-  sch.mask = p.tile_mask;
+  auto sched_of = [&](const FwdItem& item) {
+    FwdSched<CAUSAL, SPARSE> sch;
+    sch.t0 = 2 * item.qb;
+    sch.t1 = 2 * item.qb + 1;
+    sch.valid1 = sch.t1 < p.n_tiles;
+    sch.n_tiles = p.n_tiles;
+    sch.mask = p.tile_mask;
+    return sch;
+  };
 
   WaitCtl wc{&bars->abort, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
@@ -224,6 +251,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_ready[i], 128);
       mbar_init(&bars->o_full[i], 1);
+      mbar_init(&bars->o_empty[i], 128);
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -246,34 +274,48 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       const uint64_t keep = policy_evict_last();
-      mbar_arrive_expect_tx(&bars->q_full, Cfg::kTileBytes * (sch.valid1 ? 2 : 1));
-      for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-        tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, sch.t0 * 128, bh);
-      if (sch.valid1)
+      int it = 0;   // K/V tiles loaded so far (ring position, continues across items)
+      int nq = 0;   // Q blocks loaded so far
+      bool ok = true;
+      FwdItem item;
+      for (int k = 0; ok && fwd_item<CAUSAL>(p.n_items, p.n_qblocks, p.BH, k, item); ++k) {
+        const auto sch = sched_of(item);
+        // The previous item's S products must be done with the Q buffer.
+        if (k > 0 && !mbar_wait(&bars->q_empty, (k - 1) & 1, wc, kSiteFwdQEmpty)) break;
+        mbar_arrive_expect_tx(&bars->q_full, Cfg::kTileBytes * (sch.valid1 ? 2 : 1));
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-          tma_load_3d(sQ + Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64,
-                      sch.t1 * 128, bh);
-      int it = 0;
-      uint32_t b;
-      for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b), ++it) {
-        const int st = it % S;
-        const int n = it / S;
-        if (n > 0 && !mbar_wait(&bars->kv_empty[st], (n - 1) & 1, wc, kSiteFwdKvEmpty)) break;
-        uint8_t* dk = sK + st * Cfg::kTileBytes;
-        uint8_t* dv = sV + st * Cfg::kTileBytes;
-        mbar_arrive_expect_tx(&bars->k_full[st], Cfg::kTileBytes);
-        for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-          tma_load_3d_hint(dk + cb * Cfg::kBlockBytes, &tm_k, &bars->k_full[st], cb * 64, j * 128, bh, keep);
-        mbar_arrive_expect_tx(&bars->v_full[st], Cfg::kTileBytes);
-        for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-          tma_load_3d_hint(dv + cb * Cfg::kBlockBytes, &tm_v, &bars->v_full[st], cb * 64, j * 128, bh, keep);
+          tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, sch.t0 * 128, item.bh);
+        if (sch.valid1)
+          for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+            tma_load_3d(sQ + Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64,
+                        sch.t1 * 128, item.bh);
+        ++nq;
+        uint32_t b;
+        for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b), ++it) {
+          const int st = it % S;
+          const int n = it / S;
+          if (n > 0 && !mbar_wait(&bars->kv_empty[st], (n - 1) & 1, wc, kSiteFwdKvEmpty)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dk = sK + st * Cfg::kTileBytes;
+          uint8_t* dv = sV + st * Cfg::kTileBytes;
+          mbar_arrive_expect_tx(&bars->k_full[st], Cfg::kTileBytes);
+          for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+            tma_load_3d_hint(dk + cb * Cfg::kBlockBytes, &tm_k, &bars->k_full[st], cb * 64, j * 128, item.bh,
+                             keep);
+          mbar_arrive_expect_tx(&bars->v_full[st], Cfg::kTileBytes);
+          for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
+            tma_load_3d_hint(dv + cb * Cfg::kBlockBytes, &tm_v, &bars->v_full[st], cb * 64, j * 128, item.bh,
+                             keep);
+        }
       }
       // On abort, wait (bounded) for this thread's own copies still in flight.
       if (bars->abort) {
-        mbar_wait_drain(&bars->q_full, 0, wc, kSiteFwdDrain);
-        for (int i = (it > S ? it - S : 0); i < it; ++i) {
-          mbar_wait_drain(&bars->k_full[i % S], (i / S) & 1, wc, kSiteFwdDrain);
-          mbar_wait_drain(&bars->v_full[i % S], (i / S) & 1, wc, kSiteFwdDrain);
+        if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1, wc, kSiteFwdDrain);
+        for (int x = (it > S ? it - S : 0); x < it; ++x) {
+          mbar_wait_drain(&bars->k_full[x % S], (x / S) & 1, wc, kSiteFwdDrain);
+          mbar_wait_drain(&bars->v_full[x % S], (x / S) & 1, wc, kSiteFwdDrain);
         }
       }
     }
@@ -305,54 +347,69 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                  sdesc_sw128(va + k * 16 * 128, Cfg::kBlockBytes, 1024), idO, (acc || k > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&bars->q_full, 0, wc, kSiteFwdQ);
-      tc_fence_after();
-      uint32_t issued = 0;
-      int cnt[2] = {0, 0};
-      int it = 0;
-      uint32_t b = 0, bn = 0;
-      int j = ok ? sch.next(-1, b) : -1;
-      while (j >= 0) {
-        const int st = it % S;
-        const uint32_t ph = (it / S) & 1;
-        const int jn = sch.next(j, bn);
-        const int stn = (it + 1) % S;
-        const uint32_t phn = ((it + 1) / S) & 1;
-        const uint32_t need = b & ~issued;
-        if (need) {
-          if (!mbar_wait(&bars->k_full[st], ph, wc, kSiteFwdKFull)) { ok = false; break; }
-          tc_fence_after();
-          for (int i = 0; i < 2; ++i)
-            if (need & (1u << i)) {
-              issue_s(i, st);
-              mma_commit(&bars->s_full[i]);
-            }
-        }
-        if (!mbar_wait(&bars->v_full[st], ph, wc, kSiteFwdVFull)) { ok = false; break; }
+      bool ok = true;
+      int it = 0;               // K/V ring position (continues across items)
+      int cnt[2] = {0, 0};      // S_i / P_i handshakes so far (continue across items)
+      FwdItem item;
+      for (int kk = 0; ok && fwd_item<CAUSAL>(p.n_items, p.n_qblocks, p.BH, kk, item); ++kk) {
+        const auto sch = sched_of(item);
+        if (!mbar_wait(&bars->q_full, kk & 1, wc, kSiteFwdQ)) { ok = false; break; }
         tc_fence_after();
-        uint32_t next_issued = 0;
-        for (int i = 0; i < 2; ++i) {
-          if (!(b & (1u << i))) continue;
-          if (!mbar_wait(&bars->p_ready[i], cnt[i] & 1, wc, kSiteFwdPReady)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(i, st, cnt[i] > 0);
-          ++cnt[i];
-          if (jn >= 0 && (bn & (1u << i))) {
-            if (!mbar_wait(&bars->k_full[stn], phn, wc, kSiteFwdKFull)) { ok = false; break; }
+        uint32_t issued = 0;
+        bool first_pv[2] = {true, true};
+        uint32_t b = 0, bn = 0;
+        int j = sch.next(-1, b);
+        if (j < 0) mma_commit(&bars->q_empty);  // nothing to do for this block
+        while (j >= 0) {
+          const int st = it % S;
+          const uint32_t ph = (it / S) & 1;
+          const int jn = sch.next(j, bn);
+          const int stn = (it + 1) % S;
+          const uint32_t phn = ((it + 1) / S) & 1;
+          const uint32_t need = b & ~issued;
+          if (need) {
+            if (!mbar_wait(&bars->k_full[st], ph, wc, kSiteFwdKFull)) { ok = false; break; }
             tc_fence_after();
-            issue_s(i, stn);
-            mma_commit(&bars->s_full[i]);
-            next_issued |= 1u << i;
+            for (int i = 0; i < 2; ++i)
+              if (need & (1u << i)) {
+                issue_s(i, st);
+                mma_commit(&bars->s_full[i]);
+              }
           }
+          // Every S product of this item has now been issued: release Q when they finish.
+          if (jn < 0) mma_commit(&bars->q_empty);
+          if (!mbar_wait(&bars->v_full[st], ph, wc, kSiteFwdVFull)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t next_issued = 0;
+          for (int i = 0; i < 2; ++i) {
+            if (!(b & (1u << i))) continue;
+            if (!mbar_wait(&bars->p_ready[i], cnt[i] & 1, wc, kSiteFwdPReady)) { ok = false; break; }
+            // The first P.V of an item overwrites O_i: the previous item's epilogue must
+            // have read it.
+            if (first_pv[i] && kk > 0 && !mbar_wait(&bars->o_empty[i], (kk - 1) & 1, wc, kSiteFwdOEmpty)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(i, st, !first_pv[i]);
+            first_pv[i] = false;
+            ++cnt[i];
+            if (jn >= 0 && (bn & (1u << i))) {
+              if (!mbar_wait(&bars->k_full[stn], phn, wc, kSiteFwdKFull)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(i, stn);
+              mma_commit(&bars->s_full[i]);
+              next_issued |= 1u << i;
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars->kv_empty[st]);
+          issued = next_issued;
+          b = bn;
+          j = jn;
+          ++it;
         }
         if (!ok) break;
-        mma_commit(&bars->kv_empty[st]);
-        issued = next_issued;
-        b = bn;
-        j = jn;
-        ++it;
-      }
-      if (ok) {
         mma_commit(&bars->o_full[0]);
         mma_commit(&bars->o_full[1]);
       }
@@ -375,86 +432,104 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int i = (warp - 4) >> 2;  // Q tile of this warpgroup
     const int quarter = warp & 3;   // TMEM lane quarter
     const int r = quarter * 32 + lane;
-    const int tile = i == 0 ? sch.t0 : sch.t1;
-    const bool active = (i == 0) || sch.valid1;
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
     const float c = p.c_log2;
-    float m = -INFINITY, l = 0.f;
-    int cnt = 0;
+    int cnt = 0;  // S_i tiles consumed so far (continues across items)
     bool ok = true;
-    if (active) {
-      uint32_t b;
-      for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b)) {
-        if (!(b & (1u << i))) continue;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], cnt & 1, wc, kSiteFwdSFull))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float s[128];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t raw[32];
-          tmem_ld32(trow + Cfg::tm_s(i) + q4 * 32, raw);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) s[q4 * 32 + t] = __uint_as_float(raw[t]);
-        }
-        tmem_wait_ld();
-        float sum, alpha, m_use;
-        if (CAUSAL && j == tile)
-          softmax_row<true>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
-        else
-          softmax_row<false>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
-        const bool rescale = m_use != m;
-        l = l * alpha + sum;
-        if (__any_sync(0xffffffffu, rescale) && cnt > 0) {
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int t = 0; t < 32; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * alpha);
-            tmem_st32(trow + Cfg::tm_o(i) + cc * 32, ov);
+    FwdItem item;
+    for (int kk = 0; ok && fwd_item<CAUSAL>(p.n_items, p.n_qblocks, p.BH, kk, item); ++kk) {
+      const auto sch = sched_of(item);
+      const int tile = i == 0 ? sch.t0 : sch.t1;
+      const bool active = (i == 0) || sch.valid1;
+      float m = -INFINITY, l = 0.f;
+      int local = 0;  // tiles of this item
+      if (active) {
+        uint32_t b;
+        for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b)) {
+          if (!(b & (1u << i))) continue;
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], cnt & 1, wc, kSiteFwdSFull))) {
+            ok = false;
+            break;
           }
-        }
-        m = m_use;
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_ready[i]);
-        ++cnt;
-      }
-      // ---------------------------------------------------------- epilogue
-      const size_t row = size_t(bh) * p.N + size_t(tile) * 128 + r;
-      __nv_bfloat16* orow = p.o + row * D;
-      if (ok && cnt > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[i], 0, wc, kSiteFwdOFull));
-        if (ok) {
           tc_fence_after();
-          const float inv_l = 1.f / l;
+          float s[128];
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, ov);
-            tmem_wait_ld();
-            uint4 pk[4];
-            uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t raw[32];
+            tmem_ld32(trow + Cfg::tm_s(i) + q4 * 32, raw);
 #pragma unroll
-            for (int t = 0; t < 16; ++t)
-              pw[t] = pack_bf16(__uint_as_float(ov[2 * t]) * inv_l, __uint_as_float(ov[2 * t + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) dst[t] = pk[t];
+            for (int t = 0; t < 32; ++t) s[q4 * 32 + t] = __uint_as_float(raw[t]);
           }
-          p.lse[row] = (m + __log2f(l)) * 0.69314718055994531f;
-        }
-      } else if (ok) {
-        // No visible key for this row (only possible with a block mask).
-        uint4 z = make_uint4(0, 0, 0, 0);
-        uint4* dst = reinterpret_cast<uint4*>(orow);
+          tmem_wait_ld();
+          float sum, alpha, m_use;
+          if (CAUSAL && j == tile)
+            softmax_row<true, PolyShare<D>::kPer8>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+          else
+            softmax_row<false, PolyShare<D>::kPer8>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+          const bool rescale = m_use != m;
+          l = l * alpha + sum;
+          if (__any_sync(0xffffffffu, rescale) && local > 0) {
 #pragma unroll
-        for (int t = 0; t < D / 8; ++t) dst[t] = z;
-        p.lse[row] = -INFINITY;
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t ov[32];
+              tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int t = 0; t < 32; ++t) ov[t] = __float_as_uint(__uint_as_float(ov[t]) * alpha);
+              tmem_st32(trow + Cfg::tm_o(i) + cc * 32, ov);
+            }
+          }
+          m = m_use;
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars->p_ready[i]);
+          ++cnt;
+          ++local;
+        }
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      // Every item ends with one o_full phase per tile and one o_empty arrival per
+      // thread, whether or not this tile had work, so the phases stay in step.
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[i], kk & 1, wc, kSiteFwdOFull))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const size_t row = size_t(item.bh) * p.N + size_t(tile) * 128 + r;
+      __nv_bfloat16* orow = p.o + row * D;
+      if (active && local > 0) {
+        const float inv_l = 1.f / l;
+        uint32_t ov[D];
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc)
+          tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc * 32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->o_empty[i]);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            pw[t] = pack_bf16(__uint_as_float(ov[cc * 32 + 2 * t]) * inv_l,
+                              __uint_as_float(ov[cc * 32 + 2 * t + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) dst[t] = pk[t];
+        }
+        p.lse[row] = (m + __log2f(l)) * 0.69314718055994531f;
+      } else {
+        mbar_arrive(&bars->o_empty[i]);
+        if (active) {
+          // No visible key for this row (only possible with a block mask).
+          const uint4 z = make_uint4(0, 0, 0, 0);
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int t = 0; t < D / 8; ++t) dst[t] = z;
+          p.lse[row] = -INFINITY;
+        }
       }
     }
     tc_fence_before();

@@ -373,11 +373,16 @@ __device__ __forceinline__ uint64_t ex2_mufu_x2(uint64_t x) {
   return f2(ex2(v.x), ex2(v.y));
 }
 
-// Which column pairs use the polynomial: pairs t with (t mod 8) < kPolyPer8. Called
-// from fully unrolled loops, so the choice is made at compile time.
-constexpr int kPolyPer8 = 3;
+// Which column pairs use the polynomial: pairs t with (t mod 8) < POLY8. Called from
+// fully unrolled loops, so the choice is made at compile time. (Measured on B200: 3 of
+// 8 beats 5 of 8 at head dim 64, where more polynomial work costs issue slots.)
+template <int D>
+struct PolyShare {
+  static constexpr int kPer8 = 3;
+};
+template <int POLY8>
 __device__ __forceinline__ uint64_t ex2_split_x2(uint64_t x, int t) {
-  return ((t & 7) < kPolyPer8) ? ex2_poly_x2(x) : ex2_mufu_x2(x);
+  return ((t & 7) < POLY8) ? ex2_poly_x2(x) : ex2_mufu_x2(x);
 }
 
 }  // namespace fa

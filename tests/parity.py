@@ -30,11 +30,13 @@ def max_abs(a, b) -> float:
 
 
 def tol_o_sharp(v) -> float:
-    """O tolerance for peaked softmaxes (scales far from 1/sqrt(d)).
+    """O tolerance for stress cases: peaked softmaxes (scales far from 1/sqrt(d)) and
+    tensors with many more rows than the workloads, where outputs near max|V| occur.
 
-    O = sum_j P_j V_j / l with P rounded to bf16 (relative error <= 2^-9 per term)
-    and O itself rounded to bf16 (<= 2^-9 relative): |dO| <= 2^-8 max|V| plus fp32
-    terms. Twice that bound, and never below the workload tolerance 1e-2.
+    O = sum_j P_j V_j / l with P rounded to bf16 and O itself rounded to bf16. bf16 keeps
+    8 significant bits (unit roundoff 2^-8), so the P rounding moves O by at most
+    2^-8 max|V| and the output rounding by at most 2^-8 |O| <= 2^-8 max|V|: the bound
+    is 2^-7 max|V| (plus fp32 terms), and never below the workload tolerance 1e-2.
     """
     vmax = float(v.detach().float().abs().max()) if torch.is_tensor(v) else float(np.max(np.abs(v)))
     return max(TOL_O, 2.0 ** -7 * vmax)
