@@ -115,6 +115,7 @@ fa_status set_smem(K kernel, int bytes, std::once_flag (&flags)[kMaxDevices], cu
   return errs[dev] == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+
 template <int D, bool CAUSAL, bool SPARSE>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      cudaStream_t stream) {
@@ -181,6 +182,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+
 // Workspace: fp32 D rows [BH*N], then fp32 lse*log2(e) rows [BH*N], each 256-aligned.
 size_t bwd_ws_bytes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
@@ -192,7 +194,7 @@ size_t bwd_ws_bytes(int B, int H, int N, int d) {
 // pool between warpgroups; refuse to launch if the build gave them fewer registers
 // per thread than that split needs.
 template <typename K>
-fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mk,
+fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid /* work items */, const CUtensorMap& mq, const CUtensorMap& mk,
                             const CUtensorMap& mv, const CUtensorMap& mdo, const fa::BwdParams& p,
                             cudaStream_t stream, std::once_flag (&flags)[kMaxDevices],
                             cudaError_t (&errs)[kMaxDevices], int (&regs)[kMaxDevices]) {
@@ -205,6 +207,10 @@ fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid, const CUtensorMap
     regs[dev] = attr.numRegs;
   }
   if (regs[dev] * fa::kBwdThreads < fa::kBwdRegsNeeded) return FA_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return FA_ERR_CUDA;
+  if (grid > unsigned(sms)) grid = unsigned(sms);  // persistent: at most one CTA per SM
   kernel<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -12,21 +12,23 @@
 //
 // Three launches, all deterministic (no atomics):
 //  1. fa_bwd_pre_kernel: D and -lse * log2(e) into the workspace.
-//  2. fa_bwd_dkdv_kernel: one CTA per (128-key tile j, batch*head), looping over the
+//  2. fa_bwd_dkdv_kernel: work item = (128-key tile j, batch*head), looping over the
 //     query tiles i that see tile j (causal: i >= j; block-sparse: mask[i][j] = 1).
 //     The transposed products put key rows on TMEM lanes:
 //       S^T  = K_j Q_i^T   (SS, both K-major)       dP^T = V_j dO_i^T  (SS)
 //       dV  += P^T dO_i    (TS: P^T from TMEM, dO_i N-major)
 //       dK  += dS^T Q_i    (TS: dS^T from TMEM, Q_i N-major)
 //     so the TMA-loaded Q/dO tiles serve as K-major and N-major operands alike.
-//  3. fa_bwd_dq_kernel: one CTA per (128-query tile i, batch*head), looping over the
+//  3. fa_bwd_dq_kernel: work item = (128-query tile i, batch*head), looping over the
 //     key tiles j that tile i sees; it recomputes S = Q_i K_j^T and dP = dO_i V_j^T,
 //     forms dS and accumulates dQ_i += dS K_j in TMEM (TS: dS from TMEM, K_j N-major),
 //     then writes dQ_i once. Recomputing S and dP (2 of its 3 products) costs tensor
 //     time but removes the fp32 atomic accumulation of dQ, whose L2 traffic bounded a
 //     single fused kernel.
 //
-// Both main kernels: 384 threads; warp 0 TMA producer, warp 1 MMA issuer + TMEM
+// Both main kernels are persistent (one CTA per SM walking a static list of items;
+// ring positions and barrier phases run on across items so loads and first products
+// of the next item overlap the previous epilogue). 384 threads; warp 0 TMA producer, warp 1 MMA issuer + TMEM
 // owner, warps 4-11 two "compute" warpgroups (thread = TMEM lane; warpgroup h takes
 // the tile columns [64h, 64h+64)). A packed bf16 result for column c goes to TMEM
 // column c/2, so warpgroup 1 writes columns that warpgroup 0 reads as fp32: both
@@ -225,10 +227,53 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t tadd
   }
 }
 
+// NCOL fp32 values of the thread's row (in registers), times mul, as bf16 to dst.
+template <int NCOL>
+__device__ __forceinline__ void store_regs_bf16(__nv_bfloat16* dst, const uint32_t (&v)[NCOL], float mul) {
+#pragma unroll
+  for (int cc = 0; cc < NCOL / 32; ++cc) {
+    uint4 o4[4];
+    uint32_t* w = reinterpret_cast<uint32_t*>(o4);
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      w[t] = pack_bf16(__uint_as_float(v[cc * 32 + 2 * t]) * mul, __uint_as_float(v[cc * 32 + 2 * t + 1]) * mul);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) d4[t] = o4[t];
+  }
+}
+
+// ---------------------------------------------------------------- persistent schedule
+
+// The k-th work item (tile index, batch*head) of this CTA, or false when it has none.
+// Without the causal mask all items cost the same and go head-major (the tiles of one
+// head together, sharing its other operand tiles through L2); with it, an item's cost
+// grows as its tile index falls (key tiles, dK/dV kernel) or rises (query tiles, dQ
+// kernel), and items go costliest first across all heads, which with the alternating
+// deal of item_position balances the CTAs' work.
+struct BwdItem {
+  int bh, tile;
+};
+template <bool CAUSAL, bool HEAVY_LOW>
+__device__ __forceinline__ bool bwd_item(int n_tiles, int BH, int k, BwdItem& it) {
+  const long long pos = item_position(static_cast<long long>(n_tiles) * BH, k);
+  if (pos < 0) return false;
+  if (CAUSAL) {
+    const int rank = static_cast<int>(pos / BH);  // 0 = most work
+    it.tile = HEAVY_LOW ? rank : n_tiles - 1 - rank;
+    it.bh = static_cast<int>(pos % BH);
+  } else {
+    it.bh = static_cast<int>(pos / n_tiles);
+    it.tile = static_cast<int>(pos % n_tiles);
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- dK / dV kernel
 
 struct DkdvBars {
   uint64_t kv_full;
+  uint64_t kv_empty;  // the item's S^T and dP^T products are done with K_j, V_j
   uint64_t t_full[2];
   uint64_t t_empty[2];
   uint64_t s_full;
@@ -236,6 +281,7 @@ struct DkdvBars {
   uint64_t p_ready;
   uint64_t ds_ready;
   uint64_t acc_done;
+  uint64_t acc_empty;  // the epilogue has read dK and dV (the next item may overwrite them)
   uint64_t mma_done;
   uint64_t rd_s;   // both compute warpgroups have read S^T of this tile
   uint64_t rd_dp;  // ... and dP^T
@@ -261,16 +307,11 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   const int warp = warp_id();
   const int lane = lane_id();
-  // Head-major order (the key tiles of one head run together and share its Q/dO
-  // tiles through L2), small j first within a head (most query tiles when causal).
-  const int lin = blockIdx.x;
-  const int bh = lin / p.n_tiles;
-  const int j = lin % p.n_tiles;
-  KeySched<CAUSAL, SPARSE> sch{j, p.n_tiles, p.tile_mask};
   WaitCtl wc{&bars->abort, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->t_full[s], 1);
       mbar_init(&bars->t_empty[s], 1);
@@ -280,6 +321,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->acc_done, 1);
+    mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->rd_s, 256);
     mbar_init(&bars->rd_dp, 256);
@@ -304,30 +346,42 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kTileBytes);
-      for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-        tma_load_3d(sK + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full, cb * 64, j * 128, bh);
-        tma_load_3d(sV + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full, cb * 64, j * 128, bh);
-      }
       const uint64_t keep = policy_evict_last();
-      int it = 0;
-      for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
-        const int st = it & 1;
-        const int n = it >> 1;
-        if (n > 0 && !mbar_wait(&bars->t_empty[st], (n - 1) & 1, wc, kSiteBwdTEmpty)) break;
-        mbar_arrive_expect_tx(&bars->t_full[st], kTileTx);
+      int it = 0;  // Q/dO tiles loaded so far (ring position, continues across items)
+      int nkv = 0;
+      bool ok = true;
+      BwdItem item;
+      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_tiles, p.BH, kk, item); ++kk) {
+        const int j = item.tile, bh = item.bh;
+        KeySched<CAUSAL, SPARSE> sch{j, p.n_tiles, p.tile_mask};
+        if (kk > 0 && !mbar_wait(&bars->kv_empty, (kk - 1) & 1, wc, kSiteBwdTEmpty)) break;
+        mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-          tma_load_3d_hint(sQ + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->t_full[st], cb * 64,
-                           i * 128, bh, keep);
-          tma_load_3d_hint(sDO + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_do, &bars->t_full[st],
-                           cb * 64, i * 128, bh, keep);
+          tma_load_3d(sK + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full, cb * 64, j * 128, bh);
+          tma_load_3d(sV + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full, cb * 64, j * 128, bh);
         }
-        const size_t roff = size_t(bh) * p.N + size_t(i) * 128;
-        bulk_load(sL + st * 128, p.lse2 + roff, 512, &bars->t_full[st]);
-        bulk_load(sDr + st * 128, p.Drow + roff, 512, &bars->t_full[st]);
+        ++nkv;
+        for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
+          const int st = it & 1;
+          const int n = it >> 1;
+          if (n > 0 && !mbar_wait(&bars->t_empty[st], (n - 1) & 1, wc, kSiteBwdTEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->t_full[st], kTileTx);
+          for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
+            tma_load_3d_hint(sQ + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->t_full[st],
+                             cb * 64, i * 128, bh, keep);
+            tma_load_3d_hint(sDO + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_do, &bars->t_full[st],
+                             cb * 64, i * 128, bh, keep);
+          }
+          const size_t roff = size_t(bh) * p.N + size_t(i) * 128;
+          bulk_load(sL + st * 128, p.lse2 + roff, 512, &bars->t_full[st]);
+          bulk_load(sDr + st * 128, p.Drow + roff, 512, &bars->t_full[st]);
+        }
       }
       if (bars->abort) {
-        mbar_wait_drain(&bars->kv_full, 0, wc, kSiteBwdDrain);
+        if (nkv > 0) mbar_wait_drain(&bars->kv_full, (nkv - 1) & 1, wc, kSiteBwdDrain);
         for (int x = (it > 2 ? it - 2 : 0); x < it; ++x)
           mbar_wait_drain(&bars->t_full[x & 1], (x >> 1) & 1, wc, kSiteBwdDrain);
       }
@@ -340,51 +394,64 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     regs_dec<kBwdRegsCtl>();
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
-      bool ok = mbar_wait(&bars->kv_full, 0, wc, kSiteBwdKV);
-      tc_fence_after();
-      int i = ok ? sch.first() : -1;
-      int it = 0;
-      if (i >= 0) {
-        if (!mbar_wait(&bars->t_full[0], 0, wc, kSiteBwdTFull)) {
-          ok = false;
-          i = -1;
-        } else {
+      bool ok = true;
+      int it = 0;  // query tiles processed so far (continues across items)
+      BwdItem item;
+      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_tiles, p.BH, kk, item); ++kk) {
+        KeySched<CAUSAL, SPARSE> sch{item.tile, p.n_tiles, p.tile_mask};
+        if (!mbar_wait(&bars->kv_full, kk & 1, wc, kSiteBwdKV)) { ok = false; break; }
+        tc_fence_after();
+        int i = sch.first();
+        if (i < 0) mma_commit(&bars->kv_empty);
+        if (i >= 0) {
+          if (!mbar_wait(&bars->t_full[it & 1], (it >> 1) & 1, wc, kSiteBwdTFull)) { ok = false; break; }
           tc_fence_after();
-          mma_tile_nt<D>(tmem + Cfg::kTmS, aK, aQ);
+          mma_tile_nt<D>(tmem + Cfg::kTmS, aK, aQ + (it & 1) * Cfg::kTileBytes);
           mma_commit(&bars->s_full);
-          mma_tile_nt<D>(tmem + Cfg::kTmDP, aV, aDO);
+          mma_tile_nt<D>(tmem + Cfg::kTmDP, aV, aDO + (it & 1) * Cfg::kTileBytes);
           mma_commit(&bars->dp_full);
         }
-      }
-      while (i >= 0) {
-        const int st = it & 1;
-        const int in = sch.next(i);
-        const int stn = (it + 1) & 1;
-        const uint32_t phn = ((it + 1) >> 1) & 1;
-        // dV += P^T dO_i, then the next S^T (it overwrites P^T only after this dV
-        // product has read it: products execute in issue order).
-        if (!mbar_wait(&bars->p_ready, it & 1, wc, kSiteBwdPReady)) { ok = false; break; }
-        tc_fence_after();
-        mma_tile_tn<D>(tmem + Cfg::kTmDV, tmem + Cfg::kTmS, aDO + st * Cfg::kTileBytes, it > 0);
-        if (in >= 0) {
-          if (!mbar_wait(&bars->t_full[stn], phn, wc, kSiteBwdTFull)) { ok = false; break; }
+        bool first = true;
+        while (i >= 0) {
+          const int st = it & 1;
+          const int in = sch.next(i);
+          const int stn = (it + 1) & 1;
+          const uint32_t phn = ((it + 1) >> 1) & 1;
+          // All S^T / dP^T products of this item are issued: K_j, V_j free when done.
+          if (in < 0) mma_commit(&bars->kv_empty);
+          // dV += P^T dO_i, then the next S^T (it overwrites P^T only after this dV
+          // product has read it: products execute in issue order).
+          if (!mbar_wait(&bars->p_ready, it & 1, wc, kSiteBwdPReady)) { ok = false; break; }
+          // The first dV/dK products of an item overwrite the accumulators: the
+          // previous item's epilogue must have read them.
+          if (first && kk > 0 && !mbar_wait(&bars->acc_empty, (kk - 1) & 1, wc, kSiteBwdAcc)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          mma_tile_nt<D>(tmem + Cfg::kTmS, aK, aQ + stn * Cfg::kTileBytes);
-          mma_commit(&bars->s_full);
+          mma_tile_tn<D>(tmem + Cfg::kTmDV, tmem + Cfg::kTmS, aDO + st * Cfg::kTileBytes, !first);
+          if (in >= 0) {
+            if (!mbar_wait(&bars->t_full[stn], phn, wc, kSiteBwdTFull)) { ok = false; break; }
+            tc_fence_after();
+            mma_tile_nt<D>(tmem + Cfg::kTmS, aK, aQ + stn * Cfg::kTileBytes);
+            mma_commit(&bars->s_full);
+          }
+          // dK += dS^T Q_i, then the next dP^T (over dS^T, in issue order).
+          if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteBwdDsReady)) { ok = false; break; }
+          tc_fence_after();
+          mma_tile_tn<D>(tmem + Cfg::kTmDK, tmem + Cfg::kTmDP, aQ + st * Cfg::kTileBytes, !first);
+          mma_commit(&bars->t_empty[st]);
+          if (in >= 0) {
+            mma_tile_nt<D>(tmem + Cfg::kTmDP, aV, aDO + stn * Cfg::kTileBytes);
+            mma_commit(&bars->dp_full);
+          }
+          first = false;
+          i = in;
+          ++it;
         }
-        // dK += dS^T Q_i, then the next dP^T (over dS^T, in issue order).
-        if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteBwdDsReady)) { ok = false; break; }
-        tc_fence_after();
-        mma_tile_tn<D>(tmem + Cfg::kTmDK, tmem + Cfg::kTmDP, aQ + st * Cfg::kTileBytes, it > 0);
-        mma_commit(&bars->t_empty[st]);
-        if (in >= 0) {
-          mma_tile_nt<D>(tmem + Cfg::kTmDP, aV, aDO + stn * Cfg::kTileBytes);
-          mma_commit(&bars->dp_full);
-        }
-        i = in;
-        ++it;
+        if (!ok) break;
+        mma_commit(&bars->acc_done);
       }
-      if (ok) mma_commit(&bars->acc_done);
       mma_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, wc, kSiteBwdDrain);
     }
@@ -407,88 +474,109 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;
     bool ok = true;
-    int it = 0;
-    for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
-      const int st = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->t_full[st], (it >> 1) & 1, wc, kSiteBwdTFull)) ||
-          !__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float* lse2 = sL + st * 128 + h * 64;
-      const float* Dr = sDr + st * 128 + h * 64;
-      const bool diag = CAUSAL && (i == j);  // query c visible to key r iff c >= r
-      // ---- P^T row r, query columns 64h + (0..63), packed bf16 pairs
-      uint32_t pk[32];
-      {
-        uint32_t raw[64];
-        tmem_ld64(trow + Cfg::kTmS + h * 64, raw);
-        tmem_wait_ld();
-        mbar_arrive(&bars->rd_s);
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_s, it & 1, wc, kSiteBwdRead))) {
+    int it = 0;  // query tiles processed so far (continues across items)
+    BwdItem item;
+    for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_tiles, p.BH, kk, item); ++kk) {
+      const int j = item.tile;
+      KeySched<CAUSAL, SPARSE> sch{j, p.n_tiles, p.tile_mask};
+      int local = 0;
+      for (int i = sch.first(); i >= 0; i = sch.next(i), ++it, ++local) {
+        const int st = it & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->t_full[st], (it >> 1) & 1, wc, kSiteBwdTFull)) ||
+            !__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
           ok = false;
           break;
         }
-        const uint64_t c2v = f2(c2, c2);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const int c0 = 2 * t;
-          const float2 nl = *reinterpret_cast<const float2*>(lse2 + c0);  // -lse log2 e
-          uint64_t pv = ex2_split_x2<PolyShare<D>::kPer8>(f2_fma(f2(__uint_as_float(raw[c0]), __uint_as_float(raw[c0 + 1])), c2v,
-                                            f2(nl.x, nl.y)), t);
-          if (diag) {
-            const float2 v = f2_split(pv);
-            pv = f2((h * 64 + c0 < r) ? 0.f : v.x, (h * 64 + c0 + 1 < r) ? 0.f : v.y);
-          }
-          const float2 v = f2_split(pv);
-          pk[t] = pack_bf16(v.x, v.y);
-        }
-      }
-      tmem_st32(trow + Cfg::kTmS + h * 32, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_ready);
-      // ---- dS^T = P^T * (dP^T - D) into TMEM (A operand of dK)
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, wc, kSiteBwdDpFull))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      {
-        uint32_t dpr[64];
-        tmem_ld64(trow + Cfg::kTmDP + h * 64, dpr);
-        tmem_wait_ld();
-        mbar_arrive(&bars->rd_dp);
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
-          ok = false;
-          break;
-        }
-        uint32_t ds[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float2 pp = unpack_bf16(pk[t]);
-          const float2 dd = *reinterpret_cast<const float2*>(Dr + 2 * t);
-          const uint64_t diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), f2(dd.x, dd.y));
-          const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
-          ds[t] = pack_bf16(v.x, v.y);
-        }
-        tmem_st32(trow + Cfg::kTmDP + h * 32, ds);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->ds_ready);
-    }
-    // ---------------------------------------------------------- epilogue: dK (h = 0), dV (h = 1)
-    if (ok) {
-      const bool any = it > 0;
-      if (any) ok = __all_sync(0xffffffffu, mbar_wait(&bars->acc_done, 0, wc, kSiteBwdAcc));
-      if (ok) {
         tc_fence_after();
-        const size_t row = size_t(bh) * p.N + size_t(j) * 128 + r;
-        store_row_bf16<D>((h == 0 ? p.dk : p.dv) + row * D, trow + (h == 0 ? Cfg::kTmDK : Cfg::kTmDV),
-                          h == 0 ? p.scale : 1.f, !any);
+        const float* lse2 = sL + st * 128 + h * 64;
+        const float* Dr = sDr + st * 128 + h * 64;
+        const bool diag = CAUSAL && (i == j);  // query c visible to key r iff c >= r
+        // ---- P^T row r, query columns 64h + (0..63), packed bf16 pairs
+        uint32_t pk[32];
+        {
+          uint32_t raw[64];
+          tmem_ld64(trow + Cfg::kTmS + h * 64, raw);
+          tmem_wait_ld();
+          // The packed P^T of query q goes to column q / 2: warpgroup 1 writes columns
+          // 32..63, which hold scores warpgroup 0 reads. Both finish reading first.
+          mbar_arrive(&bars->rd_s);
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_s, it & 1, wc, kSiteBwdRead))) {
+            ok = false;
+            break;
+          }
+          const uint64_t c2v = f2(c2, c2);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const int c0 = 2 * t;
+            const float2 nl = *reinterpret_cast<const float2*>(lse2 + c0);  // -lse log2 e
+            uint64_t pv = ex2_split_x2<PolyShare<D>::kPer8>(
+                f2_fma(f2(__uint_as_float(raw[c0]), __uint_as_float(raw[c0 + 1])), c2v, f2(nl.x, nl.y)), t);
+            if (diag) {
+              const float2 v = f2_split(pv);
+              pv = f2((h * 64 + c0 < r) ? 0.f : v.x, (h * 64 + c0 + 1 < r) ? 0.f : v.y);
+            }
+            const float2 v = f2_split(pv);
+            pk[t] = pack_bf16(v.x, v.y);
+          }
+        }
+        tmem_st32(trow + Cfg::kTmS + h * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready);
+        // ---- dS^T = P^T * (dP^T - D) into TMEM (A operand of dK)
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, wc, kSiteBwdDpFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        {
+          uint32_t dpr[64];
+          tmem_ld64(trow + Cfg::kTmDP + h * 64, dpr);
+          tmem_wait_ld();
+          mbar_arrive(&bars->rd_dp);
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
+            ok = false;
+            break;
+          }
+          uint32_t ds[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float2 pp = unpack_bf16(pk[t]);
+            const float2 dd = *reinterpret_cast<const float2*>(Dr + 2 * t);
+            const uint64_t diff =
+                f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), f2(dd.x, dd.y));
+            const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
+            ds[t] = pack_bf16(v.x, v.y);
+          }
+          tmem_st32(trow + Cfg::kTmDP + h * 32, ds);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->ds_ready);
       }
+      if (!ok) break;
+      // -------------------------------------------------------- epilogue: dK (h = 0), dV (h = 1)
+      // One acc_done phase and one acc_empty arrival per thread for every item.
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_done, kk & 1, wc, kSiteBwdAcc))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const size_t row = size_t(item.bh) * p.N + size_t(j) * 128 + r;
+      uint32_t acc[D];
+      if (local > 0) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc)
+          tmem_ld32(trow + (h == 0 ? Cfg::kTmDK : Cfg::kTmDV) + cc * 32,
+                    *reinterpret_cast<uint32_t(*)[32]>(&acc[cc * 32]));
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int t = 0; t < D; ++t) acc[t] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty);
+      store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * D, acc, h == 0 ? p.scale : 1.f);
     }
     tc_fence_before();
     __syncthreads();
@@ -501,6 +589,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 struct DqBars {
   uint64_t q_full;
+  uint64_t q_empty;   // the item's S and dP products are done with Q_i, dO_i
   uint64_t kv_full[2];
   uint64_t kv_empty[2];
   uint64_t s_full;
@@ -508,6 +597,7 @@ struct DqBars {
   uint64_t s_read;    // both compute warpgroups have read S (the next S may start)
   uint64_t ds_ready;
   uint64_t acc_done;
+  uint64_t acc_empty;  // the epilogue has read dQ (the next item may overwrite it)
   uint64_t mma_done;
   uint64_t rd_dp;
   uint32_t tmem_base;
@@ -530,15 +620,11 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   const int warp = warp_id();
   const int lane = lane_id();
-  // Head-major order, longest causal query tiles first within a head.
-  const int lin = blockIdx.x;
-  const int bh = lin / p.n_tiles;
-  const int i = p.n_tiles - 1 - lin % p.n_tiles;
-  QuerySched<CAUSAL, SPARSE> sch{i, p.n_tiles, p.tile_mask};
   WaitCtl wc{&bars->abort, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
@@ -548,6 +634,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(&bars->s_read, 256);
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->acc_done, 1);
+    mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->rd_dp, 256);
     bars->abort = 0;
@@ -570,27 +657,39 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&bars->q_full, 2 * Cfg::kTileBytes);
-      for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-        tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, i * 128, bh);
-        tma_load_3d(sDO + cb * Cfg::kBlockBytes, &tm_do, &bars->q_full, cb * 64, i * 128, bh);
-      }
       const uint64_t keep = policy_evict_last();
-      int it = 0;
-      for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it) {
-        const int st = it & 1;
-        const int n = it >> 1;
-        if (n > 0 && !mbar_wait(&bars->kv_empty[st], (n - 1) & 1, wc, kSiteBwdTEmpty)) break;
-        mbar_arrive_expect_tx(&bars->kv_full[st], 2 * Cfg::kTileBytes);
+      int it = 0;  // K/V tiles loaded so far (ring position, continues across items)
+      int nq = 0;
+      bool ok = true;
+      BwdItem item;
+      for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
+        const int i = item.tile, bh = item.bh;
+        QuerySched<CAUSAL, SPARSE> sch{i, p.n_tiles, p.tile_mask};
+        if (kk > 0 && !mbar_wait(&bars->q_empty, (kk - 1) & 1, wc, kSiteBwdTEmpty)) break;
+        mbar_arrive_expect_tx(&bars->q_full, 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-          tma_load_3d_hint(sK + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full[st], cb * 64,
-                           jj * 128, bh, keep);
-          tma_load_3d_hint(sV + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full[st], cb * 64,
-                           jj * 128, bh, keep);
+          tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, i * 128, bh);
+          tma_load_3d(sDO + cb * Cfg::kBlockBytes, &tm_do, &bars->q_full, cb * 64, i * 128, bh);
+        }
+        ++nq;
+        for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it) {
+          const int st = it & 1;
+          const int n = it >> 1;
+          if (n > 0 && !mbar_wait(&bars->kv_empty[st], (n - 1) & 1, wc, kSiteBwdTEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->kv_full[st], 2 * Cfg::kTileBytes);
+          for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
+            tma_load_3d_hint(sK + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full[st],
+                             cb * 64, jj * 128, bh, keep);
+            tma_load_3d_hint(sV + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full[st],
+                             cb * 64, jj * 128, bh, keep);
+          }
         }
       }
       if (bars->abort) {
-        mbar_wait_drain(&bars->q_full, 0, wc, kSiteBwdDrain);
+        if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1, wc, kSiteBwdDrain);
         for (int x = (it > 2 ? it - 2 : 0); x < it; ++x)
           mbar_wait_drain(&bars->kv_full[x & 1], (x >> 1) & 1, wc, kSiteBwdDrain);
       }
@@ -603,48 +702,61 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     regs_dec<kBwdRegsCtl>();
     if (lane == 0) {
       const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(&bars->q_full, 0, wc, kSiteBwdKV);
-      tc_fence_after();
-      int jj = ok ? sch.first() : -1;
-      int it = 0;
-      if (jj >= 0) {
-        if (!mbar_wait(&bars->kv_full[0], 0, wc, kSiteBwdTFull)) {
-          ok = false;
-          jj = -1;
-        } else {
-          tc_fence_after();
-          mma_tile_nt<D>(tmem + Cfg::kQTmS, aQ, aK);
-          mma_commit(&bars->s_full);
-          mma_tile_nt<D>(tmem + Cfg::kQTmDP, aDO, aV);
-          mma_commit(&bars->dp_full);
-        }
-      }
-      while (jj >= 0) {
-        const int st = it & 1;
-        const int jn = sch.next(jj);
-        const int stn = (it + 1) & 1;
-        const uint32_t phn = ((it + 1) >> 1) & 1;
-        // Next S as soon as both warpgroups have read this one.
-        if (jn >= 0) {
-          if (!mbar_wait(&bars->s_read, it & 1, wc, kSiteBwdSRead)) { ok = false; break; }
-          if (!mbar_wait(&bars->kv_full[stn], phn, wc, kSiteBwdTFull)) { ok = false; break; }
-          tc_fence_after();
-          mma_tile_nt<D>(tmem + Cfg::kQTmS, aQ, aK + stn * Cfg::kTileBytes);
-          mma_commit(&bars->s_full);
-        }
-        // dQ += dS K_j, then the next dP (over dS, in issue order).
-        if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteBwdDsReady)) { ok = false; break; }
+      bool ok = true;
+      int it = 0;  // key tiles processed so far (continues across items)
+      BwdItem item;
+      for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
+        QuerySched<CAUSAL, SPARSE> sch{item.tile, p.n_tiles, p.tile_mask};
+        if (!mbar_wait(&bars->q_full, kk & 1, wc, kSiteBwdKV)) { ok = false; break; }
         tc_fence_after();
-        mma_tile_tn<D>(tmem + Cfg::kQTmDQ, tmem + Cfg::kQTmDP, aK + st * Cfg::kTileBytes, it > 0);
-        mma_commit(&bars->kv_empty[st]);
-        if (jn >= 0) {
-          mma_tile_nt<D>(tmem + Cfg::kQTmDP, aDO, aV + stn * Cfg::kTileBytes);
+        int jj = sch.first();
+        if (jj < 0) mma_commit(&bars->q_empty);
+        if (jj >= 0) {
+          if (!mbar_wait(&bars->kv_full[it & 1], (it >> 1) & 1, wc, kSiteBwdTFull)) { ok = false; break; }
+          tc_fence_after();
+          mma_tile_nt<D>(tmem + Cfg::kQTmS, aQ, aK + (it & 1) * Cfg::kTileBytes);
+          mma_commit(&bars->s_full);
+          mma_tile_nt<D>(tmem + Cfg::kQTmDP, aDO, aV + (it & 1) * Cfg::kTileBytes);
           mma_commit(&bars->dp_full);
         }
-        jj = jn;
-        ++it;
+        bool first = true;
+        while (jj >= 0) {
+          const int st = it & 1;
+          const int jn = sch.next(jj);
+          const int stn = (it + 1) & 1;
+          const uint32_t phn = ((it + 1) >> 1) & 1;
+          // All S and dP products of this item are issued: Q_i, dO_i free when done.
+          if (jn < 0) mma_commit(&bars->q_empty);
+          // Next S as soon as both warpgroups have read this one.
+          if (jn >= 0) {
+            if (!mbar_wait(&bars->s_read, it & 1, wc, kSiteBwdSRead)) { ok = false; break; }
+            if (!mbar_wait(&bars->kv_full[stn], phn, wc, kSiteBwdTFull)) { ok = false; break; }
+            tc_fence_after();
+            mma_tile_nt<D>(tmem + Cfg::kQTmS, aQ, aK + stn * Cfg::kTileBytes);
+            mma_commit(&bars->s_full);
+          }
+          // dQ += dS K_j, then the next dP (over dS, in issue order). The first dQ
+          // product of an item overwrites the accumulator: the previous item's
+          // epilogue must have read it.
+          if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteBwdDsReady)) { ok = false; break; }
+          if (first && kk > 0 && !mbar_wait(&bars->acc_empty, (kk - 1) & 1, wc, kSiteBwdAcc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_tn<D>(tmem + Cfg::kQTmDQ, tmem + Cfg::kQTmDP, aK + st * Cfg::kTileBytes, !first);
+          mma_commit(&bars->kv_empty[st]);
+          if (jn >= 0) {
+            mma_tile_nt<D>(tmem + Cfg::kQTmDP, aDO, aV + stn * Cfg::kTileBytes);
+            mma_commit(&bars->dp_full);
+          }
+          first = false;
+          jj = jn;
+          ++it;
+        }
+        if (!ok) break;
+        mma_commit(&bars->acc_done);
       }
-      if (ok) mma_commit(&bars->acc_done);
       mma_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0, wc, kSiteBwdDrain);
     }
@@ -665,75 +777,92 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int r = quarter * 32 + lane;  // query row within tile i
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;
-    const size_t row = size_t(bh) * p.N + size_t(i) * 128 + r;
-    const float l2 = p.lse2[row];
-    const float Dv = p.Drow[row];
     bool ok = true;
-    int it = 0;
-    for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const bool diag = CAUSAL && (jj == i);  // key c visible to query r iff c <= r
-      uint32_t pk[32];
-      {
-        uint32_t raw[64];
-        tmem_ld64(trow + Cfg::kQTmS + h * 64, raw);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars->s_read);
-        const uint64_t c2v = f2(c2, c2), nl2 = f2(l2, l2);  // l2 = -lse log2 e
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          uint64_t pv = ex2_split_x2<PolyShare<D>::kPer8>(
-              f2_fma(f2(__uint_as_float(raw[2 * t]), __uint_as_float(raw[2 * t + 1])), c2v, nl2), t);
-          if (diag) {
-            const float2 v = f2_split(pv);
-            pv = f2((h * 64 + 2 * t > r) ? 0.f : v.x, (h * 64 + 2 * t + 1 > r) ? 0.f : v.y);
-          }
-          const float2 v = f2_split(pv);
-          pk[t] = pack_bf16(v.x, v.y);
-        }
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, wc, kSiteBwdDpFull))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      {
-        uint32_t dpr[64];
-        tmem_ld64(trow + Cfg::kQTmDP + h * 64, dpr);
-        tmem_wait_ld();
-        mbar_arrive(&bars->rd_dp);
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
+    int it = 0;  // key tiles processed so far (continues across items)
+    BwdItem item;
+    for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
+      const int i = item.tile;
+      QuerySched<CAUSAL, SPARSE> sch{i, p.n_tiles, p.tile_mask};
+      const size_t row = size_t(item.bh) * p.N + size_t(i) * 128 + r;
+      const float l2 = p.lse2[row];
+      const float Dv = p.Drow[row];
+      int local = 0;
+      for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it, ++local) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
           ok = false;
           break;
         }
-        const uint64_t dv2 = f2(Dv, Dv);
-        uint32_t ds[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float2 pp = unpack_bf16(pk[t]);
-          const uint64_t diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), dv2);
-          const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
-          ds[t] = pack_bf16(v.x, v.y);
-        }
-        tmem_st32(trow + Cfg::kQTmDP + h * 32, ds);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->ds_ready);
-    }
-    // ---------------------------------------------------------- epilogue: dQ columns [h D/2, (h+1) D/2)
-    if (ok) {
-      const bool any = it > 0;
-      if (any) ok = __all_sync(0xffffffffu, mbar_wait(&bars->acc_done, 0, wc, kSiteBwdAcc));
-      if (ok) {
         tc_fence_after();
-        store_row_bf16<D / 2>(p.dq + row * D + h * (D / 2), trow + Cfg::kQTmDQ + h * (D / 2), p.scale, !any);
+        const bool diag = CAUSAL && (jj == i);  // key c visible to query r iff c <= r
+        uint32_t pk[32];
+        {
+          uint32_t raw[64];
+          tmem_ld64(trow + Cfg::kQTmS + h * 64, raw);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&bars->s_read);
+          const uint64_t c2v = f2(c2, c2), nl2 = f2(l2, l2);  // l2 = -lse log2 e
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            uint64_t pv = ex2_split_x2<PolyShare<D>::kPer8>(
+                f2_fma(f2(__uint_as_float(raw[2 * t]), __uint_as_float(raw[2 * t + 1])), c2v, nl2), t);
+            if (diag) {
+              const float2 v = f2_split(pv);
+              pv = f2((h * 64 + 2 * t > r) ? 0.f : v.x, (h * 64 + 2 * t + 1 > r) ? 0.f : v.y);
+            }
+            const float2 v = f2_split(pv);
+            pk[t] = pack_bf16(v.x, v.y);
+          }
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, wc, kSiteBwdDpFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        {
+          uint32_t dpr[64];
+          tmem_ld64(trow + Cfg::kQTmDP + h * 64, dpr);
+          tmem_wait_ld();
+          mbar_arrive(&bars->rd_dp);
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
+            ok = false;
+            break;
+          }
+          const uint64_t dv2 = f2(Dv, Dv);
+          uint32_t ds[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float2 pp = unpack_bf16(pk[t]);
+            const uint64_t diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), dv2);
+            const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
+            ds[t] = pack_bf16(v.x, v.y);
+          }
+          tmem_st32(trow + Cfg::kQTmDP + h * 32, ds);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->ds_ready);
       }
+      if (!ok) break;
+      // -------------------------------------------------------- epilogue: dQ columns [h D/2, (h+1) D/2)
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_done, kk & 1, wc, kSiteBwdAcc))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t acc[D / 2];
+      if (local > 0) {
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc)
+          tmem_ld32(trow + Cfg::kQTmDQ + h * (D / 2) + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[cc * 32]));
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int t = 0; t < D / 2; ++t) acc[t] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty);
+      store_regs_bf16<D / 2>(p.dq + row * D + h * (D / 2), acc, p.scale);
     }
     tc_fence_before();
     __syncthreads();

@@ -88,19 +88,17 @@ struct FwdBars {
 };
 
 // Persistent schedule: the k-th work item of this CTA, or false when it has none.
-// Rounds of gridDim.x items are dealt to the CTAs alternately forwards and backwards.
-// Item order: with all items equal (no causal mask) head-major, so the query blocks
-// of one head run together and share its K/V tiles through L2; with the causal mask
-// the cost of a block grows with its index, so items go longest first across all
-// heads (block-major), which with the alternating deal balances the CTAs' work.
+// Without the causal mask all items cost the same and go head-major (the query blocks
+// of one head together, sharing its K/V tiles through L2). With it, a block's cost
+// grows with its index, and items go longest first across all heads (block-major),
+// which with the alternating deal of item_position balances the CTAs' work.
 struct FwdItem {
   int bh, qb;
 };
 template <bool CAUSAL>
 __device__ __forceinline__ bool fwd_item(int n_items, int n_qblocks, int BH, int k, FwdItem& it) {
-  const int G = gridDim.x, c = blockIdx.x;
-  const long long pos = static_cast<long long>(k) * G + ((k & 1) ? (G - 1 - c) : c);
-  if (pos >= n_items) return false;
+  const long long pos = item_position(n_items, k);
+  if (pos < 0) return false;
   if (CAUSAL) {
     it.qb = n_qblocks - 1 - static_cast<int>(pos / BH);
     it.bh = static_cast<int>(pos % BH);

@@ -280,6 +280,17 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------------------------ persistent schedules
+
+// Position of this CTA's k-th work item in the global item order, or -1 when it has
+// none: rounds of gridDim.x positions are dealt alternately forwards and backwards,
+// so a CTA that drew a costly item in one round draws a cheap one in the next.
+__device__ __forceinline__ long long item_position(long long n_items, int k) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const long long pos = static_cast<long long>(k) * G + ((k & 1) ? (G - 1 - c) : c);
+  return pos < n_items ? pos : -1;
+}
+
 // ------------------------------------------------------------------ math helpers
 
 __device__ __forceinline__ float ex2(float x) {

@@ -1,4 +1,4 @@
-"""GPU parity of the backward path (pre-processing, main kernel, dQ conversion),
+"""GPU parity of the backward path (pre-processing, dK/dV kernel, dQ kernel),
 called through the C ABI, against the fp64 oracle."""
 import math
 
@@ -169,3 +169,21 @@ def test_sweep_points(cuda_device, N, d):
         t, (dq, dk, dv), _ = _full_check(B, H, N, d, causal, cuda_device, do_scale=0.5,
                                           heads=[(0, 0), (B - 1, H - 1)])
         _invariants(t, dk, dv)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_many_items_per_cta(cuda_device, causal, d):
+    """More (tile, head) items than SMs: each persistent CTA of both backward
+    kernels runs several, with an odd tile count."""
+    _full_check(2, 80, 640, d, causal, cuda_device, seed=51 + d)
+
+
+def test_many_items_blocksparse(cuda_device):
+    N = 768
+    mask = make_tile_mask(N // 128, seed=11, density=0.4)
+    mask[2, :] = 0
+    mask[:, 3] = 0
+    t, (dq, dk, dv), _ = _full_check(1, 160, N, 64, False, cuda_device, seed=53, mask=mask)
+    assert torch.all(dq[:, :, 256:384] == 0)
+    assert torch.all(dk[:, :, 384:512] == 0) and torch.all(dv[:, :, 384:512] == 0)
