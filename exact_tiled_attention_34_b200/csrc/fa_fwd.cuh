@@ -155,23 +155,22 @@ enum FwdSite : int {
 template <bool DIAG, int POLY8>
 __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, float m, uint32_t tp, float& sum,
                                             float& alpha, float& m_use) {
+  // Four independent accumulators keep the reduction chains short.
   float mx;
   if (c >= 0.f) {
-    float a0 = -INFINITY, a1 = -INFINITY;
+    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int t = 0; t < 128; t += 4) {
-      a0 = max3f(a0, (DIAG && t > r) ? -INFINITY : s[t], (DIAG && t + 1 > r) ? -INFINITY : s[t + 1]);
-      a1 = max3f(a1, (DIAG && t + 2 > r) ? -INFINITY : s[t + 2], (DIAG && t + 3 > r) ? -INFINITY : s[t + 3]);
-    }
-    mx = fmaxf(a0, a1) * c;
+    for (int t = 0; t < 128; t += 2)
+      a[(t >> 1) & 3] = max3f(a[(t >> 1) & 3], (DIAG && t > r) ? -INFINITY : s[t],
+                              (DIAG && t + 1 > r) ? -INFINITY : s[t + 1]);
+    mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * c;
   } else {
-    float a0 = INFINITY, a1 = INFINITY;
+    float a[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
 #pragma unroll
-    for (int t = 0; t < 128; t += 4) {
-      a0 = min3f(a0, (DIAG && t > r) ? INFINITY : s[t], (DIAG && t + 1 > r) ? INFINITY : s[t + 1]);
-      a1 = min3f(a1, (DIAG && t + 2 > r) ? INFINITY : s[t + 2], (DIAG && t + 3 > r) ? INFINITY : s[t + 3]);
-    }
-    mx = fminf(a0, a1) * c;
+    for (int t = 0; t < 128; t += 2)
+      a[(t >> 1) & 3] = min3f(a[(t >> 1) & 3], (DIAG && t > r) ? INFINITY : s[t],
+                              (DIAG && t + 1 > r) ? INFINITY : s[t + 1]);
+    mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * c;
   }
   const float m_new = fmaxf(m, mx);
   const bool rescale = __any_sync(0xffffffffu, m_new > m + 8.f);
@@ -179,7 +178,7 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, flo
   const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
   alpha = ex2(m - m_sub);  // 0 on the first tile (m = -inf), 1 when the max is kept
   const uint64_t c2 = f2(c, c), nm2 = f2(-m_sub, -m_sub);
-  uint64_t acc = f2(0.f, 0.f);
+  uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t pk[32];
@@ -192,22 +191,22 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, flo
         const float2 v = f2_split(pv);
         pv = f2((c0 > r) ? 0.f : v.x, (c0 + 1 > r) ? 0.f : v.y);
       }
-      acc = f2_add(acc, pv);
+      acc[t & 3] = f2_add(acc[t & 3], pv);
       const float2 v = f2_split(pv);
       pk[t] = pack_bf16(v.x, v.y);
     }
     tmem_st32(tp + h * 32, pk);
   }
-  const float2 a = f2_split(acc);
+  const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
   sum = a.x + a.y;
 }
 
 // Register split of the 384-thread forward block (launched with 168 per thread,
-// 64,512 in all): the producer/MMA warpgroup drops to 80, the two softmax
-// warpgroups rise to 200 -> 128 * (80 + 2 * 200) = 61,440. Only the softmax
+// 64,512 in all): the producer/MMA warpgroup drops to 104, the two softmax
+// warpgroups rise to 184 -> 128 * (104 + 2 * 184) = 60,416. Only the softmax
 // warpgroups increase, once, by less than the first warpgroup releases.
-constexpr int kFwdRegsCtl = 80;
-constexpr int kFwdRegsSoftmax = 200;
+constexpr int kFwdRegsCtl = 104;
+constexpr int kFwdRegsSoftmax = 184;
 constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 
 template <int D, bool CAUSAL, bool SPARSE>
