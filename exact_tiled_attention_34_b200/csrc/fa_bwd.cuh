@@ -509,7 +509,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int t = 0; t < 32; ++t) {
             const int c0 = 2 * t;
             const float2 nl = *reinterpret_cast<const float2*>(lse2 + c0);  // -lse log2 e
-            uint64_t pv = ex2_split_x2<PolyShare<D>::kPer8>(
+            uint64_t pv = ex2_split_x2<PolyShare<D>::kDkdv>(
                 f2_fma(f2(__uint_as_float(raw[c0]), __uint_as_float(raw[c0 + 1])), c2v, f2(nl.x, nl.y)), t);
             if (diag) {
               const float2 v = f2_split(pv);
@@ -804,7 +804,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const uint64_t c2v = f2(c2, c2), nl2 = f2(l2, l2);  // l2 = -lse log2 e
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
-            uint64_t pv = ex2_split_x2<PolyShare<D>::kPer8>(
+            uint64_t pv = ex2_split_x2<PolyShare<D>::kDq>(
                 f2_fma(f2(__uint_as_float(raw[2 * t]), __uint_as_float(raw[2 * t + 1])), c2v, nl2), t);
             if (diag) {
               const float2 v = f2_split(pv);

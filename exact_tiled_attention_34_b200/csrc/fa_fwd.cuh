@@ -460,9 +460,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           tmem_wait_ld();
           float sum, alpha, m_use;
           if (CAUSAL && j == tile)
-            softmax_row<true, PolyShare<D>::kPer8>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+            softmax_row<true, PolyShare<D>::kFwd>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
           else
-            softmax_row<false, PolyShare<D>::kPer8>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+            softmax_row<false, PolyShare<D>::kFwd>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
           const bool rescale = m_use != m;
           l = l * alpha + sum;
           if (__any_sync(0xffffffffu, rescale) && local > 0) {

@@ -385,11 +385,15 @@ __device__ __forceinline__ uint64_t ex2_mufu_x2(uint64_t x) {
 }
 
 // Which column pairs use the polynomial: pairs t with (t mod 8) < POLY8. Called from
-// fully unrolled loops, so the choice is made at compile time. (Measured on B200: 3 of
-// 8 beats 5 of 8 at head dim 64, where more polynomial work costs issue slots.)
+// fully unrolled loops, so the choice is made at compile time. The shares were chosen
+// by timing every value from 0 to 5 of 8 on B200 (same GPU, same run): the polynomial
+// pays only where MUFU limits the softmax (forward at head dim 64); elsewhere its
+// extra instructions cost more than the MUFU time they save.
 template <int D>
 struct PolyShare {
-  static constexpr int kPer8 = 3;
+  static constexpr int kFwd = (D == 64) ? 2 : 0;
+  static constexpr int kDkdv = 1;
+  static constexpr int kDq = 0;
 };
 template <int POLY8>
 __device__ __forceinline__ uint64_t ex2_split_x2(uint64_t x, int t) {
