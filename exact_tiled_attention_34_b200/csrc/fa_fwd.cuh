@@ -109,7 +109,10 @@ __device__ __forceinline__ bool fwd_item(int n_items, int n_qblocks, int BH, int
   return true;
 }
 
-// Which of the CTA's two Q tiles need K/V tile j (bit 0: tile 0, bit 1: tile 1).
+// Which of the CTA's two Q tiles need K/V tile j (bit 0: tile 0, bit 1: tile 1); the
+// K/V tiles are visited in increasing order. (Visiting the causal tiles diagonal-first,
+// or tile 1's extra diagonal tile earlier, was measured: up to 6% faster at N = 2048 but
+// 1-2% slower at N >= 8192, so the plain order stays.)
 template <bool CAUSAL, bool SPARSE>
 struct FwdSched {
   int t0, t1;
@@ -126,7 +129,7 @@ struct FwdSched {
     }
     return (k0 ? 1u : 0u) | (k1 ? 2u : 0u);
   }
-  // Next j > j0 with a non-empty bit set (or -1).
+  // The K/V tile visited after j0 with a non-empty bit set (or -1).
   __device__ __forceinline__ int next(int j0, uint32_t& b) const {
     const int jl = last();
     for (int j = j0 + 1; j <= jl; ++j) {
@@ -136,6 +139,7 @@ struct FwdSched {
     b = 0;
     return -1;
   }
+  __device__ __forceinline__ int first(uint32_t& b) const { return next(-1, b); }
 };
 
 // Wait-site codes reported through the status word (detail field).
@@ -288,7 +292,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         sch.t1 * 128, item.bh);
         ++nq;
         uint32_t b;
-        for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b), ++it) {
+        for (int j = sch.first(b); j >= 0; j = sch.next(j, b), ++it) {
           const int st = it % S;
           const int n = it / S;
           if (n > 0 && !mbar_wait(&bars->kv_empty[st], (n - 1) & 1, wc, kSiteFwdKvEmpty)) {
@@ -355,7 +359,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint32_t issued = 0;
         bool first_pv[2] = {true, true};
         uint32_t b = 0, bn = 0;
-        int j = sch.next(-1, b);
+        int j = sch.first(b);
         if (j < 0) mma_commit(&bars->q_empty);  // nothing to do for this block
         while (j >= 0) {
           const int st = it % S;
@@ -370,6 +374,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int i = 0; i < 2; ++i)
               if (need & (1u << i)) {
                 issue_s(i, st);
+                mma_commit(&bars->s_full[i]);
+              }
+          }
+          // With a block mask the two Q tiles often need different K/V tiles: a tile with
+          // no work on this K/V tile but some on the next one gets its next S now, so
+          // that its softmax overlaps the other tile's (measured +17% at 25% density).
+          // Without a mask both tiles need every K/V tile, and with the causal mask only
+          // the last K/V tile of a block is for one tile alone.
+          const uint32_t ahead = (SPARSE && jn >= 0) ? (bn & ~b) : 0u;
+          if (ahead) {
+            if (!mbar_wait(&bars->k_full[stn], phn, wc, kSiteFwdKFull)) { ok = false; break; }
+            tc_fence_after();
+            for (int i = 0; i < 2; ++i)
+              if (ahead & (1u << i)) {
+                issue_s(i, stn);
                 mma_commit(&bars->s_full[i]);
               }
           }
@@ -401,7 +420,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
           if (!ok) break;
           mma_commit(&bars->kv_empty[st]);
-          issued = next_issued;
+          issued = next_issued | ahead;
           b = bn;
           j = jn;
           ++it;
@@ -442,7 +461,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       int local = 0;  // tiles of this item
       if (active) {
         uint32_t b;
-        for (int j = sch.next(-1, b); j >= 0; j = sch.next(j, b)) {
+        for (int j = sch.first(b); j >= 0; j = sch.next(j, b)) {
           if (!(b & (1u << i))) continue;
           if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], cnt & 1, wc, kSiteFwdSFull))) {
             ok = false;
