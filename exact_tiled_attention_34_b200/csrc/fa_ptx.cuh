@@ -280,6 +280,36 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------------------------ row stores
+
+// Stores the calling warp's 32 rows (lane = row) of 2 * NW bf16 values, given as NW
+// packed words per lane, to global rows row0 + lane * ld (ld in elements). Each lane's
+// words go through `stage` (32 * NW words of this warp's shared memory, 16-byte
+// aligned) so that every global store instruction writes 32 / (NW / 4) whole rows of
+// NW * 4 bytes instead of 32 scattered 16-byte pieces. The 16-byte chunks of a row are
+// rotated by the row index in the stage, which keeps both passes free of bank
+// conflicts. NW is 16 or 32.
+template <int NW>
+__device__ __forceinline__ void warp_store_rows(uint32_t* stage, const uint32_t (&w)[NW], __nv_bfloat16* row0,
+                                                size_t ld) {
+  constexpr int kCpr = NW / 4;       // 16-byte chunks per row
+  constexpr int kRpi = 32 / kCpr;    // rows per store instruction
+  const int lane = static_cast<int>(lane_id());
+  uint4* st4 = reinterpret_cast<uint4*>(stage);
+#pragma unroll
+  for (int c = 0; c < kCpr; ++c)
+    st4[lane * kCpr + (c ^ (lane & (kCpr - 1)))] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+  __syncwarp();
+  const int c = lane & (kCpr - 1);
+#pragma unroll
+  for (int k = 0; k < kCpr; ++k) {
+    const int row = k * kRpi + lane / kCpr;
+    const uint4 v = st4[row * kCpr + (c ^ (row & (kCpr - 1)))];
+    *reinterpret_cast<uint4*>(row0 + size_t(row) * ld + c * 8) = v;
+  }
+  __syncwarp();  // the stage may be rewritten after this
+}
+
 // ------------------------------------------------------------------ persistent schedules
 
 // Position of this CTA's k-th work item in the global item order, or -1 when it has
