@@ -11,7 +11,7 @@ is missing or a tensor is not a CUDA tensor, the call raises.
     dq, dk, dv = backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None)
 
 Tensors are bf16 [B, H, N, d] contiguous on one CUDA device; lse is fp32 [B, H, N];
-tile_mask is uint8 [N/128, N/128] on the same device. N % 128 == 0, d in {64, 128}.
+tile_mask is uint8 [ceil(N/128), ceil(N/128)] on the same device. Any N >= 1, d in {64, 128}.
 """
 from __future__ import annotations
 
@@ -134,7 +134,7 @@ def _check_mask(tile_mask, q, mask_block):
     import torch
     if tile_mask.dtype != torch.uint8 or not tile_mask.is_contiguous() or tile_mask.device != q.device:
         raise ValueError("tile_mask must be a contiguous uint8 tensor on the device of q")
-    nt = q.shape[2] // mask_block
+    nt = -(-q.shape[2] // mask_block)  # ceil: a partial last tile has its own mask entry
     if tuple(tile_mask.shape) != (nt, nt):
         raise ValueError(f"tile_mask must be [{nt}, {nt}]")
 

@@ -29,8 +29,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 fa_status check_sizes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
-  const long long rows = static_cast<long long>(B) * H * N;
+  // Padded rows (N rounded up to whole 128-row tiles) index the backward's row arrays.
+  const long long rows = static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128 * 128);
   if (rows > INT_MAX || static_cast<long long>(B) * H > INT_MAX / 2) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
@@ -165,7 +165,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.timeout_ns = kTimeoutNs;
   p.N = N;
   p.BH = BH;
-  p.n_tiles = N / 128;
+  p.n_tiles = (N + 127) / 128;
   p.n_qblocks = (p.n_tiles + 1) / 2;
   p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
@@ -183,10 +183,11 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 
-// Workspace: fp32 D rows [BH*N], then fp32 lse*log2(e) rows [BH*N], each 256-aligned.
+// Workspace: fp32 D rows, then fp32 -lse*log2(e) rows, each [BH * Npad] (Npad = N
+// rounded up to a multiple of 128) and 256-aligned.
 size_t bwd_ws_bytes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
-  const size_t rows = size_t(B) * H * N;
+  const size_t rows = size_t(B) * H * ((size_t(N) + 127) / 128 * 128);
   return 2 * round256(rows * 4);
 }
 
@@ -237,7 +238,8 @@ fa_status launch_dq(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
 
 struct BwdArgs {
   int BH;
-  size_t rows;
+  int Npad;     // N rounded up to a multiple of 128
+  size_t rows;  // BH * Npad
   float* Drow;
   float* lse2;
 };
@@ -250,7 +252,8 @@ fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d,
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
   if (ws_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
   a->BH = B * H;
-  a->rows = size_t(a->BH) * N;
+  a->Npad = (N + 127) / 128 * 128;
+  a->rows = size_t(a->BH) * a->Npad;
   a->Drow = static_cast<float*>(const_cast<void*>(ws));
   a->lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(const_cast<void*>(ws)) + round256(a->rows * 4));
   return FA_OK;
@@ -267,10 +270,11 @@ fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, siz
   const unsigned grid = unsigned((threads + 255) / 256);
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
+  const long long rows = static_cast<long long>(a.rows);
   if (d == 64)
-    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, static_cast<long long>(a.rows));
+    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, rows);
   else
-    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, static_cast<long long>(a.rows));
+    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, rows);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -307,7 +311,7 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.timeout_ns = kTimeoutNs;
   p.N = N;
   p.BH = a.BH;
-  p.n_tiles = N / 128;
+  p.n_tiles = (N + 127) / 128;
   p.scale = scale;
 #define FA_BWD_DISPATCH(LAUNCH)                                                                  \
   if (mask)                                                                                      \

@@ -42,18 +42,26 @@ namespace fa {
 // ---------------------------------------------------------------- pre-processing
 
 // D[row] = sum_c dO[row, c] O[row, c] and nl2[row] = -lse[row] log2(e) (fp32), so
-// that the exponent of the recomputed P is one fused multiply-add: s c + nl2.
+// that the exponent of the recomputed P is one fused multiply-add: s c + nl2. The two
+// row arrays hold Npad = 128 * ceil(N / 128) rows per (batch, head): a tile's rows are
+// one 512-byte run. The pad rows of the last tile (n >= N, when N % 128 != 0) get
+// D = 0 and nl2 = -inf, so their recomputed P is 0 and they add nothing to dK or dV.
 // D / 8 threads per row, 16 bytes each.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse, float* __restrict__ Drow,
-                                                         float* __restrict__ lse2, long long rows) {
+                                                         float* __restrict__ lse2, int N, int Npad,
+                                                         long long rows_pad) {
   constexpr int TPR = D / 8;
   const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = g / TPR;
+  const long long prow = g / TPR;  // padded row index: bh * Npad + n
   const int part = static_cast<int>(g % TPR);
-  const bool valid = row < rows;
+  const bool inrange = prow < rows_pad;
+  const long long bh = prow / Npad;
+  const int n = static_cast<int>(prow - bh * Npad);
+  const bool valid = inrange && n < N;
+  const long long row = bh * N + n;  // row of O, dO and lse
   float s = 0.f;
   if (valid) {
     const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
@@ -70,26 +78,26 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   }
 #pragma unroll
   for (int w = TPR / 2; w > 0; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
-  if (valid && part == 0) {
-    Drow[row] = s;
-    lse2[row] = -lse[row] * 1.4426950408889634f;
+  if (inrange && part == 0) {
+    Drow[prow] = s;
+    lse2[prow] = valid ? -lse[row] * 1.4426950408889634f : -INFINITY;
   }
 }
 
 // ---------------------------------------------------------------- common
 
 struct BwdParams {
-  const float* lse2;    // [BH, N] -lse * log2(e)
-  const float* Drow;    // [BH, N]
+  const float* lse2;    // [BH, Npad] -lse * log2(e) (Npad = 128 * n_tiles; pad rows -inf)
+  const float* Drow;    // [BH, Npad]
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;
   unsigned long long timeout_ns;
-  int N;
+  int N;                // sequence length (any N >= 1)
   int BH;
-  int n_tiles;
+  int n_tiles;          // ceil(N / 128)
   float scale;          // softmax scale
 };
 
@@ -375,7 +383,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tma_load_3d_hint(sDO + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_do, &bars->t_full[st],
                              cb * 64, i * 128, bh, keep);
           }
-          const size_t roff = size_t(bh) * p.N + size_t(i) * 128;
+          const size_t roff = (size_t(bh) * p.n_tiles + size_t(i)) * 128;  // padded row arrays
           bulk_load(sL + st * 128, p.lse2 + roff, 512, &bars->t_full[st]);
           bulk_load(sDr + st * 128, p.Drow + roff, 512, &bars->t_full[st]);
         }
@@ -576,7 +584,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
-      store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * D, acc, h == 0 ? p.scale : 1.f);
+      if (j * 128 + r < p.N)  // key rows past N (last tile, N % 128 != 0) do not exist
+        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * D, acc, h == 0 ? p.scale : 1.f);
     }
     tc_fence_before();
     __syncthreads();
@@ -784,8 +793,9 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int i = item.tile;
       QuerySched<CAUSAL, SPARSE> sch{i, p.n_tiles, p.tile_mask};
       const size_t row = size_t(item.bh) * p.N + size_t(i) * 128 + r;
-      const float l2 = p.lse2[row];
-      const float Dv = p.Drow[row];
+      const size_t prow = (size_t(item.bh) * p.n_tiles + size_t(i)) * 128 + r;  // padded row arrays
+      const float l2 = p.lse2[prow];
+      const float Dv = p.Drow[prow];
       int local = 0;
       for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it, ++local) {
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
@@ -862,7 +872,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
-      store_regs_bf16<D / 2>(p.dq + row * D + h * (D / 2), acc, p.scale);
+      if (i * 128 + r < p.N)  // query rows past N (last tile, N % 128 != 0) do not exist
+        store_regs_bf16<D / 2>(p.dq + row * D + h * (D / 2), acc, p.scale);
     }
     tc_fence_before();
     __syncthreads();

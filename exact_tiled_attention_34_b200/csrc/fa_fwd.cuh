@@ -40,9 +40,9 @@ struct FwdParams {
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;               // library status word (global)
   unsigned long long timeout_ns;
-  int N;                     // sequence length (multiple of 128)
+  int N;                     // sequence length (any N >= 1)
   int BH;                    // B * H
-  int n_tiles;               // N / 128
+  int n_tiles;               // ceil(N / 128); the last tile holds N - 128 (n_tiles - 1) rows
   int n_qblocks;             // ceil(n_tiles / 2)
   int n_items;               // n_qblocks * BH work items (query block, batch*head)
   float c_log2;              // scale * log2(e)
@@ -160,9 +160,11 @@ enum FwdSite : int {
 // reference max m_use. The rescale decision is warp-uniform (see the file header).
 // Pairs of columns go through packed f32x2 arithmetic; the exponentials are split
 // between the special-function unit and a polynomial on the FMA pipe.
-// DIAG: the tile on the causal diagonal; column t is visible iff t <= r.
-template <bool DIAG, int POLY8>
-__device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, float m, uint32_t tp, float& sum,
+// MASK: only columns t < lim are visible, for the tile on the causal diagonal
+// (lim = r + 1) or the last K/V tile of a sequence whose length is not a multiple of
+// 128 (lim = number of keys in it).
+template <bool MASK, int POLY8>
+__device__ __forceinline__ void softmax_row(float (&s)[128], int lim, float c, float m, uint32_t tp, float& sum,
                                             float& alpha, float& m_use) {
   // Four independent accumulators keep the reduction chains short.
   float mx;
@@ -170,15 +172,15 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, flo
     float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int t = 0; t < 128; t += 2)
-      a[(t >> 1) & 3] = max3f(a[(t >> 1) & 3], (DIAG && t > r) ? -INFINITY : s[t],
-                              (DIAG && t + 1 > r) ? -INFINITY : s[t + 1]);
+      a[(t >> 1) & 3] = max3f(a[(t >> 1) & 3], (MASK && t >= lim) ? -INFINITY : s[t],
+                              (MASK && t + 1 >= lim) ? -INFINITY : s[t + 1]);
     mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * c;
   } else {
     float a[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
 #pragma unroll
     for (int t = 0; t < 128; t += 2)
-      a[(t >> 1) & 3] = min3f(a[(t >> 1) & 3], (DIAG && t > r) ? INFINITY : s[t],
-                              (DIAG && t + 1 > r) ? INFINITY : s[t + 1]);
+      a[(t >> 1) & 3] = min3f(a[(t >> 1) & 3], (MASK && t >= lim) ? INFINITY : s[t],
+                              (MASK && t + 1 >= lim) ? INFINITY : s[t + 1]);
     mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * c;
   }
   const float m_new = fmaxf(m, mx);
@@ -196,9 +198,9 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int r, float c, flo
       const int c0 = h * 64 + 2 * t;
       const uint64_t x = f2_fma(f2(s[c0], s[c0 + 1]), c2, nm2);
       uint64_t pv = ex2_split_x2<POLY8>(x, t);
-      if (DIAG) {
+      if (MASK) {
         const float2 v = f2_split(pv);
-        pv = f2((c0 > r) ? 0.f : v.x, (c0 + 1 > r) ? 0.f : v.y);
+        pv = f2((c0 >= lim) ? 0.f : v.x, (c0 + 1 >= lim) ? 0.f : v.y);
       }
       acc[t & 3] = f2_add(acc[t & 3], pv);
       const float2 v = f2_split(pv);
@@ -484,10 +486,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
           tmem_wait_ld();
           float sum, alpha, m_use;
-          if (CAUSAL && j == tile)
-            softmax_row<true, PolyShare<D>::kFwd>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+          // Masked columns: above the diagonal (causal), or keys past N in the last
+          // K/V tile (with the causal mask those are above the diagonal of every row
+          // that exists). The choice of variant is per tile, so warp-uniform.
+          const bool diag = CAUSAL && j == tile;
+          const bool tail = !CAUSAL && j == p.n_tiles - 1 && (p.N & 127) != 0;
+          if (diag || tail)
+            softmax_row<true, PolyShare<D>::kFwd>(s, diag ? r + 1 : p.N - 128 * j, c, m, trow + Cfg::tm_p(i), sum,
+                                                  alpha, m_use);
           else
-            softmax_row<false, PolyShare<D>::kFwd>(s, r, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+            softmax_row<false, PolyShare<D>::kFwd>(s, 128, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
           const bool rescale = m_use != m;
           l = l * alpha + sum;
           if (__any_sync(0xffffffffu, rescale) && local > 0) {
@@ -520,6 +528,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_after();
       const size_t row = size_t(item.bh) * p.N + size_t(tile) * 128 + r;
       __nv_bfloat16* orow = p.o + row * D;
+      const bool row_ok = tile * 128 + r < p.N;  // rows past N (last tile) do not exist
       if (active && local > 0) {
         const float inv_l = 1.f / l;
         uint32_t ov[D];
@@ -539,9 +548,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int t = 0; t < 32; ++t)
               w[t] = pack_bf16(__uint_as_float(ov[cb * 64 + 2 * t]) * inv_l,
                                __uint_as_float(ov[cb * 64 + 2 * t + 1]) * inv_l);
-            warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, D);
+            warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, D, p.N - (tile * 128 + r - lane));
           }
-        } else {
+        } else if (row_ok) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint4 pk[4];
@@ -555,10 +564,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int t = 0; t < 4; ++t) dst[t] = pk[t];
           }
         }
-        p.lse[row] = (m + __log2f(l)) * 0.69314718055994531f;
+        if (row_ok) p.lse[row] = (m + __log2f(l)) * 0.69314718055994531f;
       } else {
         mbar_arrive(&bars->o_empty[i]);
-        if (active) {
+        if (active && row_ok) {
           // No visible key for this row (only possible with a block mask).
           const uint4 z = make_uint4(0, 0, 0, 0);
           uint4* dst = reinterpret_cast<uint4*>(orow);

@@ -283,7 +283,8 @@ __device__ __forceinline__ void regs_inc() {
 // ------------------------------------------------------------------ row stores
 
 // Stores the calling warp's 32 rows (lane = row) of 2 * NW bf16 values, given as NW
-// packed words per lane, to global rows row0 + lane * ld (ld in elements). Each lane's
+// packed words per lane, to global rows row0 + lane * ld (ld in elements); rows at or
+// past `nrows` are not written (the tail of the last tile). Each lane's
 // words go through `stage` (32 * NW words of this warp's shared memory, 16-byte
 // aligned) so that every global store instruction writes 32 / (NW / 4) whole rows of
 // NW * 4 bytes instead of 32 scattered 16-byte pieces. The 16-byte chunks of a row are
@@ -291,7 +292,7 @@ __device__ __forceinline__ void regs_inc() {
 // conflicts. NW is 16 or 32.
 template <int NW>
 __device__ __forceinline__ void warp_store_rows(uint32_t* stage, const uint32_t (&w)[NW], __nv_bfloat16* row0,
-                                                size_t ld) {
+                                                size_t ld, int nrows) {
   constexpr int kCpr = NW / 4;       // 16-byte chunks per row
   constexpr int kRpi = 32 / kCpr;    // rows per store instruction
   const int lane = static_cast<int>(lane_id());
@@ -305,7 +306,7 @@ __device__ __forceinline__ void warp_store_rows(uint32_t* stage, const uint32_t 
   for (int k = 0; k < kCpr; ++k) {
     const int row = k * kRpi + lane / kCpr;
     const uint4 v = st4[row * kCpr + (c ^ (row & (kCpr - 1)))];
-    *reinterpret_cast<uint4*>(row0 + size_t(row) * ld + c * 8) = v;
+    if (row < nrows) *reinterpret_cast<uint4*>(row0 + size_t(row) * ld + c * 8) = v;
   }
   __syncwarp();  // the stage may be rewritten after this
 }

@@ -28,12 +28,14 @@
  *    a row that sees no key (possible only with a block mask).
  *  - All pointers are DEVICE pointers on the current device, except where noted.
  *    Every base pointer must be 16-byte aligned.
- *  - Supported sizes: B, H, N >= 1; N % 128 == 0; d in {64, 128}. B*H*N must fit
- *    in int32.
+ *  - Supported sizes: B, H, N >= 1 (any N; the kernels work on 128-row tiles and
+ *    the last tile of a sequence may be partial); d in {64, 128}. B*H*Npad must
+ *    fit in int32, where Npad = 128 * ceil(N / 128).
  *  - Causal: key j is visible to query i iff j <= i (top-left aligned; N_q = N_k).
- *  - Block mask (tile_mask): uint8 [N/128, N/128] device array, row-major,
- *    1 = tile kept, 0 = tile skipped, shared by every (b, h). Within a kept tile
- *    every element is visible (the mask is not combined with causal).
+ *  - Block mask (tile_mask): uint8 [nT, nT] device array with nT = ceil(N / 128),
+ *    row-major, 1 = tile kept, 0 = tile skipped, shared by every (b, h); tile t
+ *    covers rows 128 t .. min(128 t + 128, N) - 1. Within a kept tile every
+ *    element is visible (the mask is not combined with causal).
  *  - Ownership: the caller owns every buffer. The library allocates and frees no
  *    device memory on these paths; scratch is caller-provided ("workspace").
  *  - Asynchrony: each call only enqueues work on `stream` (a cudaStream_t, or
@@ -61,7 +63,7 @@ extern "C" {
 typedef enum fa_status {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, non-finite scale */
-  FA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, N % 128 != 0, mask_block != 128 */
+  FA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, sizes beyond int32 rows, mask_block != 128 */
   FA_ERR_ALIGNMENT = 3,       /* a base pointer is not 16-byte aligned */
   FA_ERR_WORKSPACE = 4,       /* workspace too small */
   FA_ERR_CUDA = 5,            /* the CUDA runtime or driver reported an error */
@@ -94,8 +96,9 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
 
 /*
  * Bytes of device scratch that fa_bwd / fa_bwd_blocksparse need for these sizes:
- * two fp32 [B,H,N] row arrays (D_i = sum_c dO_ic O_ic, and lse_i * log2 e), each
- * rounded up to 256 bytes. Returns 0 for non-positive sizes.
+ * two fp32 [B,H,Npad] row arrays (D_i = sum_c dO_ic O_ic, and lse_i * log2 e;
+ * Npad = 128 * ceil(N / 128), so each tile's rows are one run), each rounded up to
+ * 256 bytes: 2 * round_up_256(4 * B*H*Npad). Returns 0 for non-positive sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -163,7 +166,7 @@ fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
  * array compiled into the library: FA_BWD_NOALLOC_SCRATCH_BYTES bytes of device
  * memory on every GPU that loads the library, held until the process exits.
  *  - Sizes: needs fa_bwd_workspace_bytes(B,H,N,d) <= FA_BWD_NOALLOC_SCRATCH_BYTES,
- *    i.e. B*H*N <= 1,048,576 rows (any d); larger sizes return FA_ERR_WORKSPACE
+ *    i.e. B*H*Npad <= 1,048,576 rows (any d); larger sizes return FA_ERR_WORKSPACE
  *    and enqueue nothing.
  *  - Allocation: none. No cudaMalloc, cudaFree or allocating library call.
  *  - Set-up: the first call on a device (with that device current) looks up the

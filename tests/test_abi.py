@@ -57,7 +57,10 @@ def test_fwd_argument_checks(L):
     assert _fwd(L, N=0) == INVALID
     assert _fwd(L, d=32) == UNSUPPORTED
     assert _fwd(L, d=96) == UNSUPPORTED
-    assert _fwd(L, N=130) == UNSUPPORTED
+    # Any N >= 1 passes validation (the last 128-row tile may be partial): such a call
+    # gets as far as a valid one, which on a machine without a GPU is FA_ERR_CUDA.
+    assert _fwd(L, N=130) == _fwd(L, N=128) not in (INVALID, UNSUPPORTED, ALIGN)
+    assert _fwd(L, N=1) == _fwd(L, N=128)
     assert _fwd(L, B=1 << 16, H=1 << 16, N=128) == UNSUPPORTED  # B*H*N beyond int32
     assert _fwd(L, scale=float("nan")) == INVALID
     assert _fwd(L, scale=float("inf")) == INVALID
@@ -74,6 +77,10 @@ def test_workspace_bytes(L):
     up = lambda x: (x + 255) // 256 * 256
     for (B, H, N, d) in ((1, 1, 128, 64), (8, 16, 2048, 64), (2, 16, 8192, 128), (3, 5, 384, 128)):
         rows = B * H * N
+        assert L.fa_bwd_workspace_bytes(B, H, N, d) == 2 * up(rows * 4)
+    # N not a multiple of 128: rows are padded to whole tiles per (batch, head).
+    for (B, H, N, d) in ((1, 1, 1, 64), (2, 3, 130, 128), (1, 16, 2000, 64)):
+        rows = B * H * ((N + 127) // 128 * 128)
         assert L.fa_bwd_workspace_bytes(B, H, N, d) == 2 * up(rows * 4)
     assert L.fa_bwd_workspace_bytes(0, 1, 128, 64) == 0
     assert L.fa_bwd_workspace_bytes(1, 1, -128, 64) == 0
