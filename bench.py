@@ -232,7 +232,7 @@ def cpu_oracle_sample(wl, budget_s: float, seed: int = 0):
                 m = None
                 if dens is not None:
                     if dens not in masks:
-                        masks[dens] = make_tile_mask(N // 128, seed=seed, density=dens).numpy()
+                        masks[dens] = make_tile_mask(-(-N // 128), seed=seed, density=dens).numpy()
                     m = masks[dens]
                 kept = 1.0 if m is None else float(m.sum()) / m.size
                 t0 = time.perf_counter()
@@ -308,7 +308,7 @@ def run_ours(args, wl_name, wl):
     masks = {}
     for (_, _, dens) in wl["variants"]:
         if dens is not None:
-            masks[dens] = make_tile_mask(N // 128, seed=0, density=dens).to(dev)
+            masks[dens] = make_tile_mask(-(-N // 128), seed=0, density=dens).to(dev)
     ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
     outs = {}
     for (label, _, _) in wl["variants"]:
@@ -505,7 +505,8 @@ def run_table(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse"]
+    names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse", "b8h16n2000d64_ragged",
+             "b2h16n8000d128_ragged_causal"]
     names += [f"sweep_N{N}_d{d}{c}" for d in SWEEP_D for N in SWEEP_N for c in ("", "_causal")]
     if args.only:
         names = [n for n in names if any(o in n for o in args.only.split(","))]
@@ -522,7 +523,7 @@ def run_table(args):
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         dq, dk, dv = (torch.empty_like(t["q"]) for _ in range(3))
         for (label, causal, dens) in wl["variants"]:
-            mask = None if dens is None else make_tile_mask(N // 128, seed=0, density=dens).to(dev)
+            mask = None if dens is None else make_tile_mask(-(-N // 128), seed=0, density=dens).to(dev)
             kept = 1.0 if mask is None else float(mask.float().mean())
             F = fwd_flops(B, H, N, d, causal, kept)
 

@@ -24,6 +24,9 @@ WORKLOADS = {
     "b2h16n8192d128_causal": dict(B=2, H=16, N=8192, d=128, causal=(True,), backward=True),
     "b1h16n16384d64_sparse": dict(B=1, H=16, N=16384, d=64, causal=(False,), backward=True,
                                   sparse_density=0.25),
+    # Sequence lengths that are not a multiple of the 128-row tile (last tile partial).
+    "b8h16n2000d64_ragged": dict(B=8, H=16, N=2000, d=64, causal=(False, True), backward=True),
+    "b2h16n8000d128_ragged_causal": dict(B=2, H=16, N=8000, d=128, causal=(True,), backward=True),
 }
 
 SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384)

@@ -22,9 +22,11 @@ Attention with IO-Awareness", method paragraph). The oracle is therefore the
 definition itself; it deliberately does what the method avoids (store S and P).
 
 Masks:
-  * causal: key j is visible to query i iff j <= i (square problems only; the
-    review's "Proposed method" bullet on causal masking gives no formula, and every
-    workload here has N_q = N_k).
+  * causal: key j is visible to query i iff j <= i + (N_k - N_q): the last query
+    sees every key (bottom-right alignment, the usual reading for decoding and for
+    a query block appended to a longer key sequence); for N_q = N_k this is j <= i.
+    The review's "Proposed method" bullet on causal masking gives no formula; the
+    alignment for N_q != N_k is this library's reading.
   * block-sparse: a [ceil(N/T), ceil(N/T)] 0/1 tile mask with T = ``mask_block``
     keeps S_ij iff mask[i // T][j // T] != 0 (the block-sparse paragraph of the
     Stanford summary page; the granularity T = 128 is this library's choice).
@@ -68,13 +70,15 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def _visible(n_q_rows: np.ndarray, n_k: int, causal: bool, block_mask, mask_block: int) -> np.ndarray:
-    """Boolean [len(rows), n_k] visibility for the given absolute query rows."""
+def _visible(n_q_rows: np.ndarray, n_k: int, causal: bool, block_mask, mask_block: int,
+             causal_offset: int = 0) -> np.ndarray:
+    """Boolean [len(rows), n_k] visibility for the given absolute query rows; with the
+    causal mask key j is visible to row i iff j <= i + causal_offset."""
     rows = np.asarray(n_q_rows, dtype=np.int64)
     cols = np.arange(n_k, dtype=np.int64)
     vis = np.ones((rows.shape[0], n_k), dtype=bool)
     if causal:
-        vis &= cols[None, :] <= rows[:, None]
+        vis &= cols[None, :] <= rows[:, None] + causal_offset
     if block_mask is not None:
         bm = np.asarray(block_mask) != 0
         vis &= bm[rows[:, None] // mask_block, cols[None, :] // mask_block]
@@ -82,18 +86,24 @@ def _visible(n_q_rows: np.ndarray, n_k: int, causal: bool, block_mask, mask_bloc
 
 
 def attn_scores_ref(q, k, scale: float, causal: bool = False, block_mask=None,
-                    mask_block: int = 128, rows=None) -> np.ndarray:
-    """Masked, scaled scores S for one head: q [Nq, d], k [N, d] -> [Nq, N] fp64.
+                    mask_block: int = 128, rows=None, n_q=None) -> np.ndarray:
+    """Masked, scaled scores S for one head: q [R, d], k [N_k, d] -> [R, N_k] fp64.
 
-    ``rows`` gives the absolute index of each query row (default 0..Nq-1); masked
-    entries are -inf.
+    ``rows`` gives the absolute index of each query row (default 0..R-1) and ``n_q``
+    the problem's number of query rows N_q (default: R when ``rows`` is not given,
+    else N_k, i.e. sampled rows of a square problem); masked entries are -inf.
     """
     q = _f64(q)
     k = _f64(k)
+    n_k = k.shape[0]
     if rows is None:
         rows = np.arange(q.shape[0])
+        if n_q is None:
+            n_q = q.shape[0]
+    if n_q is None:
+        n_q = n_k
     s = float(scale) * (q @ k.T)
-    vis = _visible(rows, k.shape[0], causal, block_mask, mask_block)
+    vis = _visible(rows, n_k, causal, block_mask, mask_block, n_k - n_q)
     return np.where(vis, s, -np.inf)
 
 
@@ -119,7 +129,8 @@ def attn_probs_ref(q, k, scale: float, causal: bool = False, block_mask=None,
 
 def attn_fwd_ref(q, k, v, causal: bool = False, scale: float | None = None,
                  block_mask=None, mask_block: int = 128):
-    """Forward for [B, H, N, d] inputs -> (O [B,H,N,d], lse [B,H,N]) in fp64.
+    """Forward for q [B, H, N_q, d], k and v [B, H, N_k, d] -> (O [B,H,N_q,d],
+    lse [B,H,N_q]) in fp64.
 
     One (b, h) at a time: S materialised, masked, softmaxed, multiplied by V.
     """
@@ -139,33 +150,33 @@ def attn_fwd_ref(q, k, v, causal: bool = False, scale: float | None = None,
 
 
 def attn_fwd_rows_ref(q_rows, rows, k, v, causal: bool, scale: float,
-                      block_mask=None, mask_block: int = 128):
+                      block_mask=None, mask_block: int = 128, n_q=None):
     """Forward for a sample of query rows of ONE head.
 
     q_rows [R, d] are the queries at absolute positions ``rows`` (length R); k, v are
     the head's full [N, d] keys and values. Returns (O [R, d], lse [R]). Used for
     sampled checks at sizes where the full N x N matrix is too large to hold.
     """
-    s = attn_scores_ref(q_rows, k, scale, causal, block_mask, mask_block, rows=rows)
+    s = attn_scores_ref(q_rows, k, scale, causal, block_mask, mask_block, rows=rows, n_q=n_q)
     p, lse = _softmax_rows(s)
     return p @ _f64(v), lse
 
 
 def attn_bwd_ref(q, k, v, do, causal: bool = False, scale: float | None = None,
                  block_mask=None, mask_block: int = 128):
-    """Gradients of L = sum(O * dO) for [B, H, N, d] inputs, in fp64.
+    """Gradients of L = sum(O * dO) for q, dO [B, H, N_q, d] and k, v [B, H, N_k, d],
+    in fp64.
 
-    Returns a dict with dq, dk, dv ([B,H,N,d]), D ([B,H,N], sum_j P dP), and the
-    forward's o and lse. D is computed both as sum_j P_ij dP_ij and as
-    sum_c dO_ic O_ic; the two must agree (asserted).
+    Returns a dict with dq ([B,H,N_q,d]), dk, dv ([B,H,N_k,d]), D ([B,H,N_q],
+    sum_j P dP), and the forward's o and lse. D is computed both as
+    sum_j P_ij dP_ij and as sum_c dO_ic O_ic; the two must agree (asserted).
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / np.sqrt(d)
-    out = {name: np.zeros_like(q) for name in ("dq", "dk")}
-    out["dv"] = np.zeros_like(v)
-    out["o"] = np.zeros_like(v)
+    out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v)}
+    out["o"] = np.zeros((B, H, N, v.shape[-1]))
     out["lse"] = np.zeros((B, H, N))
     out["D"] = np.zeros((B, H, N))
     for b in range(B):
@@ -190,7 +201,7 @@ def attn_bwd_ref(q, k, v, do, causal: bool = False, scale: float | None = None,
 
 
 def attn_dq_rows_ref(q_rows, rows, k, v, do_rows, causal: bool, scale: float,
-                     block_mask=None, mask_block: int = 128) -> np.ndarray:
+                     block_mask=None, mask_block: int = 128, n_q=None) -> np.ndarray:
     """dQ for a sample of query rows of ONE head (same definition as attn_bwd_ref).
 
     Row i needs only its own scores: P_i = softmax(S_i), dP_i = dO_i V^T,
@@ -198,7 +209,7 @@ def attn_dq_rows_ref(q_rows, rows, k, v, do_rows, causal: bool, scale: float,
     q_rows, do_rows [R, d] at absolute positions ``rows``; k, v the head's [N, d].
     """
     k, v, do_rows = _f64(k), _f64(v), _f64(do_rows)
-    s = attn_scores_ref(q_rows, k, scale, causal, block_mask, mask_block, rows=rows)
+    s = attn_scores_ref(q_rows, k, scale, causal, block_mask, mask_block, rows=rows, n_q=n_q)
     p, _ = _softmax_rows(s)
     dp = do_rows @ v.T
     D = np.sum(p * dp, axis=1)

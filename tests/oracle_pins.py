@@ -281,6 +281,87 @@ def pin_dq_rows_match_full(mod):
         assert np.allclose(dq, g["dq"][0, 0, rows], atol=1e-12)
 
 
+# ---------------------------------------------------------------- N_q != N_k (bottom-right causal)
+
+def pin_cross_decode_sees_every_key(mod):
+    """One query against N_k keys with the causal mask: the last (only) query sees every
+    key, so the result is the unmasked one."""
+    q, k, v, do = _rand((1, 2, 1, 6), 40), _rand((1, 2, 9, 6), 41), _rand((1, 2, 9, 6), 42), _rand((1, 2, 1, 6), 43)
+    oc, lc = mod.attn_fwd_ref(q, k, v, True, 0.6)
+    on, ln = mod.attn_fwd_ref(q, k, v, False, 0.6)
+    assert np.array_equal(oc, on) and np.array_equal(lc, ln)
+    gc, gn = mod.attn_bwd_ref(q, k, v, do, True, 0.6), mod.attn_bwd_ref(q, k, v, do, False, 0.6)
+    for name in ("dq", "dk", "dv"):
+        assert gc[name].shape == (q.shape if name == "dq" else k.shape)
+        assert np.array_equal(gc[name], gn[name])
+
+
+def pin_cross_is_suffix_of_square(mod):
+    """N_q < N_k, causal: the queries are the last N_q rows of a square causal problem
+    whose first N_k - N_q query rows are arbitrary. O, lse and dQ are those rows of the
+    square problem; dK and dV are the square problem's when the extra rows' dO is 0."""
+    nq, nk = 5, 9
+    q, k, v = _rand((1, 2, nq, 4), 44), _rand((1, 2, nk, 4), 45), _rand((1, 2, nk, 4), 46)
+    do = _rand((1, 2, nq, 4), 47)
+    extra = _rand((1, 2, nk - nq, 4), 48)
+    qs = np.concatenate([extra, q], axis=2)
+    dos = np.concatenate([np.zeros_like(extra), do], axis=2)
+    o, lse = mod.attn_fwd_ref(q, k, v, True, 0.9)
+    osq, lsq = mod.attn_fwd_ref(qs, k, v, True, 0.9)
+    assert np.allclose(o, osq[:, :, nk - nq:], atol=1e-13) and np.allclose(lse, lsq[:, :, nk - nq:], atol=1e-13)
+    g, gs = mod.attn_bwd_ref(q, k, v, do, True, 0.9), mod.attn_bwd_ref(qs, k, v, dos, True, 0.9)
+    assert np.allclose(g["dq"], gs["dq"][:, :, nk - nq:], atol=1e-12)
+    assert np.allclose(g["dk"], gs["dk"], atol=1e-12) and np.allclose(g["dv"], gs["dv"], atol=1e-12)
+
+
+def pin_cross_more_queries_than_keys(mod):
+    """N_q > N_k, causal: query i sees keys j <= i - (N_q - N_k); the first N_q - N_k
+    queries see none (O = 0, lse = -inf, dQ = 0) and the rest form the square causal
+    problem of the last N_k queries."""
+    nq, nk = 9, 4
+    q, k, v, do = _rand((1, 1, nq, 3), 49), _rand((1, 1, nk, 3), 50), _rand((1, 1, nk, 3), 51), _rand((1, 1, nq, 3), 52)
+    o, lse = mod.attn_fwd_ref(q, k, v, True, 1.1)
+    assert np.all(o[:, :, :nq - nk] == 0) and np.all(np.isneginf(lse[:, :, :nq - nk]))
+    osq, lsq = mod.attn_fwd_ref(q[:, :, nq - nk:], k, v, True, 1.1)
+    assert np.allclose(o[:, :, nq - nk:], osq, atol=1e-13) and np.allclose(lse[:, :, nq - nk:], lsq, atol=1e-13)
+    g = mod.attn_bwd_ref(q, k, v, do, True, 1.1)
+    gs = mod.attn_bwd_ref(q[:, :, nq - nk:], k, v, do[:, :, nq - nk:], True, 1.1)
+    assert np.all(g["dq"][:, :, :nq - nk] == 0) and np.allclose(g["dq"][:, :, nq - nk:], gs["dq"], atol=1e-12)
+    assert np.allclose(g["dk"], gs["dk"], atol=1e-12) and np.allclose(g["dv"], gs["dv"], atol=1e-12)
+
+
+def pin_cross_brute_force(mod):
+    """N_q = 3, N_k = 5, causal, written out element by element: key j counts for query
+    i when j - i <= N_k - N_q; O_i = sum exp(s_ij) v_j / sum exp(s_ij), lse_i = ln sum."""
+    q, k, v = _rand((3, 2), 53), _rand((5, 2), 54), _rand((5, 2), 55)
+    sc = 0.7
+    o_ref, lse_ref = np.zeros((3, 2)), np.zeros(3)
+    for i in range(3):
+        num, den = np.zeros(2), 0.0
+        for j in range(5):
+            if j - i <= 5 - 3:
+                e = math.exp(sc * float(q[i] @ k[j]))
+                num += e * v[j]
+                den += e
+        o_ref[i], lse_ref[i] = num / den, math.log(den)
+    o, lse = mod.attn_fwd_ref(q[None, None], k[None, None], v[None, None], True, sc)
+    assert np.allclose(o[0, 0], o_ref, atol=1e-13) and np.allclose(lse[0, 0], lse_ref, atol=1e-13)
+
+
+def pin_cross_rows_match_full(mod):
+    """Sampled-row forward and dQ of an N_q != N_k causal problem (n_q given) equal the
+    full computation's rows."""
+    nq, nk = 6, 11
+    q, k, v, do = _rand((nq, 4), 56), _rand((nk, 4), 57), _rand((nk, 4), 58), _rand((nq, 4), 59)
+    rows = np.array([0, 2, 5])
+    o, lse = mod.attn_fwd_ref(q[None, None], k[None, None], v[None, None], True, 0.5)
+    orow, lrow = mod.attn_fwd_rows_ref(q[rows], rows, k, v, True, 0.5, n_q=nq)
+    assert np.allclose(orow, o[0, 0][rows], atol=1e-13) and np.allclose(lrow, lse[0, 0][rows], atol=1e-13)
+    g = mod.attn_bwd_ref(q[None, None], k[None, None], v[None, None], do[None, None], True, 0.5)
+    dqr = mod.attn_dq_rows_ref(q[rows], rows, k, v, do[rows], True, 0.5, n_q=nq)
+    assert np.allclose(dqr, g["dq"][0, 0][rows], atol=1e-12)
+
+
 FORWARD_PINS = [
     pin_probs_rows_sum_to_one,
     pin_equal_keys_mean_of_v,
@@ -302,4 +383,11 @@ BACKWARD_PINS = [
     pin_gradient_invariants,
     pin_dq_rows_match_full,
 ]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS
+CROSS_PINS = [
+    pin_cross_decode_sees_every_key,
+    pin_cross_is_suffix_of_square,
+    pin_cross_more_queries_than_keys,
+    pin_cross_brute_force,
+    pin_cross_rows_match_full,
+]
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS + CROSS_PINS

@@ -35,8 +35,11 @@ def test_oracle_does_not_import_cuda_path():
 # transposed operand, an off-by-one in a mask.
 MUTATIONS = {
     "dropped_scale": ("s = float(scale) * (q @ k.T)", "s = (q @ k.T)"),
-    "causal_off_by_one": ("cols[None, :] <= rows[:, None]", "cols[None, :] < rows[:, None]"),
-    "causal_flipped": ("cols[None, :] <= rows[:, None]", "cols[None, :] >= rows[:, None]"),
+    "causal_off_by_one": ("cols[None, :] <= rows[:, None] + causal_offset", "cols[None, :] < rows[:, None] + causal_offset"),
+    "causal_flipped": ("cols[None, :] <= rows[:, None] + causal_offset", "cols[None, :] >= rows[:, None] + causal_offset"),
+    "causal_offset_sign": ("mask_block, n_k - n_q)", "mask_block, n_q - n_k)"),
+    "causal_offset_dropped": ("mask_block, n_k - n_q)", "mask_block, 0)"),
+    "dk_shaped_like_q": ('"dk": np.zeros_like(k)', '"dk": np.zeros_like(q)'),
     "block_mask_transposed": ("bm[rows[:, None] // mask_block, cols[None, :] // mask_block]",
                               "bm[cols[None, :] // mask_block, rows[:, None] // mask_block]"),
     "pv_transposed": ("o[b, h] = p @ v[b, h]", "o[b, h] = p.T @ v[b, h]"),
