@@ -51,7 +51,7 @@ def workload(name: str):
         d = int(parts[2][1:])
         B, H = sweep_shape(N, d)
         causal = len(parts) > 3 and parts[3] == "causal"
-        return dict(B=B, H=H, N=N, d=d, variants=[("causal" if causal else "noncausal", causal, None)],
+        return dict(B=B, H=H, N=N, Nk=N, d=d, variants=[("causal" if causal else "noncausal", causal, None)],
                     do_scale=0.5)
     w = WORKLOADS[name]
     variants = []
@@ -60,7 +60,7 @@ def workload(name: str):
     else:
         for c in w["causal"]:
             variants.append(("causal" if c else "noncausal", c, None))
-    return dict(B=w["B"], H=w["H"], N=w["N"], d=w["d"], variants=variants, do_scale=1.0)
+    return dict(B=w["B"], H=w["H"], N=w["N"], Nk=w.get("Nk", w["N"]), d=w["d"], variants=variants, do_scale=1.0)
 
 
 # ---------------------------------------------------------------- multi-rank helpers
@@ -89,11 +89,14 @@ def job_throughput(world: int, flops_per_rank_step: float, steps: int, max_ms: f
     return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
 
 
-def fwd_flops(B, H, N, d, causal, density=1.0):
-    f = 4.0 * B * H * N * N * d
-    if causal:
-        f *= 0.5
-    return f * density
+def fwd_flops(B, H, N, d, causal, density=1.0, Nk=None):
+    """Forward FLOPs 4 B H N Nk d over the visible (query, key) pairs: causal counts
+    Nq Nk - Nq^2 / 2 pairs (exactly half for Nq = Nk, the square convention; the
+    causal mask is bottom-right aligned and Nq <= Nk here); block-sparse scales by
+    the kept-tile fraction."""
+    Nk = N if Nk is None else Nk
+    pairs = N * Nk - 0.5 * N * N if causal else N * Nk
+    return 4.0 * B * H * pairs * d * density
 
 
 # ---------------------------------------------------------------- clocks
@@ -506,7 +509,7 @@ def run_table(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse", "b8h16n2000d64_ragged",
-             "b2h16n8000d128_ragged_causal"]
+             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal"]
     names += [f"sweep_N{N}_d{d}{c}" for d in SWEEP_D for N in SWEEP_N for c in ("", "_causal")]
     if args.only:
         names = [n for n in names if any(o in n for o in args.only.split(","))]
@@ -515,17 +518,20 @@ def run_table(args):
     stream = torch.cuda.current_stream(dev)
     for name in names:
         wl = workload(name)
-        B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
+        B, H, N, Nk, d = wl["B"], wl["H"], wl["N"], wl["Nk"], wl["d"]
         sc = 1.0 / math.sqrt(d)
         t = {k: v.to(dev) for k, v in make_qkv(B, H, N, d, seed=0, do_scale=wl["do_scale"]).items()}
+        if Nk != N:  # keys and values of their own length
+            kv = make_qkv(B, H, Nk, d, seed=1, with_do=False)
+            t["k"], t["v"] = kv["k"].to(dev), kv["v"].to(dev)
         ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
         o = torch.empty_like(t["q"])
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-        dq, dk, dv = (torch.empty_like(t["q"]) for _ in range(3))
+        dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
         for (label, causal, dens) in wl["variants"]:
             mask = None if dens is None else make_tile_mask(-(-N // 128), seed=0, density=dens).to(dev)
             kept = 1.0 if mask is None else float(mask.float().mean())
-            F = fwd_flops(B, H, N, d, causal, kept)
+            F = fwd_flops(B, H, N, d, causal, kept, Nk)
 
             def fwd():
                 if mask is None:
@@ -560,7 +566,16 @@ def run_table(args):
             row = {"workload": name, "variant": label, "B": B, "H": H, "N": N, "d": d, "kept": round(kept, 4),
                    "fwd_ms": round(t_f, 4), "fwd_tflops": round(F / t_f / 1e9, 1),
                    "fwd_pct_peak": round(100 * F / t_f / 1e9 / pk["bf16_tflops"], 1)}
-            if name != "pr1":
+            if Nk != N:
+                # The staged calls are for Nq = Nk; time the whole backward through the API.
+                def bwd_all():
+                    fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=causal, scale=sc, workspace=ws,
+                                grads=(dq, dk, dv))
+                t_b = timed([bwd_all])
+                row.update({"Nk": Nk, "bwd_ms": round(t_b, 4), "bwd_tflops": round(2.5 * F / t_b / 1e9, 1),
+                            "bwd_pct_peak": round(100 * 2.5 * F / t_b / 1e9 / pk["bf16_tflops"], 1),
+                            "fwd_bwd_tflops": round(3.5 * F / (t_f + t_b) / 1e9, 1)})
+            elif name != "pr1":
                 pre()
                 t_kv = timed([dkdv])
                 t_q = timed([dqk])

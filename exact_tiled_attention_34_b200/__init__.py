@@ -10,8 +10,11 @@ is missing or a tensor is not a CUDA tensor, the call raises.
     dq, dk, dv = backward(q, k, v, o, lse, do, causal=False, scale=None)
     dq, dk, dv = backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None)
 
-Tensors are bf16 [B, H, N, d] contiguous on one CUDA device; lse is fp32 [B, H, N];
-tile_mask is uint8 [ceil(N/128), ceil(N/128)] on the same device. Any N >= 1, d in {64, 128}.
+Tensors are bf16 contiguous on one CUDA device: q, o, do [B, H, Nq, d]; k, v
+[B, H, Nk, d]; lse fp32 [B, H, Nq]. Nq and Nk may differ (then the causal mask is
+bottom-right aligned: query i sees key j iff j <= i + Nk - Nq); the block-sparse
+calls need Nq = Nk = N and a uint8 tile_mask [ceil(N/128), ceil(N/128)]. Any N >= 1,
+d in {64, 128}.
 """
 from __future__ import annotations
 
@@ -51,9 +54,11 @@ _SIGS = {
     "fa_status_string": ([_i], ctypes.c_char_p),
     "fa_version": ([], _i),
     "fa_fwd": ([_vp] * 5 + [_i] * 5 + [_f, _vp], _i),
+    "fa_fwd_qk": ([_vp] * 5 + [_i] * 6 + [_f, _vp], _i),
     "fa_fwd_blocksparse": ([_vp] * 6 + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_workspace_bytes": ([_i] * 4, _sz),
     "fa_bwd": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_qk": ([_vp] * 10 + [_sz] + [_i] * 6 + [_f, _vp], _i),
     "fa_bwd_blocksparse": ([_vp] * 10 + [_sz, _vp, _i] + [_i] * 4 + [_f, _vp], _i),
     "fa_device_status": ([_vp, ctypes.POINTER(_i)], _i),
     "fa_bwd_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
@@ -96,20 +101,24 @@ def _stream_ptr(dev):
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
-def _check_qkv(*ts):
+def _check_qkv(q, k, v, *qlike):
+    """q and the tensors in qlike (o, dO) are [B, H, Nq, d]; k and v are [B, H, Nk, d]."""
     import torch
-    t0 = ts[0]
-    for t in ts:
+    for t in (q, k, v) + qlike:
         if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors (no CPU path)")
         if t.dtype != torch.bfloat16:
             raise ValueError("q, k, v, o, dO must be bfloat16")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous [B, H, N, d]")
-        if t.shape != t0.shape or t.device != t0.device:
-            raise ValueError("q, k, v (and o, dO) must share shape and device")
-    if t0.dim() != 4:
+        if t.device != q.device:
+            raise ValueError("all tensors must be on one device")
+    if q.dim() != 4 or k.dim() != 4:
         raise ValueError("expected [B, H, N, d] tensors")
+    if k.shape != v.shape or any(t.shape != q.shape for t in qlike):
+        raise ValueError("k and v must share a shape, as must q, o and dO")
+    if (q.shape[0], q.shape[1], q.shape[3]) != (k.shape[0], k.shape[1], k.shape[3]):
+        raise ValueError("q and k must agree in batch, heads and head dim")
 
 
 def _scale(scale, d):
@@ -121,11 +130,16 @@ def forward(q, k, v, causal: bool = False, scale=None, out=None, lse=None):
     import torch
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     with torch.cuda.device(q.device):
-        st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
-                          B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+        if Nk == N:
+            st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                              B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+        else:
+            st = lib().fa_fwd_qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                 B, H, N, Nk, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
     _check(st, "fa_fwd")
     return o, l
 
@@ -178,10 +192,17 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=No
     import torch
     workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     with torch.cuda.device(q.device):
-        st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                          B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+        if Nk == N:
+            st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                              B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+        else:
+            st = lib().fa_bwd_qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                 workspace.numel(), B, H, N, Nk, d, int(bool(causal)), _scale(scale, d),
+                                 _stream_ptr(q.device))
     _check(st, "fa_bwd")
     return dq, dk, dv
 

@@ -116,13 +116,13 @@ fa_status set_smem(K kernel, int bytes, std::once_flag (&flags)[kMaxDevices], cu
 }
 
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE>;
+  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK>;
   constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
   // The kernel re-divides its register pool between warpgroups: refuse to launch a
@@ -144,10 +144,12 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 }
 
 fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
-                     int B, int H, int N, int d, int causal, float scale, void* stream) {
+                     int B, int H, int N, int Nk, int d, int causal, float scale, void* stream) {
   fa_status s;
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
+  if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
+  if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
   int* status;
@@ -155,8 +157,8 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   if ((s = make_map(&mq, q, BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mk, k, BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mv, v, BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, BH, Nk, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, BH, Nk, d, 128)) != FA_OK) return s;
   fa::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -164,8 +166,11 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.status = status;
   p.timeout_ns = kTimeoutNs;
   p.N = N;
+  p.Nk = Nk;
   p.BH = BH;
   p.n_tiles = (N + 127) / 128;
+  p.n_ktiles = (Nk + 127) / 128;
+  p.off = Nk - N;
   p.n_qblocks = (p.n_tiles + 1) / 2;
   p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
@@ -173,6 +178,9 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   if (mask) {
     return d == 64 ? launch_fwd<64, false, true>(mq, mk, mv, p, st) : launch_fwd<128, false, true>(mq, mk, mv, p, st);
   }
+  if (causal && Nk != N)  // causal mask with an offset (N_q != N_k)
+    return d == 64 ? launch_fwd<64, true, false, true>(mq, mk, mv, p, st)
+                   : launch_fwd<128, true, false, true>(mq, mk, mv, p, st);
   if (causal) {
     return d == 64 ? launch_fwd<64, true, false>(mq, mk, mv, p, st) : launch_fwd<128, true, false>(mq, mk, mv, p, st);
   }
@@ -216,23 +224,23 @@ fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid /* work items */, 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
 fa_status launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                       const fa::BwdParams& p, cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  return launch_bwd_kernel(fa::fa_bwd_dkdv_kernel<D, CAUSAL, SPARSE>, fa::BwdCfg<D>::kSmemBytes,
-                           unsigned(p.n_tiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
+  return launch_bwd_kernel(fa::fa_bwd_dkdv_kernel<D, CAUSAL, SPARSE, XQK>, fa::BwdCfg<D>::kSmemBytes,
+                           unsigned(p.n_ktiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
 }
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
 fa_status launch_dq(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                     const fa::BwdParams& p, cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  return launch_bwd_kernel(fa::fa_bwd_dq_kernel<D, CAUSAL, SPARSE>, fa::BwdCfg<D>::kQSmemBytes,
+  return launch_bwd_kernel(fa::fa_bwd_dq_kernel<D, CAUSAL, SPARSE, XQK>, fa::BwdCfg<D>::kQSmemBytes,
                            unsigned(p.n_tiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
 }
 
@@ -281,23 +289,25 @@ fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, siz
 enum class BwdStage { kDkdv, kDq };
 
 // dK/dV (stage kDkdv: dk, dv written) or dQ (stage kDq: dq written).
+// N: query rows (the workspace's rows), Nk: key rows.
 fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v, const void* dO, void* out0,
                     void* out1, const void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H,
-                    int N, int d, int causal, float scale, void* stream) {
+                    int N, int Nk, int d, int causal, float scale, void* stream) {
   fa_status s;
   if ((s = check_ptrs({q, k, v, dO, out0})) != FA_OK) return s;
   if (stage == BwdStage::kDkdv && (s = check_ptrs({out1})) != FA_OK) return s;
-  if (mask != nullptr && (mask_block != 128 || causal)) return FA_ERR_UNSUPPORTED;
+  if (mask != nullptr && (mask_block != 128 || causal || Nk != N)) return FA_ERR_UNSUPPORTED;
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
   int* status;
   if ((s = device_status_ptr(&status)) != FA_OK) return s;
   CUtensorMap mq, mk, mv, mdo;
   if ((s = make_map(&mq, q, a.BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mk, k, a.BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mv, v, a.BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, a.BH, Nk, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, a.BH, Nk, d, 128)) != FA_OK) return s;
   if ((s = make_map(&mdo, dO, a.BH, N, d, 128)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fa::BwdParams p;
@@ -310,13 +320,19 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.status = status;
   p.timeout_ns = kTimeoutNs;
   p.N = N;
+  p.Nk = Nk;
   p.BH = a.BH;
   p.n_tiles = (N + 127) / 128;
+  p.n_ktiles = (Nk + 127) / 128;
+  p.off = Nk - N;
   p.scale = scale;
 #define FA_BWD_DISPATCH(LAUNCH)                                                                  \
   if (mask)                                                                                      \
     return d == 64 ? LAUNCH<64, false, true>(mq, mk, mv, mdo, p, st)                             \
                    : LAUNCH<128, false, true>(mq, mk, mv, mdo, p, st);                           \
+  if (causal && Nk != N)                                                                         \
+    return d == 64 ? LAUNCH<64, true, false, true>(mq, mk, mv, mdo, p, st)                       \
+                   : LAUNCH<128, true, false, true>(mq, mk, mv, mdo, p, st);                     \
   if (causal)                                                                                    \
     return d == 64 ? LAUNCH<64, true, false>(mq, mk, mv, mdo, p, st)                             \
                    : LAUNCH<128, true, false>(mq, mk, mv, mdo, p, st);                           \
@@ -331,18 +347,20 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
 
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int B, int H,
-                     int N, int d, int causal, float scale, void* stream) {
+                     int N, int Nk, int d, int causal, float scale, void* stream) {
   fa_status s;
   // Validate everything before the first launch so that an error writes nothing.
   if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv})) != FA_OK) return s;
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if ((s = check_scale(scale)) != FA_OK) return s;
+  if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
   if ((s = bwd_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, d, causal, scale,
+  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, Nk, d, causal, scale,
                      stream)) != FA_OK)
     return s;
-  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, ws, ws_bytes, mask, 128, B, H, N, d, causal, scale,
+  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, ws, ws_bytes, mask, 128, B, H, N, Nk, d, causal, scale,
                    stream);
 }
 
@@ -386,7 +404,12 @@ int fa_version(void) { return 100; }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  int causal, float scale, void* stream) {
-  return fwd_common(q, k, v, o, lse, nullptr, B, H, N, d, causal != 0, scale, stream);
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, N, N, d, causal != 0, scale, stream);
+}
+
+fa_status fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                    int d, int causal, float scale, void* stream) {
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, Nq, Nk, d, causal != 0, scale, stream);
 }
 
 fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -394,7 +417,7 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                              void* stream) {
   if (tile_mask == nullptr) return FA_ERR_INVALID_ARG;
   if (mask_block != 128) return FA_ERR_UNSUPPORTED;
-  return fwd_common(q, k, v, o, lse, tile_mask, B, H, N, d, 0, scale, stream);
+  return fwd_common(q, k, v, o, lse, tile_mask, B, H, N, N, d, 0, scale, stream);
 }
 
 fa_status fa_device_status(void* stream, int* detail) {
@@ -419,8 +442,15 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) { return bwd_ws_bytes(
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                  int causal, float scale, void* stream) {
-  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d, causal != 0,
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, N, d, causal != 0,
                     scale, stream);
+}
+
+fa_status fa_bwd_qk(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Nq,
+                    int Nk, int d, int causal, float scale, void* stream) {
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, Nq, Nk, d,
+                    causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace,
@@ -432,14 +462,14 @@ fa_status fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* d
                       const void* workspace, size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B,
                       int H, int N, int d, int causal, float scale, void* stream) {
   return bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N,
-                   d, causal != 0, scale, stream);
+                   N, d, causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, const void* workspace,
                     size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B, int H, int N, int d,
                     int causal, float scale, void* stream) {
   return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, workspace, workspace_bytes, tile_mask, mask_block, B, H,
-                   N, d, causal != 0, scale, stream);
+                   N, N, d, causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -448,7 +478,7 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
                              void* stream) {
   if (tile_mask == nullptr) return FA_ERR_INVALID_ARG;
   if (mask_block != 128) return FA_ERR_UNSUPPORTED;
-  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, B, H, N, d, 0, scale,
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, B, H, N, N, d, 0, scale,
                     stream);
 }
 
@@ -505,9 +535,9 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
   // earlier call left in the array does not matter.
   const size_t bytes = size_t(FA_BWD_NOALLOC_SCRATCH_BYTES);
   if ((s = bwd_pre(o, dO, lse, scratch, bytes, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, scratch, bytes, tile_mask, mask_block, B, H, N, d,
+  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, scratch, bytes, tile_mask, mask_block, B, H, N, N, d,
                      causal, scale, stream)) != FA_OK)
     return s;
-  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, scratch, bytes, tile_mask, mask_block, B, H, N, d, causal,
-                   scale, stream);
+  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, scratch, bytes, tile_mask, mask_block, B, H, N, N, d,
+                   causal, scale, stream);
 }

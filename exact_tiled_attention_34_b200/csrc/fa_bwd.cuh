@@ -95,9 +95,12 @@ struct BwdParams {
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;
   unsigned long long timeout_ns;
-  int N;                // sequence length (any N >= 1)
+  int N;                // query rows N_q (any N >= 1)
+  int Nk;               // key rows N_k
   int BH;
-  int n_tiles;          // ceil(N / 128)
+  int n_tiles;          // query tiles ceil(N_q / 128)
+  int n_ktiles;         // key tiles ceil(N_k / 128)
+  int off;              // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
   float scale;          // softmax scale
 };
 
@@ -148,29 +151,49 @@ enum BwdSite : int {
   kSiteBwdDpFull, kSiteBwdAcc, kSiteBwdDrain, kSiteBwdRead, kSiteBwdSRead
 };
 
-// Query tiles that see key tile j (dK/dV kernel).
-template <bool CAUSAL, bool SPARSE>
+// Causal limits between tiles (key j visible to query i iff j <= i + off):
+// the first query tile that sees key tile j, and the last key tile query tile i sees
+// (clamped to the key tiles; -1 for none).
+__device__ __forceinline__ int causal_qfirst(int j, int off) {
+  const long long x = 128LL * j - 127 - off;  // query tile t sees key tile j iff 128 t >= x
+  return x <= 0 ? 0 : static_cast<int>((x + 127) >> 7);
+}
+__device__ __forceinline__ int causal_klast_b(int i, int off, int n_ktiles) {
+  const long long x = 128LL * i + 127 + off;
+  const long long l = x < 0 ? -1 : (x >> 7);
+  return static_cast<int>(l < n_ktiles - 1 ? l : n_ktiles - 1);
+}
+
+// Query tiles that see key tile j (dK/dV kernel). The block mask is [n_tiles, n_ktiles].
+// i_first: the first query tile that can see tile j (0 without the causal mask).
+template <bool CAUSAL, bool SPARSE, bool XQK>
 struct KeySched {
-  int j, n_tiles;
+  int j, n_tiles, n_ktiles, i_first;
   const uint8_t* mask;
+  __device__ __forceinline__ KeySched(int j_, int n_tiles_, int n_ktiles_, int off, const uint8_t* mask_)
+      : j(j_), n_tiles(n_tiles_), n_ktiles(n_ktiles_),
+        i_first(CAUSAL ? (XQK ? causal_qfirst(j_, off) : j_) : 0), mask(mask_) {}
   __device__ __forceinline__ int next(int i0) const {
-    for (int i = (CAUSAL ? (i0 < j ? j : i0 + 1) : i0 + 1); i < n_tiles; ++i) {
-      if (!SPARSE || mask[size_t(i) * n_tiles + j] != 0) return i;
+    for (int i = (i0 + 1 > i_first ? i0 + 1 : i_first); i < n_tiles; ++i) {
+      if (!SPARSE || mask[size_t(i) * n_ktiles + j] != 0) return i;
     }
     return -1;
   }
-  __device__ __forceinline__ int first() const { return next(CAUSAL ? j - 1 : -1); }
+  __device__ __forceinline__ int first() const { return next(-1); }
 };
 
-// Key tiles that query tile i sees (dQ kernel).
-template <bool CAUSAL, bool SPARSE>
+// Key tiles that query tile i sees (dQ kernel). j_last: the last key tile tile i can
+// see (-1 for none).
+template <bool CAUSAL, bool SPARSE, bool XQK>
 struct QuerySched {
-  int i, n_tiles;
+  int i, n_ktiles, j_last;
   const uint8_t* mask;
+  __device__ __forceinline__ QuerySched(int i_, int n_ktiles_, int off, const uint8_t* mask_)
+      : i(i_), n_ktiles(n_ktiles_),
+        j_last(CAUSAL ? (XQK ? causal_klast_b(i_, off, n_ktiles_) : i_) : n_ktiles_ - 1), mask(mask_) {}
   __device__ __forceinline__ int next(int j0) const {
-    const int last = CAUSAL ? i : n_tiles - 1;
-    for (int j = j0 + 1; j <= last; ++j) {
-      if (!SPARSE || mask[size_t(i) * n_tiles + j] != 0) return j;
+    for (int j = j0 + 1; j <= j_last; ++j) {
+      if (!SPARSE || mask[size_t(i) * n_ktiles + j] != 0) return j;
     }
     return -1;
   }
@@ -297,12 +320,14 @@ struct DkdvBars {
   int abort;
 };
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const BwdParams p) {
   using Cfg = BwdCfg<D>;
+  // Causal offset N_k - N_q: a compile-time 0 in the N_q = N_k kernels (XQK false).
+  const int off_ = XQK ? p.off : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem + Cfg::kOffBar);
@@ -359,9 +384,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int nkv = 0;
       bool ok = true;
       BwdItem item;
-      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_tiles, p.BH, kk, item); ++kk) {
+      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
         const int j = item.tile, bh = item.bh;
-        KeySched<CAUSAL, SPARSE> sch{j, p.n_tiles, p.tile_mask};
+        KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
         if (kk > 0 && !mbar_wait(&bars->kv_empty, (kk - 1) & 1, wc, kSiteBwdTEmpty)) break;
         mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
@@ -405,8 +430,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       bool ok = true;
       int it = 0;  // query tiles processed so far (continues across items)
       BwdItem item;
-      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_tiles, p.BH, kk, item); ++kk) {
-        KeySched<CAUSAL, SPARSE> sch{item.tile, p.n_tiles, p.tile_mask};
+      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
+        KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
         if (!mbar_wait(&bars->kv_full, kk & 1, wc, kSiteBwdKV)) { ok = false; break; }
         tc_fence_after();
         int i = sch.first();
@@ -484,9 +509,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     bool ok = true;
     int it = 0;  // query tiles processed so far (continues across items)
     BwdItem item;
-    for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_tiles, p.BH, kk, item); ++kk) {
+    for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
       const int j = item.tile;
-      KeySched<CAUSAL, SPARSE> sch{j, p.n_tiles, p.tile_mask};
+      KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
       int local = 0;
       for (int i = sch.first(); i >= 0; i = sch.next(i), ++it, ++local) {
         const int st = it & 1;
@@ -498,7 +523,15 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tc_fence_after();
         const float* lse2 = sL + st * 128 + h * 64;
         const float* Dr = sDr + st * 128 + h * 64;
-        const bool diag = CAUSAL && (i == j);  // query c visible to key r iff c >= r
+        // Query 128 i + c sees key 128 j + r iff c >= r + cbase; the tile is partial
+        // (element mask) iff some (r, c) fails, i.e. cbase + 127 > 0.
+        int cbase = 0;  // N_q = N_k: only the diagonal tile (i == j) is partial, with cbase 0
+        if constexpr (XQK) {
+          const long long cb64 = 128LL * (j - i) - off_;  // clamped: beyond +-256 no row is partial
+          cbase = static_cast<int>(cb64 < -256 ? -256 : (cb64 > 256 ? 256 : cb64));
+        }
+        const bool diag = CAUSAL && (XQK ? cbase > -127 : i == j);
+        const int cmin = cbase + r;
         // ---- P^T row r, query columns 64h + (0..63), packed bf16 pairs
         uint32_t pk[32];
         {
@@ -521,7 +554,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 f2_fma(f2(__uint_as_float(raw[c0]), __uint_as_float(raw[c0 + 1])), c2v, f2(nl.x, nl.y)), t);
             if (diag) {
               const float2 v = f2_split(pv);
-              pv = f2((h * 64 + c0 < r) ? 0.f : v.x, (h * 64 + c0 + 1 < r) ? 0.f : v.y);
+              pv = f2((h * 64 + c0 < cmin) ? 0.f : v.x, (h * 64 + c0 + 1 < cmin) ? 0.f : v.y);
             }
             const float2 v = f2_split(pv);
             pk[t] = pack_bf16(v.x, v.y);
@@ -570,7 +603,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         break;
       }
       tc_fence_after();
-      const size_t row = size_t(item.bh) * p.N + size_t(j) * 128 + r;
+      const size_t row = size_t(item.bh) * p.Nk + size_t(j) * 128 + r;  // key row
       uint32_t acc[D];
       if (local > 0) {
 #pragma unroll
@@ -584,7 +617,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
-      if (j * 128 + r < p.N)  // key rows past N (last tile, N % 128 != 0) do not exist
+      if (j * 128 + r < p.Nk)  // key rows past N_k (last tile, N_k % 128 != 0) do not exist
         store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * D, acc, h == 0 ? p.scale : 1.f);
     }
     tc_fence_before();
@@ -613,12 +646,14 @@ struct DqBars {
   int abort;
 };
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                  const BwdParams p) {
   using Cfg = BwdCfg<D>;
+  // Causal offset N_k - N_q: a compile-time 0 in the N_q = N_k kernels (XQK false).
+  const int off_ = XQK ? p.off : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   DqBars* bars = reinterpret_cast<DqBars*>(smem + Cfg::kQOffBar);
@@ -673,7 +708,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
         const int i = item.tile, bh = item.bh;
-        QuerySched<CAUSAL, SPARSE> sch{i, p.n_tiles, p.tile_mask};
+        QuerySched<CAUSAL, SPARSE, XQK> sch{i, p.n_ktiles, off_, p.tile_mask};
         if (kk > 0 && !mbar_wait(&bars->q_empty, (kk - 1) & 1, wc, kSiteBwdTEmpty)) break;
         mbar_arrive_expect_tx(&bars->q_full, 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
@@ -715,7 +750,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       int it = 0;  // key tiles processed so far (continues across items)
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
-        QuerySched<CAUSAL, SPARSE> sch{item.tile, p.n_tiles, p.tile_mask};
+        QuerySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_ktiles, off_, p.tile_mask};
         if (!mbar_wait(&bars->q_full, kk & 1, wc, kSiteBwdKV)) { ok = false; break; }
         tc_fence_after();
         int jj = sch.first();
@@ -791,7 +826,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     BwdItem item;
     for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
       const int i = item.tile;
-      QuerySched<CAUSAL, SPARSE> sch{i, p.n_tiles, p.tile_mask};
+      QuerySched<CAUSAL, SPARSE, XQK> sch{i, p.n_ktiles, off_, p.tile_mask};
       const size_t row = size_t(item.bh) * p.N + size_t(i) * 128 + r;
       const size_t prow = (size_t(item.bh) * p.n_tiles + size_t(i)) * 128 + r;  // padded row arrays
       const float l2 = p.lse2[prow];
@@ -803,7 +838,15 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           break;
         }
         tc_fence_after();
-        const bool diag = CAUSAL && (jj == i);  // key c visible to query r iff c <= r
+        // Key 128 jj + c is visible to query 128 i + r iff c <= r + cbase; the tile is
+        // partial (element mask) iff cbase < 127.
+        int cbase = 0;  // N_q = N_k: only the diagonal tile (jj == i) is partial, with cbase 0
+        if constexpr (XQK) {
+          const long long cb64 = 128LL * (i - jj) + off_;  // clamped: beyond +-256 no row is partial
+          cbase = static_cast<int>(cb64 < -256 ? -256 : (cb64 > 256 ? 256 : cb64));
+        }
+        const bool diag = CAUSAL && (XQK ? cbase < 127 : jj == i);
+        const int cmax = cbase + r;
         uint32_t pk[32];
         {
           uint32_t raw[64];
@@ -818,7 +861,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 f2_fma(f2(__uint_as_float(raw[2 * t]), __uint_as_float(raw[2 * t + 1])), c2v, nl2), t);
             if (diag) {
               const float2 v = f2_split(pv);
-              pv = f2((h * 64 + 2 * t > r) ? 0.f : v.x, (h * 64 + 2 * t + 1 > r) ? 0.f : v.y);
+              pv = f2((h * 64 + 2 * t > cmax) ? 0.f : v.x, (h * 64 + 2 * t + 1 > cmax) ? 0.f : v.y);
             }
             const float2 v = f2_split(pv);
             pk[t] = pack_bf16(v.x, v.y);

@@ -40,9 +40,12 @@ struct FwdParams {
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;               // library status word (global)
   unsigned long long timeout_ns;
-  int N;                     // sequence length (any N >= 1)
+  int N;                     // query rows N_q (any N >= 1)
+  int Nk;                    // key rows N_k (any N_k >= 1)
   int BH;                    // B * H
-  int n_tiles;               // ceil(N / 128); the last tile holds N - 128 (n_tiles - 1) rows
+  int n_tiles;               // query tiles ceil(N_q / 128); the last may be partial
+  int n_ktiles;              // key tiles ceil(N_k / 128)
+  int off;                   // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
   int n_qblocks;             // ceil(n_tiles / 2)
   int n_items;               // n_qblocks * BH work items (query block, batch*head)
   float c_log2;              // scale * log2(e)
@@ -114,23 +117,35 @@ __device__ __forceinline__ bool fwd_item(int n_items, int n_qblocks, int BH, int
   return true;
 }
 
+// Last key tile that query tile t sees with the causal mask (key j visible to query i
+// iff j <= i + off), clamped to the key tiles; -1 when the tile sees no key.
+__device__ __forceinline__ int causal_klast(int t, int off, int n_ktiles) {
+  const long long x = 128LL * t + 127 + off;  // last key the tile's last row sees
+  const long long l = x < 0 ? -1 : (x >> 7);
+  return static_cast<int>(l < n_ktiles - 1 ? l : n_ktiles - 1);
+}
+
 // Which of the CTA's two Q tiles need K/V tile j (bit 0: tile 0, bit 1: tile 1); the
 // K/V tiles are visited in increasing order. (Visiting the causal tiles diagonal-first,
 // or tile 1's extra diagonal tile earlier, was measured: up to 6% faster at N = 2048 but
 // 1-2% slower at N >= 8192, so the plain order stays.)
-template <bool CAUSAL, bool SPARSE>
+template <bool CAUSAL, bool SPARSE, bool XQK>
 struct FwdSched {
   int t0, t1;
   bool valid1;
-  int n_tiles;
+  int n_ktiles;
+  int klast0, klast1;  // causal with N_q != N_k (XQK): last key tile of Q tile 0 / 1
   const uint8_t* mask;
-  __device__ __forceinline__ int last() const { return CAUSAL ? (valid1 ? t1 : t0) : n_tiles - 1; }
+  // With N_q = N_k the causal limit of Q tile t is key tile t (its diagonal).
+  __device__ __forceinline__ int kl0() const { return XQK ? klast0 : t0; }
+  __device__ __forceinline__ int kl1() const { return XQK ? klast1 : t1; }
+  __device__ __forceinline__ int last() const { return CAUSAL ? (valid1 ? kl1() : kl0()) : n_ktiles - 1; }
   __device__ __forceinline__ uint32_t bits(int j) const {
-    bool k0 = CAUSAL ? (j <= t0) : true;
-    bool k1 = valid1 && (CAUSAL ? (j <= t1) : true);
+    bool k0 = CAUSAL ? (j <= kl0()) : true;
+    bool k1 = valid1 && (CAUSAL ? (j <= kl1()) : true);
     if (SPARSE) {
-      k0 = k0 && (mask[size_t(t0) * n_tiles + j] != 0);
-      k1 = k1 && (mask[size_t(t1) * n_tiles + j] != 0);
+      k0 = k0 && (mask[size_t(t0) * n_ktiles + j] != 0);
+      k1 = k1 && (mask[size_t(t1) * n_ktiles + j] != 0);
     }
     return (k0 ? 1u : 0u) | (k1 ? 2u : 0u);
   }
@@ -220,12 +235,14 @@ constexpr int kFwdRegsCtl = 104;
 constexpr int kFwdRegsSoftmax = 184;
 constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK>
 __global__ void __launch_bounds__(384, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int S = Cfg::kStages;
+  // Causal offset N_k - N_q: a compile-time 0 in the N_q = N_k kernels (XQK false).
+  const int off_ = XQK ? p.off : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   FwdBars<S>* bars = reinterpret_cast<FwdBars<S>*>(smem + Cfg::kOffBar);
@@ -237,11 +254,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int warp = warp_id();
   const int lane = lane_id();
   auto sched_of = [&](const FwdItem& item) {
-    FwdSched<CAUSAL, SPARSE> sch;
+    FwdSched<CAUSAL, SPARSE, XQK> sch;
     sch.t0 = 2 * item.qb;
     sch.t1 = 2 * item.qb + 1;
     sch.valid1 = sch.t1 < p.n_tiles;
-    sch.n_tiles = p.n_tiles;
+    sch.n_ktiles = p.n_ktiles;
+    sch.klast0 = XQK ? causal_klast(sch.t0, off_, p.n_ktiles) : 0;
+    sch.klast1 = XQK ? causal_klast(sch.t1, off_, p.n_ktiles) : 0;
     sch.mask = p.tile_mask;
     return sch;
   };
@@ -486,16 +505,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
           tmem_wait_ld();
           float sum, alpha, m_use;
-          // Masked columns: above the diagonal (causal), or keys past N in the last
-          // K/V tile (with the causal mask those are above the diagonal of every row
-          // that exists). The choice of variant is per tile, so warp-uniform.
-          const bool diag = CAUSAL && j == tile;
-          const bool tail = !CAUSAL && j == p.n_tiles - 1 && (p.N & 127) != 0;
-          if (diag || tail)
-            softmax_row<true, PolyShare<D>::kFwd>(s, diag ? r + 1 : p.N - 128 * j, c, m, trow + Cfg::tm_p(i), sum,
-                                                  alpha, m_use);
-          else
+          // Masked columns: keys past the causal limit (key 128 j + t is visible to
+          // row 128 tile + r iff t < r + 1 + 128 (tile - j) + off), and keys past N_k in
+          // the last K/V tile. The choice of variant is per tile, so warp-uniform.
+          // Row r sees t < r + 1 + dbase; dbase is clamped to [-256, 256], beyond which
+          // a tile is fully hidden or fully visible for every row.
+          int dbase = 0;  // N_q = N_k: only the diagonal tile (j == tile) is partial, with dbase 0
+          if constexpr (XQK) {
+            const long long db64 = 128LL * (tile - j) + off_;
+            dbase = static_cast<int>(db64 < -256 ? -256 : (db64 > 256 ? 256 : db64));
+          }
+          const bool diag = CAUSAL && (XQK ? dbase < 127 : j == tile);
+          // (With the causal mask, keys past N_k are past every existing row's limit.)
+          const int nk_last = p.Nk - 128 * (p.n_ktiles - 1);  // keys in the last K/V tile
+          const bool tail = !CAUSAL && j == p.n_ktiles - 1 && nk_last != 128;
+          if (diag || tail) {
+            int lim = diag ? r + 1 + dbase : nk_last;
+            if (XQK && lim < 0) lim = 0;  // (only an offset makes a row see none of a scheduled tile)
+            softmax_row<true, PolyShare<D>::kFwd>(s, lim, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+          } else {
             softmax_row<false, PolyShare<D>::kFwd>(s, 128, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+          }
           const bool rescale = m_use != m;
           l = l * alpha + sum;
           if (__any_sync(0xffffffffu, rescale) && local > 0) {
@@ -530,7 +560,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __nv_bfloat16* orow = p.o + row * D;
       const bool row_ok = tile * 128 + r < p.N;  // rows past N (last tile) do not exist
       if (active && local > 0) {
-        const float inv_l = 1.f / l;
+        // l = 0: the row saw no key (causal with N_q > N_k): O = 0, lse = -inf.
+        const float inv_l = (!XQK || l > 0.f) ? 1.f / l : 0.f;
         uint32_t ov[D];
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc)
@@ -564,11 +595,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int t = 0; t < 4; ++t) dst[t] = pk[t];
           }
         }
-        if (row_ok) p.lse[row] = (m + __log2f(l)) * 0.69314718055994531f;
+        if (row_ok) p.lse[row] = (!XQK || l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       } else {
         mbar_arrive(&bars->o_empty[i]);
         if (active && row_ok) {
-          // No visible key for this row (only possible with a block mask).
+          // No visible key for this row (a block mask, or causal with N_q > N_k).
           const uint4 z = make_uint4(0, 0, 0, 0);
           uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll

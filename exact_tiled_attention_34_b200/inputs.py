@@ -27,6 +27,9 @@ WORKLOADS = {
     # Sequence lengths that are not a multiple of the 128-row tile (last tile partial).
     "b8h16n2000d64_ragged": dict(B=8, H=16, N=2000, d=64, causal=(False, True), backward=True),
     "b2h16n8000d128_ragged_causal": dict(B=2, H=16, N=8000, d=128, causal=(True,), backward=True),
+    # Different query and key lengths: 512 new queries against 8192 keys (chunked
+    # prefill), causal mask aligned bottom-right.
+    "b4h16q512k8192d128_causal": dict(B=4, H=16, N=512, Nk=8192, d=128, causal=(True,), backward=True),
 }
 
 SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384)

@@ -86,6 +86,19 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * Forward with different query and key lengths (cross-attention, or a block of new
+ * queries against a longer key sequence as in decoding). No counterpart on the
+ * pages beyond the square problem; fa_fwd(..., N, ...) is fa_fwd_qk(..., N, N, ...).
+ *   q, o    : [B,H,Nq,d] bf16;  k, v : [B,H,Nk,d] bf16;  lse : [B,H,Nq] fp32.
+ *   causal  : 1 = key j is visible to query i iff j <= i + (Nk - Nq) (bottom-right
+ *             alignment: the last query sees every key). With Nq > Nk the first
+ *             Nq - Nk queries see no key: their O rows are 0 and lse -INFINITY.
+ * Other arguments and rules as for fa_fwd.
+ */
+fa_status fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int Nq, int Nk, int d, int causal, float scale, void* stream);
+
+/*
  * Block-sparse forward (the summary's block-sparse paragraph): as fa_fwd without
  * the causal flag, restricted to the kept tiles of `tile_mask`. Skipped tiles
  * cost neither loads nor matrix products. mask_block must be 128.
@@ -121,6 +134,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const void* dO, void* dq, void* dk, void* dv,
                  void* workspace, size_t workspace_bytes,
                  int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Backward of fa_fwd_qk: dq [B,H,Nq,d], dk and dv [B,H,Nk,d]; o, lse and dO have Nq
+ * rows. The workspace holds per-query rows: fa_bwd_workspace_bytes(B, H, Nq, d).
+ * fa_bwd(..., N, ...) is fa_bwd_qk(..., N, N, ...).
+ */
+fa_status fa_bwd_qk(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dO, void* dq, void* dk, void* dv,
+                    void* workspace, size_t workspace_bytes,
+                    int B, int H, int Nq, int Nk, int d, int causal, float scale, void* stream);
 
 /* Block-sparse backward: fa_bwd restricted to the kept tiles of `tile_mask`. */
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,

@@ -66,6 +66,17 @@ def test_fwd_argument_checks(L):
     assert _fwd(L, scale=float("inf")) == INVALID
 
 
+def test_cross_argument_checks(L):
+    f = L.fa_fwd_qk
+    assert f(A, A, A, A, A, 1, 1, 128, 0, 64, 0, 0.1, None) == INVALID
+    assert f(A, A, A, A, A, 1, 1, 0, 128, 64, 0, 0.1, None) == INVALID
+    assert f(A, A, A, A, A, 1, 1, 128, 256, 96, 0, 0.1, None) == UNSUPPORTED
+    assert f(A, A, A, A, A, 1, 1, 100, 300, 64, 1, 0.1, None) == _fwd(L)  # valid: as far as a square call
+    g = L.fa_bwd_qk
+    assert g(A, A, A, A, A, A, A, A, A, A, 1 << 20, 1, 1, 128, 0, 64, 0, 0.1, None) == INVALID
+    assert g(A, A, A, A, A, A, A, A, A, A, 0, 1, 1, 128, 64, 64, 0, 0.1, None) == WORKSPACE
+
+
 def test_blocksparse_argument_checks(L):
     f = L.fa_fwd_blocksparse
     assert f(A, A, A, A, A, None, 128, 1, 1, 128, 64, 0.1, None) == INVALID
