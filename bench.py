@@ -509,7 +509,7 @@ def run_table(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse", "b8h16n2000d64_ragged",
-             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal"]
+             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal", "b4h16n4096d96"]
     names += [f"sweep_N{N}_d{d}{c}" for d in SWEEP_D for N in SWEEP_N for c in ("", "_causal")]
     if args.only:
         names = [n for n in names if any(o in n for o in args.only.split(","))]

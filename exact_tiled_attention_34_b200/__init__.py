@@ -14,7 +14,7 @@ Tensors are bf16 contiguous on one CUDA device: q, o, do [B, H, Nq, d]; k, v
 [B, H, Nk, d]; lse fp32 [B, H, Nq]. Nq and Nk may differ (then the causal mask is
 bottom-right aligned: query i sees key j iff j <= i + Nk - Nq); the block-sparse
 calls need Nq = Nk = N and a uint8 tile_mask [ceil(N/128), ceil(N/128)]. Any N >= 1,
-d in {64, 128}.
+d in {64, 96, 128}.
 """
 from __future__ import annotations
 
@@ -26,7 +26,7 @@ import re
 __all__ = [
     "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
     "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_dkdv",
-    "bwd_dq",
+    "bwd_dq", "attention", "attention_blocksparse",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -278,3 +278,57 @@ def debug_exp2(x, mode: int):
         st = lib().fa_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), mode, _stream_ptr(x.device))
     _check(st, "fa_debug_exp2")
     return y
+
+
+# ---------------------------------------------------------------- autograd
+# torch.autograd glue around forward/backward: the forward saves q, k, v, o and lse,
+# the backward hands them with dO to the library's backward. Marshalling only.
+
+def _autograd_fn():
+    import torch
+
+    class _Attention(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q, k, v, causal, scale, tile_mask):
+            if tile_mask is None:
+                o, lse = forward(q, k, v, causal=causal, scale=scale)
+            else:
+                o, lse = forward_blocksparse(q, k, v, tile_mask, scale=scale)
+            ctx.save_for_backward(q, k, v, o, lse)
+            ctx.causal, ctx.scale, ctx.tile_mask = causal, scale, tile_mask
+            ctx.mark_non_differentiable(lse)
+            return o, lse
+
+        @staticmethod
+        def backward(ctx, do, _dlse):
+            q, k, v, o, lse = ctx.saved_tensors
+            do = do.contiguous()
+            if ctx.tile_mask is None:
+                dq, dk, dv = backward(q, k, v, o, lse, do, causal=ctx.causal, scale=ctx.scale)
+            else:
+                dq, dk, dv = backward_blocksparse(q, k, v, o, lse, do, ctx.tile_mask, scale=ctx.scale)
+            return dq, dk, dv, None, None, None
+
+    return _Attention
+
+
+_ATTN = None
+
+
+def attention(q, k, v, causal: bool = False, scale=None):
+    """Differentiable O = softmax(scale q k^T [causal]) v for torch.autograd: the
+    forward and backward run in the library (q, k, v as for ``forward``)."""
+    global _ATTN
+    if _ATTN is None:
+        _ATTN = _autograd_fn()
+    o, _ = _ATTN.apply(q, k, v, bool(causal), scale, None)
+    return o
+
+
+def attention_blocksparse(q, k, v, tile_mask, scale=None):
+    """Differentiable block-sparse attention (see ``forward_blocksparse``)."""
+    global _ATTN
+    if _ATTN is None:
+        _ATTN = _autograd_fn()
+    o, _ = _ATTN.apply(q, k, v, False, scale, tile_mask)
+    return o

@@ -28,7 +28,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 fa_status check_sizes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
   // Padded rows (N rounded up to whole 128-row tiles) index the backward's row arrays.
   const long long rows = static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128 * 128);
   if (rows > INT_MAX || static_cast<long long>(B) * H > INT_MAX / 2) return FA_ERR_UNSUPPORTED;
@@ -116,13 +116,13 @@ fa_status set_smem(K kernel, int bytes, std::once_flag (&flags)[kMaxDevices], cu
 }
 
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, int DS = D>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK>;
+  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK, DS>;
   constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
   // The kernel re-divides its register pool between warpgroups: refuse to launch a
@@ -175,6 +175,12 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 96) {  // the 128-wide kernels with 96 stored columns
+    if (mask) return launch_fwd<128, false, true, false, 96>(mq, mk, mv, p, st);
+    if (causal && Nk != N) return launch_fwd<128, true, false, true, 96>(mq, mk, mv, p, st);
+    if (causal) return launch_fwd<128, true, false, false, 96>(mq, mk, mv, p, st);
+    return launch_fwd<128, false, false, false, 96>(mq, mk, mv, p, st);
+  }
   if (mask) {
     return d == 64 ? launch_fwd<64, false, true>(mq, mk, mv, p, st) : launch_fwd<128, false, true>(mq, mk, mv, p, st);
   }
@@ -274,15 +280,15 @@ fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, siz
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long threads = static_cast<long long>(a.rows) * (d / 8);
+  const long long threads = static_cast<long long>(a.rows) * (d == 64 ? 8 : 16);  // D / 8 per row
   const unsigned grid = unsigned((threads + 255) / 256);
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   const long long rows = static_cast<long long>(a.rows);
   if (d == 64)
-    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, rows);
-  else
-    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, rows);
+    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, rows);
+  else  // 96 or 128 (16 threads per row)
+    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, rows);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -325,6 +331,7 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.n_tiles = (N + 127) / 128;
   p.n_ktiles = (Nk + 127) / 128;
   p.off = Nk - N;
+  p.ds = d;
   p.scale = scale;
 #define FA_BWD_DISPATCH(LAUNCH)                                                                  \
   if (mask)                                                                                      \

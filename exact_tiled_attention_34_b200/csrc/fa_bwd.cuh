@@ -46,12 +46,12 @@ namespace fa {
 // row arrays hold Npad = 128 * ceil(N / 128) rows per (batch, head): a tile's rows are
 // one 512-byte run. The pad rows of the last tile (n >= N, when N % 128 != 0) get
 // D = 0 and nl2 = -inf, so their recomputed P is 0 and they add nothing to dK or dV.
-// D / 8 threads per row, 16 bytes each.
+// D / 8 threads per row, 16 bytes each; rows hold ds <= D columns (96 with D = 128).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse, float* __restrict__ Drow,
-                                                         float* __restrict__ lse2, int N, int Npad,
+                                                         float* __restrict__ lse2, int N, int Npad, int ds,
                                                          long long rows_pad) {
   constexpr int TPR = D / 8;
   const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -63,9 +63,9 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   const bool valid = inrange && n < N;
   const long long row = bh * N + n;  // row of O, dO and lse
   float s = 0.f;
-  if (valid) {
-    const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
-    const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+  if (valid && part * 8 < ds) {
+    const uint4 a = *reinterpret_cast<const uint4*>(o + row * ds + part * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + row * ds + part * 8);
     const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
@@ -101,6 +101,7 @@ struct BwdParams {
   int n_tiles;          // query tiles ceil(N_q / 128)
   int n_ktiles;         // key tiles ceil(N_k / 128)
   int off;              // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
+  int ds;               // head dim as stored (row length of q, k, v, dO, dq, dk, dv): D, or 96 with D = 128
   float scale;          // softmax scale
 };
 
@@ -234,35 +235,14 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
 }
 
-// NCOL fp32 columns of the thread's TMEM row (times mul, or zeros) as bf16 to dst.
+// The first ncols (a multiple of 32, at most NCOL) of NCOL fp32 values of the thread's
+// row (in registers), times mul, as bf16 to dst.
 template <int NCOL>
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t taddr, float mul, bool zero) {
+__device__ __forceinline__ void store_regs_bf16(__nv_bfloat16* dst, const uint32_t (&v)[NCOL], float mul,
+                                                int ncols) {
 #pragma unroll
   for (int cc = 0; cc < NCOL / 32; ++cc) {
-    uint32_t v[32];
-    if (!zero) {
-      tmem_ld32(taddr + cc * 32, v);
-      tmem_wait_ld();
-    } else {
-#pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] = 0u;
-    }
-    uint4 o4[4];
-    uint32_t* w = reinterpret_cast<uint32_t*>(o4);
-#pragma unroll
-    for (int t = 0; t < 16; ++t)
-      w[t] = pack_bf16(__uint_as_float(v[2 * t]) * mul, __uint_as_float(v[2 * t + 1]) * mul);
-    uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) d4[t] = o4[t];
-  }
-}
-
-// NCOL fp32 values of the thread's row (in registers), times mul, as bf16 to dst.
-template <int NCOL>
-__device__ __forceinline__ void store_regs_bf16(__nv_bfloat16* dst, const uint32_t (&v)[NCOL], float mul) {
-#pragma unroll
-  for (int cc = 0; cc < NCOL / 32; ++cc) {
+    if (cc * 32 >= ncols) break;
     uint4 o4[4];
     uint32_t* w = reinterpret_cast<uint32_t*>(o4);
 #pragma unroll
@@ -618,7 +598,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
       if (j * 128 + r < p.Nk)  // key rows past N_k (last tile, N_k % 128 != 0) do not exist
-        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * D, acc, h == 0 ? p.scale : 1.f);
+        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * p.ds, acc, h == 0 ? p.scale : 1.f, p.ds);
     }
     tc_fence_before();
     __syncthreads();
@@ -916,7 +896,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
       if (i * 128 + r < p.N)  // query rows past N (last tile, N % 128 != 0) do not exist
-        store_regs_bf16<D / 2>(p.dq + row * D + h * (D / 2), acc, p.scale);
+        store_regs_bf16<D / 2>(p.dq + row * p.ds + h * (D / 2), acc, p.scale, p.ds - h * (D / 2));
     }
     tc_fence_before();
     __syncthreads();

@@ -235,7 +235,9 @@ constexpr int kFwdRegsCtl = 104;
 constexpr int kFwdRegsSoftmax = 184;
 constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK>
+// DS: the head dim as stored (row length of q, k, v, o): D, or 96 on the D = 128 kernels
+// (the loads read zeros for columns 96..127; only DS columns of O are written).
+template <int D, bool CAUSAL, bool SPARSE, bool XQK, int DS>
 __global__ void __launch_bounds__(384, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -557,7 +559,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       tc_fence_after();
       const size_t row = size_t(item.bh) * p.N + size_t(tile) * 128 + r;
-      __nv_bfloat16* orow = p.o + row * D;
+      __nv_bfloat16* orow = p.o + row * DS;
       const bool row_ok = tile * 128 + r < p.N;  // rows past N (last tile) do not exist
       if (active && local > 0) {
         // l = 0: the row saw no key (causal with N_q > N_k): O = 0, lse = -inf.
@@ -570,8 +572,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         mbar_arrive(&bars->o_empty[i]);
         if constexpr (Cfg::kStageO) {
-          // O rows of this warp, 64 columns at a time, through the warp's stage.
-          __nv_bfloat16* row0 = p.o + (row - lane) * D;
+          // O rows of this warp, 64 columns at a time, through the warp's stage (the
+          // second block has 32 columns when the stored head dim is 96).
+          __nv_bfloat16* row0 = p.o + (row - lane) * DS;
+          const int nrows = p.N - (tile * 128 + r - lane);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb) {
             uint32_t w[32];
@@ -579,11 +583,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int t = 0; t < 32; ++t)
               w[t] = pack_bf16(__uint_as_float(ov[cb * 64 + 2 * t]) * inv_l,
                                __uint_as_float(ov[cb * 64 + 2 * t + 1]) * inv_l);
-            warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, D, p.N - (tile * 128 + r - lane));
+            if constexpr (DS == D) {
+              warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, DS, nrows);
+            } else if (cb * 64 + 64 <= DS) {
+              warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, DS, nrows);
+            } else if (cb * 64 + 32 == DS) {
+              uint32_t w16[16];
+#pragma unroll
+              for (int t = 0; t < 16; ++t) w16[t] = w[t];
+              warp_store_rows<16>(sStage + (warp - 4) * 1024, w16, row0 + cb * 64, DS, nrows);
+            }
           }
         } else if (row_ok) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
+            if (cc * 32 >= DS) break;
             uint4 pk[4];
             uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
@@ -603,7 +617,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const uint4 z = make_uint4(0, 0, 0, 0);
           uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-          for (int t = 0; t < D / 8; ++t) dst[t] = z;
+          for (int t = 0; t < D / 8; ++t)
+            if (t * 8 < DS) dst[t] = z;
           p.lse[row] = -INFINITY;
         }
       }

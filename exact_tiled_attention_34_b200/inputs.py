@@ -30,6 +30,8 @@ WORKLOADS = {
     # Different query and key lengths: 512 new queries against 8192 keys (chunked
     # prefill), causal mask aligned bottom-right.
     "b4h16q512k8192d128_causal": dict(B=4, H=16, N=512, Nk=8192, d=128, causal=(True,), backward=True),
+    # Head dim 96 (runs on the 128-wide kernels).
+    "b4h16n4096d96": dict(B=4, H=16, N=4096, d=96, causal=(False, True), backward=True),
 }
 
 SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384)

@@ -29,8 +29,10 @@
  *  - All pointers are DEVICE pointers on the current device, except where noted.
  *    Every base pointer must be 16-byte aligned.
  *  - Supported sizes: B, H, N >= 1 (any N; the kernels work on 128-row tiles and
- *    the last tile of a sequence may be partial); d in {64, 128}. B*H*Npad must
- *    fit in int32, where Npad = 128 * ceil(N / 128).
+ *    the last tile of a sequence may be partial); d in {64, 96, 128} (d = 96 runs
+ *    on the d = 128 kernels: the tensor-memory loads read zeros for columns 96..127,
+ *    which leaves every product over the first 96 columns unchanged, and only 96
+ *    columns are stored). B*H*Npad must fit in int32, where Npad = 128 * ceil(N / 128).
  *  - Causal: key j is visible to query i iff j <= i (top-left aligned; N_q = N_k).
  *  - Block mask (tile_mask): uint8 [nT, nT] device array with nT = ceil(N / 128),
  *    row-major, 1 = tile kept, 0 = tile skipped, shared by every (b, h); tile t
@@ -63,7 +65,7 @@ extern "C" {
 typedef enum fa_status {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, non-finite scale */
-  FA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, sizes beyond int32 rows, mask_block != 128 */
+  FA_ERR_UNSUPPORTED = 2,     /* d not in {64,96,128}, sizes beyond int32 rows, mask_block != 128 */
   FA_ERR_ALIGNMENT = 3,       /* a base pointer is not 16-byte aligned */
   FA_ERR_WORKSPACE = 4,       /* workspace too small */
   FA_ERR_CUDA = 5,            /* the CUDA runtime or driver reported an error */

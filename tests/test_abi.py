@@ -56,7 +56,9 @@ def test_fwd_argument_checks(L):
     assert _fwd(L, H=-1) == INVALID
     assert _fwd(L, N=0) == INVALID
     assert _fwd(L, d=32) == UNSUPPORTED
-    assert _fwd(L, d=96) == UNSUPPORTED
+    assert _fwd(L, d=96) == _fwd(L)  # head dim 96 runs on the 128-wide kernels
+    assert _fwd(L, d=80) == UNSUPPORTED
+    assert _fwd(L, d=256) == UNSUPPORTED
     # Any N >= 1 passes validation (the last 128-row tile may be partial): such a call
     # gets as far as a valid one, which on a machine without a GPU is FA_ERR_CUDA.
     assert _fwd(L, N=130) == _fwd(L, N=128) not in (INVALID, UNSUPPORTED, ALIGN)
@@ -70,7 +72,7 @@ def test_cross_argument_checks(L):
     f = L.fa_fwd_qk
     assert f(A, A, A, A, A, 1, 1, 128, 0, 64, 0, 0.1, None) == INVALID
     assert f(A, A, A, A, A, 1, 1, 0, 128, 64, 0, 0.1, None) == INVALID
-    assert f(A, A, A, A, A, 1, 1, 128, 256, 96, 0, 0.1, None) == UNSUPPORTED
+    assert f(A, A, A, A, A, 1, 1, 128, 256, 80, 0, 0.1, None) == UNSUPPORTED
     assert f(A, A, A, A, A, 1, 1, 100, 300, 64, 1, 0.1, None) == _fwd(L)  # valid: as far as a square call
     g = L.fa_bwd_qk
     assert g(A, A, A, A, A, A, A, A, A, A, 1 << 20, 1, 1, 128, 0, 64, 0, 0.1, None) == INVALID
