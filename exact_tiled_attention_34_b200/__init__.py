@@ -14,7 +14,8 @@ Tensors are bf16 contiguous on one CUDA device: q, o, do [B, H, Nq, d]; k, v
 [B, H, Nk, d]; lse fp32 [B, H, Nq]. Nq and Nk may differ (then the causal mask is
 bottom-right aligned: query i sees key j iff j <= i + Nk - Nq); the block-sparse
 calls need Nq = Nk = N and a uint8 tile_mask [ceil(N/128), ceil(N/128)]. Any N >= 1,
-d in {64, 96, 128}.
+d in {64, 96, 128}. forward/backward/attention also take layout="bnhd" for [B, N, H, d]
+tensors (lse stays [B, H, Nq]).
 """
 from __future__ import annotations
 
@@ -55,10 +56,12 @@ _SIGS = {
     "fa_version": ([], _i),
     "fa_fwd": ([_vp] * 5 + [_i] * 5 + [_f, _vp], _i),
     "fa_fwd_qk": ([_vp] * 5 + [_i] * 6 + [_f, _vp], _i),
+    "fa_fwd_ex": ([_vp] * 5 + [_i] * 7 + [_f, _vp], _i),
     "fa_fwd_blocksparse": ([_vp] * 6 + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_workspace_bytes": ([_i] * 4, _sz),
     "fa_bwd": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_qk": ([_vp] * 10 + [_sz] + [_i] * 6 + [_f, _vp], _i),
+    "fa_bwd_ex": ([_vp] * 10 + [_sz] + [_i] * 7 + [_f, _vp], _i),
     "fa_bwd_blocksparse": ([_vp] * 10 + [_sz, _vp, _i] + [_i] * 4 + [_f, _vp], _i),
     "fa_device_status": ([_vp, ctypes.POINTER(_i)], _i),
     "fa_bwd_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
@@ -101,8 +104,22 @@ def _stream_ptr(dev):
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
-def _check_qkv(q, k, v, *qlike):
-    """q and the tensors in qlike (o, dO) are [B, H, Nq, d]; k and v are [B, H, Nk, d]."""
+_LAYOUTS = {"bhnd": 0, "bnhd": 1}
+
+
+def _dims(q, k, layout):
+    """(B, H, Nq, Nk, d) of q [B, H, Nq, d] / k [B, H, Nk, d] ("bhnd") or q [B, Nq, H, d] /
+    k [B, Nk, H, d] ("bnhd")."""
+    if layout not in _LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(_LAYOUTS)}")
+    if layout == "bhnd":
+        return q.shape[0], q.shape[1], q.shape[2], k.shape[2], q.shape[3]
+    return q.shape[0], q.shape[2], q.shape[1], k.shape[1], q.shape[3]
+
+
+def _check_qkv(q, k, v, *qlike, layout="bhnd"):
+    """q and the tensors in qlike (o, dO) share a shape; k and v share one; batch, heads
+    and head dim agree (in the positions of `layout`)."""
     import torch
     for t in (q, k, v) + qlike:
         if not t.is_cuda:
@@ -117,7 +134,8 @@ def _check_qkv(q, k, v, *qlike):
         raise ValueError("expected [B, H, N, d] tensors")
     if k.shape != v.shape or any(t.shape != q.shape for t in qlike):
         raise ValueError("k and v must share a shape, as must q, o and dO")
-    if (q.shape[0], q.shape[1], q.shape[3]) != (k.shape[0], k.shape[1], k.shape[3]):
+    hq, hk = (1, 1) if layout == "bhnd" else (2, 2)
+    if (q.shape[0], q.shape[hq], q.shape[3]) != (k.shape[0], k.shape[hk], k.shape[3]):
         raise ValueError("q and k must agree in batch, heads and head dim")
 
 
@@ -125,16 +143,19 @@ def _scale(scale, d):
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
-def forward(q, k, v, causal: bool = False, scale=None, out=None, lse=None):
-    """O = softmax(scale q k^T [causal]) v and the fp32 row log-sum-exp."""
+def forward(q, k, v, causal: bool = False, scale=None, out=None, lse=None, layout: str = "bhnd"):
+    """O = softmax(scale q k^T [causal]) v and the fp32 row log-sum-exp [B, H, Nq]."""
     import torch
-    _check_qkv(q, k, v)
-    B, H, N, d = q.shape
-    Nk = k.shape[2]
+    _check_qkv(q, k, v, layout=layout)
+    B, H, N, Nk, d = _dims(q, k, layout)
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     with torch.cuda.device(q.device):
-        if Nk == N:
+        if layout != "bhnd":
+            st = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                 B, H, N, Nk, d, _LAYOUTS[layout], int(bool(causal)), _scale(scale, d),
+                                 _stream_ptr(q.device))
+        elif Nk == N:
             st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                               B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
         else:
@@ -173,10 +194,10 @@ def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
 
 
-def _bwd_prep(q, k, v, o, lse, do, workspace, grads):
+def _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout="bhnd"):
     import torch
-    _check_qkv(q, k, v, o, do)
-    B, H, N, d = q.shape
+    _check_qkv(q, k, v, o, do, layout=layout)
+    B, H, N, _, d = _dims(q, k, layout)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
         raise ValueError("lse must be contiguous fp32 [B, H, N]")
     need = bwd_workspace_bytes(B, H, N, d)
@@ -187,14 +208,19 @@ def _bwd_prep(q, k, v, o, lse, do, workspace, grads):
     return workspace, grads
 
 
-def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None, grads=None):
+def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None, grads=None,
+             layout: str = "bhnd"):
     """Gradients (dq, dk, dv) of sum(O * dO) given the forward's o and lse."""
     import torch
-    workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
-    B, H, N, d = q.shape
-    Nk = k.shape[2]
+    workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout)
+    B, H, N, Nk, d = _dims(q, k, layout)
     with torch.cuda.device(q.device):
-        if Nk == N:
+        if layout != "bhnd":
+            st = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                 workspace.numel(), B, H, N, Nk, d, _LAYOUTS[layout], int(bool(causal)),
+                                 _scale(scale, d), _stream_ptr(q.device))
+        elif Nk == N:
             st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
                               B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
@@ -289,13 +315,13 @@ def _autograd_fn():
 
     class _Attention(torch.autograd.Function):
         @staticmethod
-        def forward(ctx, q, k, v, causal, scale, tile_mask):
+        def forward(ctx, q, k, v, causal, scale, tile_mask, layout):
             if tile_mask is None:
-                o, lse = forward(q, k, v, causal=causal, scale=scale)
+                o, lse = forward(q, k, v, causal=causal, scale=scale, layout=layout)
             else:
                 o, lse = forward_blocksparse(q, k, v, tile_mask, scale=scale)
             ctx.save_for_backward(q, k, v, o, lse)
-            ctx.causal, ctx.scale, ctx.tile_mask = causal, scale, tile_mask
+            ctx.causal, ctx.scale, ctx.tile_mask, ctx.layout = causal, scale, tile_mask, layout
             ctx.mark_non_differentiable(lse)
             return o, lse
 
@@ -304,10 +330,10 @@ def _autograd_fn():
             q, k, v, o, lse = ctx.saved_tensors
             do = do.contiguous()
             if ctx.tile_mask is None:
-                dq, dk, dv = backward(q, k, v, o, lse, do, causal=ctx.causal, scale=ctx.scale)
+                dq, dk, dv = backward(q, k, v, o, lse, do, causal=ctx.causal, scale=ctx.scale, layout=ctx.layout)
             else:
                 dq, dk, dv = backward_blocksparse(q, k, v, o, lse, do, ctx.tile_mask, scale=ctx.scale)
-            return dq, dk, dv, None, None, None
+            return dq, dk, dv, None, None, None, None
 
     return _Attention
 
@@ -315,13 +341,13 @@ def _autograd_fn():
 _ATTN = None
 
 
-def attention(q, k, v, causal: bool = False, scale=None):
+def attention(q, k, v, causal: bool = False, scale=None, layout: str = "bhnd"):
     """Differentiable O = softmax(scale q k^T [causal]) v for torch.autograd: the
-    forward and backward run in the library (q, k, v as for ``forward``)."""
+    forward and backward run in the library (q, k, v and layout as for ``forward``)."""
     global _ATTN
     if _ATTN is None:
         _ATTN = _autograd_fn()
-    o, _ = _ATTN.apply(q, k, v, bool(causal), scale, None)
+    o, _ = _ATTN.apply(q, k, v, bool(causal), scale, None, layout)
     return o
 
 
@@ -330,5 +356,5 @@ def attention_blocksparse(q, k, v, tile_mask, scale=None):
     global _ATTN
     if _ATTN is None:
         _ATTN = _autograd_fn()
-    o, _ = _ATTN.apply(q, k, v, False, scale, tile_mask)
+    o, _ = _ATTN.apply(q, k, v, False, scale, tile_mask, "bhnd")
     return o

@@ -93,12 +93,23 @@ fa_status encoder() {
 
 // [BH, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 columns x
 // `box_rows` rows with 128-byte swizzle, matching the MMA operand layout.
-fa_status make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * d * 2};
-  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+fa_status make_map(CUtensorMap* m, const void* base, int B, int H, int N, int d, bool bnhd, int box_rows) {
+  // Coordinates (column, row, head, batch) for both layouts; only the strides differ:
+  // [B, H, N, d] rows are d apart and heads N*d; [B, N, H, d] rows are H*d apart and heads d.
+  const cuuint64_t e = 2;  // bytes per element
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(H), cuuint64_t(B)};
+  cuuint64_t strides[3];
+  if (bnhd) {
+    strides[0] = cuuint64_t(H) * d * e;
+    strides[1] = cuuint64_t(d) * e;
+  } else {
+    strides[0] = cuuint64_t(d) * e;
+    strides[1] = cuuint64_t(N) * d * e;
+  }
+  strides[2] = cuuint64_t(N) * H * d * e;
+  cuuint32_t box[4] = {64, cuuint32_t(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
@@ -144,8 +155,10 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 }
 
 fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
-                     int B, int H, int N, int Nk, int d, int causal, float scale, void* stream) {
+                     int B, int H, int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
   fa_status s;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
+  const bool bnhd = layout == FA_LAYOUT_BNHD;
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
@@ -156,9 +169,9 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   if ((s = device_status_ptr(&status)) != FA_OK) return s;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
-  if ((s = make_map(&mq, q, BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mk, k, BH, Nk, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mv, v, BH, Nk, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mq, q, B, H, N, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
   fa::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -168,6 +181,8 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.N = N;
   p.Nk = Nk;
   p.BH = BH;
+  p.H = H;
+  p.bnhd = bnhd ? 1 : 0;
   p.n_tiles = (N + 127) / 128;
   p.n_ktiles = (Nk + 127) / 128;
   p.off = Nk - N;
@@ -274,8 +289,10 @@ fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d,
 }
 
 fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, size_t ws_bytes, int B, int H, int N,
-                  int d, void* stream) {
+                  int d, int layout, void* stream) {
   fa_status s;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
+  const int bnhd = layout == FA_LAYOUT_BNHD ? 1 : 0;
   if ((s = check_ptrs({o, dO, lse})) != FA_OK) return s;
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
@@ -286,9 +303,9 @@ fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, siz
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   const long long rows = static_cast<long long>(a.rows);
   if (d == 64)
-    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, rows);
+    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows);
   else  // 96 or 128 (16 threads per row)
-    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, rows);
+    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -298,8 +315,10 @@ enum class BwdStage { kDkdv, kDq };
 // N: query rows (the workspace's rows), Nk: key rows.
 fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v, const void* dO, void* out0,
                     void* out1, const void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H,
-                    int N, int Nk, int d, int causal, float scale, void* stream) {
+                    int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
   fa_status s;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
+  const bool bnhd = layout == FA_LAYOUT_BNHD;
   if ((s = check_ptrs({q, k, v, dO, out0})) != FA_OK) return s;
   if (stage == BwdStage::kDkdv && (s = check_ptrs({out1})) != FA_OK) return s;
   if (mask != nullptr && (mask_block != 128 || causal || Nk != N)) return FA_ERR_UNSUPPORTED;
@@ -311,10 +330,10 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   int* status;
   if ((s = device_status_ptr(&status)) != FA_OK) return s;
   CUtensorMap mq, mk, mv, mdo;
-  if ((s = make_map(&mq, q, a.BH, N, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mk, k, a.BH, Nk, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mv, v, a.BH, Nk, d, 128)) != FA_OK) return s;
-  if ((s = make_map(&mdo, dO, a.BH, N, d, 128)) != FA_OK) return s;
+  if ((s = make_map(&mq, q, B, H, N, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mdo, dO, B, H, N, d, bnhd, 128)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fa::BwdParams p;
   p.lse2 = a.lse2;
@@ -328,6 +347,8 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.N = N;
   p.Nk = Nk;
   p.BH = a.BH;
+  p.H = H;
+  p.bnhd = bnhd ? 1 : 0;
   p.n_tiles = (N + 127) / 128;
   p.n_ktiles = (Nk + 127) / 128;
   p.off = Nk - N;
@@ -354,21 +375,22 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
 
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int B, int H,
-                     int N, int Nk, int d, int causal, float scale, void* stream) {
+                     int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
   fa_status s;
   // Validate everything before the first launch so that an error writes nothing.
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
   if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv})) != FA_OK) return s;
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
-  if ((s = bwd_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, stream)) != FA_OK) return s;
-  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, Nk, d, causal, scale,
-                     stream)) != FA_OK)
+  if ((s = bwd_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, layout, stream)) != FA_OK) return s;
+  if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, Nk, d, layout, causal,
+                     scale, stream)) != FA_OK)
     return s;
-  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, ws, ws_bytes, mask, 128, B, H, N, Nk, d, causal, scale,
-                   stream);
+  return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, ws, ws_bytes, mask, 128, B, H, N, Nk, d, layout, causal,
+                   scale, stream);
 }
 
 __global__ void fa_debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int mode) {
@@ -411,12 +433,17 @@ int fa_version(void) { return 100; }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  int causal, float scale, void* stream) {
-  return fwd_common(q, k, v, o, lse, nullptr, B, H, N, N, d, causal != 0, scale, stream);
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, N, N, d, FA_LAYOUT_BHND, causal != 0, scale, stream);
 }
 
 fa_status fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                     int d, int causal, float scale, void* stream) {
-  return fwd_common(q, k, v, o, lse, nullptr, B, H, Nq, Nk, d, causal != 0, scale, stream);
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, Nq, Nk, d, FA_LAYOUT_BHND, causal != 0, scale, stream);
+}
+
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                    int d, int layout, int causal, float scale, void* stream) {
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, Nq, Nk, d, layout, causal != 0, scale, stream);
 }
 
 fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -424,7 +451,7 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                              void* stream) {
   if (tile_mask == nullptr) return FA_ERR_INVALID_ARG;
   if (mask_block != 128) return FA_ERR_UNSUPPORTED;
-  return fwd_common(q, k, v, o, lse, tile_mask, B, H, N, N, d, 0, scale, stream);
+  return fwd_common(q, k, v, o, lse, tile_mask, B, H, N, N, d, FA_LAYOUT_BHND, 0, scale, stream);
 }
 
 fa_status fa_device_status(void* stream, int* detail) {
@@ -449,34 +476,41 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) { return bwd_ws_bytes(
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                  int causal, float scale, void* stream) {
-  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, N, d, causal != 0,
-                    scale, stream);
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, N, d,
+                    FA_LAYOUT_BHND, causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_qk(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                     void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Nq,
                     int Nk, int d, int causal, float scale, void* stream) {
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, Nq, Nk, d,
+                    FA_LAYOUT_BHND, causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int Nq,
+                    int Nk, int d, int layout, int causal, float scale, void* stream) {
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, Nq, Nk, d, layout,
                     causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace,
                             size_t workspace_bytes, int B, int H, int N, int d, void* stream) {
-  return bwd_pre(o, dO, lse, workspace, workspace_bytes, B, H, N, d, stream);
+  return bwd_pre(o, dO, lse, workspace, workspace_bytes, B, H, N, d, FA_LAYOUT_BHND, stream);
 }
 
 fa_status fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                       const void* workspace, size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B,
                       int H, int N, int d, int causal, float scale, void* stream) {
   return bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N,
-                   N, d, causal != 0, scale, stream);
+                   N, d, FA_LAYOUT_BHND, causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, const void* workspace,
                     size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B, int H, int N, int d,
                     int causal, float scale, void* stream) {
   return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, workspace, workspace_bytes, tile_mask, mask_block, B, H,
-                   N, N, d, causal != 0, scale, stream);
+                   N, N, d, FA_LAYOUT_BHND, causal != 0, scale, stream);
 }
 
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -485,8 +519,8 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
                              void* stream) {
   if (tile_mask == nullptr) return FA_ERR_INVALID_ARG;
   if (mask_block != 128) return FA_ERR_UNSUPPORTED;
-  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, B, H, N, N, d, 0, scale,
-                    stream);
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, B, H, N, N, d,
+                    FA_LAYOUT_BHND, 0, scale, stream);
 }
 
 }  // extern "C"
@@ -541,10 +575,10 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
   // The pre-pass rewrites every row the other two launches read, so whatever an
   // earlier call left in the array does not matter.
   const size_t bytes = size_t(FA_BWD_NOALLOC_SCRATCH_BYTES);
-  if ((s = bwd_pre(o, dO, lse, scratch, bytes, B, H, N, d, stream)) != FA_OK) return s;
+  if ((s = bwd_pre(o, dO, lse, scratch, bytes, B, H, N, d, FA_LAYOUT_BHND, stream)) != FA_OK) return s;
   if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, scratch, bytes, tile_mask, mask_block, B, H, N, N, d,
-                     causal, scale, stream)) != FA_OK)
+                     FA_LAYOUT_BHND, causal, scale, stream)) != FA_OK)
     return s;
   return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, scratch, bytes, tile_mask, mask_block, B, H, N, N, d,
-                   causal, scale, stream);
+                   FA_LAYOUT_BHND, causal, scale, stream);
 }

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse, float* __restrict__ Drow,
                                                          float* __restrict__ lse2, int N, int Npad, int ds,
-                                                         long long rows_pad) {
+                                                         int H, int bnhd, long long rows_pad) {
   constexpr int TPR = D / 8;
   const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long prow = g / TPR;  // padded row index: bh * Npad + n
@@ -61,11 +61,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   const long long bh = prow / Npad;
   const int n = static_cast<int>(prow - bh * Npad);
   const bool valid = inrange && n < N;
-  const long long row = bh * N + n;  // row of O, dO and lse
+  const long long row = bh * N + n;  // row of lse
   float s = 0.f;
   if (valid && part * 8 < ds) {
-    const uint4 a = *reinterpret_cast<const uint4*>(o + row * ds + part * 8);
-    const uint4 b = *reinterpret_cast<const uint4*>(dO + row * ds + part * 8);
+    const int b_ = static_cast<int>(bh / H), h_ = static_cast<int>(bh - static_cast<long long>(b_) * H);
+    const size_t off = seq_row_offset(b_, h_, n, N, H, ds, bnhd != 0) + part * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
     const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
@@ -98,6 +100,8 @@ struct BwdParams {
   int N;                // query rows N_q (any N >= 1)
   int Nk;               // key rows N_k
   int BH;
+  int H;                // heads (item bh = b * H + h)
+  int bnhd;             // 1: q, k, v, dO, dq, dk, dv are [B, N, H, d]; 0: [B, H, N, d]
   int n_tiles;          // query tiles ceil(N_q / 128)
   int n_ktiles;         // key tiles ceil(N_k / 128)
   int off;              // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
@@ -366,12 +370,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
         const int j = item.tile, bh = item.bh;
+        const int ib = bh / p.H, ih = bh - ib * p.H;  // batch, head (tensor-map coordinates)
         KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
         if (kk > 0 && !mbar_wait(&bars->kv_empty, (kk - 1) & 1, wc, kSiteBwdTEmpty)) break;
         mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-          tma_load_3d(sK + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full, cb * 64, j * 128, bh);
-          tma_load_3d(sV + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full, cb * 64, j * 128, bh);
+          tma_load_4d(sK + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full, cb * 64, j * 128, ih, ib);
+          tma_load_4d(sV + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full, cb * 64, j * 128, ih, ib);
         }
         ++nkv;
         for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
@@ -383,10 +388,10 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
           mbar_arrive_expect_tx(&bars->t_full[st], kTileTx);
           for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-            tma_load_3d_hint(sQ + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->t_full[st],
-                             cb * 64, i * 128, bh, keep);
-            tma_load_3d_hint(sDO + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_do, &bars->t_full[st],
-                             cb * 64, i * 128, bh, keep);
+            tma_load_4d_hint(sQ + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->t_full[st],
+                             cb * 64, i * 128, ih, ib, keep);
+            tma_load_4d_hint(sDO + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_do, &bars->t_full[st],
+                             cb * 64, i * 128, ih, ib, keep);
           }
           const size_t roff = (size_t(bh) * p.n_tiles + size_t(i)) * 128;  // padded row arrays
           bulk_load(sL + st * 128, p.lse2 + roff, 512, &bars->t_full[st]);
@@ -583,7 +588,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         break;
       }
       tc_fence_after();
-      const size_t row = size_t(item.bh) * p.Nk + size_t(j) * 128 + r;  // key row
+      const int ib = item.bh / p.H, ih = item.bh - ib * p.H;
+      const size_t row = seq_row_offset(ib, ih, j * 128 + r, p.Nk, p.H, p.ds, p.bnhd != 0);  // key row (elements)
       uint32_t acc[D];
       if (local > 0) {
 #pragma unroll
@@ -598,7 +604,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
       if (j * 128 + r < p.Nk)  // key rows past N_k (last tile, N_k % 128 != 0) do not exist
-        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row * p.ds, acc, h == 0 ? p.scale : 1.f, p.ds);
+        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row, acc, h == 0 ? p.scale : 1.f, p.ds);
     }
     tc_fence_before();
     __syncthreads();
@@ -688,12 +694,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
         const int i = item.tile, bh = item.bh;
+        const int ib = bh / p.H, ih = bh - ib * p.H;  // batch, head (tensor-map coordinates)
         QuerySched<CAUSAL, SPARSE, XQK> sch{i, p.n_ktiles, off_, p.tile_mask};
         if (kk > 0 && !mbar_wait(&bars->q_empty, (kk - 1) & 1, wc, kSiteBwdTEmpty)) break;
         mbar_arrive_expect_tx(&bars->q_full, 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-          tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, i * 128, bh);
-          tma_load_3d(sDO + cb * Cfg::kBlockBytes, &tm_do, &bars->q_full, cb * 64, i * 128, bh);
+          tma_load_4d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, i * 128, ih, ib);
+          tma_load_4d(sDO + cb * Cfg::kBlockBytes, &tm_do, &bars->q_full, cb * 64, i * 128, ih, ib);
         }
         ++nq;
         for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it) {
@@ -705,10 +712,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           }
           mbar_arrive_expect_tx(&bars->kv_full[st], 2 * Cfg::kTileBytes);
           for (int cb = 0; cb < Cfg::kColBlocks; ++cb) {
-            tma_load_3d_hint(sK + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full[st],
-                             cb * 64, jj * 128, bh, keep);
-            tma_load_3d_hint(sV + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full[st],
-                             cb * 64, jj * 128, bh, keep);
+            tma_load_4d_hint(sK + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full[st],
+                             cb * 64, jj * 128, ih, ib, keep);
+            tma_load_4d_hint(sV + st * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full[st],
+                             cb * 64, jj * 128, ih, ib, keep);
           }
         }
       }
@@ -807,7 +814,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
       const int i = item.tile;
       QuerySched<CAUSAL, SPARSE, XQK> sch{i, p.n_ktiles, off_, p.tile_mask};
-      const size_t row = size_t(item.bh) * p.N + size_t(i) * 128 + r;
+      const int ib = item.bh / p.H, ih = item.bh - ib * p.H;
+      const size_t row = seq_row_offset(ib, ih, i * 128 + r, p.N, p.H, p.ds, p.bnhd != 0);  // query row (elements)
       const size_t prow = (size_t(item.bh) * p.n_tiles + size_t(i)) * 128 + r;  // padded row arrays
       const float l2 = p.lse2[prow];
       const float Dv = p.Drow[prow];
@@ -896,7 +904,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
       if (i * 128 + r < p.N)  // query rows past N (last tile, N % 128 != 0) do not exist
-        store_regs_bf16<D / 2>(p.dq + row * p.ds + h * (D / 2), acc, p.scale, p.ds - h * (D / 2));
+        store_regs_bf16<D / 2>(p.dq + row + h * (D / 2), acc, p.scale, p.ds - h * (D / 2));
     }
     tc_fence_before();
     __syncthreads();

@@ -43,6 +43,8 @@ struct FwdParams {
   int N;                     // query rows N_q (any N >= 1)
   int Nk;                    // key rows N_k (any N_k >= 1)
   int BH;                    // B * H
+  int H;                     // heads (item bh = b * H + h)
+  int bnhd;                  // 1: q, k, v, o are [B, N, H, d]; 0: [B, H, N, d] (lse is [B, H, N] either way)
   int n_tiles;               // query tiles ceil(N_q / 128); the last may be partial
   int n_ktiles;              // key tiles ceil(N_k / 128)
   int off;                   // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
@@ -310,15 +312,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       FwdItem item;
       for (int k = 0; ok && fwd_item<CAUSAL>(p.n_items, p.n_qblocks, p.BH, k, item); ++k) {
         const auto sch = sched_of(item);
+        const int ib = item.bh / p.H, ih = item.bh - ib * p.H;  // batch, head (tensor-map coordinates)
         // The previous item's S products must be done with the Q buffer.
         if (k > 0 && !mbar_wait(&bars->q_empty, (k - 1) & 1, wc, kSiteFwdQEmpty)) break;
         mbar_arrive_expect_tx(&bars->q_full, Cfg::kTileBytes * (sch.valid1 ? 2 : 1));
         for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-          tma_load_3d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, sch.t0 * 128, item.bh);
+          tma_load_4d(sQ + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64, sch.t0 * 128, ih, ib);
         if (sch.valid1)
           for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-            tma_load_3d(sQ + Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64,
-                        sch.t1 * 128, item.bh);
+            tma_load_4d(sQ + Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_q, &bars->q_full, cb * 64,
+                        sch.t1 * 128, ih, ib);
         ++nq;
         uint32_t b;
         for (int j = sch.first(b); j >= 0; j = sch.next(j, b), ++it) {
@@ -332,11 +335,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           uint8_t* dv = sV + st * Cfg::kTileBytes;
           mbar_arrive_expect_tx(&bars->k_full[st], Cfg::kTileBytes);
           for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-            tma_load_3d_hint(dk + cb * Cfg::kBlockBytes, &tm_k, &bars->k_full[st], cb * 64, j * 128, item.bh,
+            tma_load_4d_hint(dk + cb * Cfg::kBlockBytes, &tm_k, &bars->k_full[st], cb * 64, j * 128, ih, ib,
                              keep);
           mbar_arrive_expect_tx(&bars->v_full[st], Cfg::kTileBytes);
           for (int cb = 0; cb < Cfg::kColBlocks; ++cb)
-            tma_load_3d_hint(dv + cb * Cfg::kBlockBytes, &tm_v, &bars->v_full[st], cb * 64, j * 128, item.bh,
+            tma_load_4d_hint(dv + cb * Cfg::kBlockBytes, &tm_v, &bars->v_full[st], cb * 64, j * 128, ih, ib,
                              keep);
         }
       }
@@ -558,8 +561,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      const size_t row = size_t(item.bh) * p.N + size_t(tile) * 128 + r;
-      __nv_bfloat16* orow = p.o + row * DS;
+      const size_t row = size_t(item.bh) * p.N + size_t(tile) * 128 + r;  // lse index
+      const int ib = item.bh / p.H, ih = item.bh - ib * p.H;
+      __nv_bfloat16* orow = p.o + seq_row_offset(ib, ih, tile * 128 + r, p.N, p.H, DS, p.bnhd != 0);
       const bool row_ok = tile * 128 + r < p.N;  // rows past N (last tile) do not exist
       if (active && local > 0) {
         // l = 0: the row saw no key (causal with N_q > N_k): O = 0, lse = -inf.
@@ -574,7 +578,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if constexpr (Cfg::kStageO) {
           // O rows of this warp, 64 columns at a time, through the warp's stage (the
           // second block has 32 columns when the stored head dim is 96).
-          __nv_bfloat16* row0 = p.o + (row - lane) * DS;
+          __nv_bfloat16* row0 = p.o + seq_row_offset(ib, ih, tile * 128 + r - lane, p.N, p.H, DS, p.bnhd != 0);
+          const size_t ld = p.bnhd ? size_t(p.H) * DS : size_t(DS);  // elements between rows
           const int nrows = p.N - (tile * 128 + r - lane);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb) {
@@ -584,14 +589,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               w[t] = pack_bf16(__uint_as_float(ov[cb * 64 + 2 * t]) * inv_l,
                                __uint_as_float(ov[cb * 64 + 2 * t + 1]) * inv_l);
             if constexpr (DS == D) {
-              warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, DS, nrows);
+              warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, ld, nrows);
             } else if (cb * 64 + 64 <= DS) {
-              warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, DS, nrows);
+              warp_store_rows<32>(sStage + (warp - 4) * 1024, w, row0 + cb * 64, ld, nrows);
             } else if (cb * 64 + 32 == DS) {
               uint32_t w16[16];
 #pragma unroll
               for (int t = 0; t < 16; ++t) w16[t] = w[t];
-              warp_store_rows<16>(sStage + (warp - 4) * 1024, w16, row0 + cb * 64, DS, nrows);
+              warp_store_rows<16>(sStage + (warp - 4) * 1024, w16, row0 + cb * 64, ld, nrows);
             }
           }
         } else if (row_ok) {

@@ -72,6 +72,13 @@ typedef enum fa_status {
   FA_ERR_DEVICE_TIMEOUT = 6   /* a kernel gave up waiting (see fa_device_status) */
 } fa_status;
 
+/* Memory layouts of q, k, v, o, dO, dq, dk, dv for fa_fwd_ex / fa_bwd_ex (lse is
+ * [B, H, N] in both). Every other call uses FA_LAYOUT_BHND. */
+enum {
+  FA_LAYOUT_BHND = 0,  /* [B, H, N, d]: element (b, h, n, c) at ((b*H + h)*N + n)*d + c */
+  FA_LAYOUT_BNHD = 1   /* [B, N, H, d]: element (b, n, h, c) at ((b*N + n)*H + h)*d + c */
+};
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(fa_status s);
 
@@ -99,6 +106,15 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  */
 fa_status fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse,
                     int B, int H, int Nq, int Nk, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_fwd_qk with a choice of memory layout: layout = FA_LAYOUT_BHND (as fa_fwd_qk)
+ * or FA_LAYOUT_BNHD ([B, N, H, d] tensors, the row of (b, h, n) H*d elements after
+ * that of (b, h, n - 1)). Any other value: FA_ERR_INVALID_ARG.
+ */
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int Nq, int Nk, int d, int layout, int causal, float scale,
+                    void* stream);
 
 /*
  * Block-sparse forward (the summary's block-sparse paragraph): as fa_fwd without
@@ -146,6 +162,13 @@ fa_status fa_bwd_qk(const void* q, const void* k, const void* v, const void* o, 
                     const void* dO, void* dq, void* dk, void* dv,
                     void* workspace, size_t workspace_bytes,
                     int B, int H, int Nq, int Nk, int d, int causal, float scale, void* stream);
+
+/* fa_bwd_qk with a choice of memory layout (as fa_fwd_ex; lse stays [B, H, Nq]). */
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dO, void* dq, void* dk, void* dv,
+                    void* workspace, size_t workspace_bytes,
+                    int B, int H, int Nq, int Nk, int d, int layout, int causal, float scale,
+                    void* stream);
 
 /* Block-sparse backward: fa_bwd restricted to the kept tiles of `tile_mask`. */
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,

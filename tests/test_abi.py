@@ -79,6 +79,15 @@ def test_cross_argument_checks(L):
     assert g(A, A, A, A, A, A, A, A, A, A, 0, 1, 1, 128, 64, 64, 0, 0.1, None) == WORKSPACE
 
 
+def test_layout_argument_checks(L):
+    f = L.fa_fwd_ex
+    assert f(A, A, A, A, A, 1, 1, 128, 128, 64, 2, 0, 0.1, None) == INVALID   # unknown layout
+    assert f(A, A, A, A, A, 1, 1, 128, 128, 64, -1, 0, 0.1, None) == INVALID
+    assert f(A, A, A, A, A, 1, 1, 128, 128, 64, 1, 0, 0.1, None) == _fwd(L)  # [B, N, H, d]: valid
+    g = L.fa_bwd_ex
+    assert g(A, A, A, A, A, A, A, A, A, A, 1 << 20, 1, 1, 128, 128, 64, 3, 0, 0.1, None) == INVALID
+
+
 def test_blocksparse_argument_checks(L):
     f = L.fa_fwd_blocksparse
     assert f(A, A, A, A, A, None, 128, 1, 1, 128, 64, 0.1, None) == INVALID
