@@ -58,13 +58,15 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   const long long prow = g / TPR;  // padded row index: bh * Npad + n
   const int part = static_cast<int>(g % TPR);
   const bool inrange = prow < rows_pad;
-  const long long bh = prow / Npad;
-  const int n = static_cast<int>(prow - bh * Npad);
+  // rows_pad <= INT_MAX (checked on the host), so 32-bit unsigned division suffices.
+  const unsigned pr = static_cast<unsigned>(inrange ? prow : 0);
+  const unsigned bh = pr / static_cast<unsigned>(Npad);
+  const int n = static_cast<int>(pr - bh * static_cast<unsigned>(Npad));
   const bool valid = inrange && n < N;
-  const long long row = bh * N + n;  // row of lse
+  const long long row = static_cast<long long>(bh) * N + n;  // row of lse
   float s = 0.f;
   if (valid && part * 8 < ds) {
-    const int b_ = static_cast<int>(bh / H), h_ = static_cast<int>(bh - static_cast<long long>(b_) * H);
+    const int b_ = static_cast<int>(bh / static_cast<unsigned>(H)), h_ = static_cast<int>(bh) - b_ * H;
     const size_t off = seq_row_offset(b_, h_, n, N, H, ds, bnhd != 0) + part * 8;
     const uint4 a = *reinterpret_cast<const uint4*>(o + off);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
