@@ -183,6 +183,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.BH = BH;
   p.H = H;
   p.bnhd = bnhd ? 1 : 0;
+  p.v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;  // rows are 128/192/256 B: all aligned alike
   p.n_tiles = (N + 127) / 128;
   p.n_ktiles = (Nk + 127) / 128;
   p.off = Nk - N;
@@ -349,6 +350,8 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.BH = a.BH;
   p.H = H;
   p.bnhd = bnhd ? 1 : 0;
+  // Rows are 128, 192 or 256 bytes, so every row of a 32-byte aligned output is aligned.
+  p.v8 = ((reinterpret_cast<uintptr_t>(out0) | (out1 ? reinterpret_cast<uintptr_t>(out1) : 0)) & 31u) == 0 ? 1 : 0;
   p.n_tiles = (N + 127) / 128;
   p.n_ktiles = (Nk + 127) / 128;
   p.off = Nk - N;

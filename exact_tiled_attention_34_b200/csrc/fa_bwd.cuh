@@ -108,6 +108,7 @@ struct BwdParams {
   int n_ktiles;         // key tiles ceil(N_k / 128)
   int off;              // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
   int ds;               // head dim as stored (row length of q, k, v, dO, dq, dk, dv): D, or 96 with D = 128
+  int v8;               // 1: the gradient outputs are 32-byte aligned (32-byte row stores)
   float scale;          // softmax scale
 };
 
@@ -243,20 +244,18 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 
 // The first ncols (a multiple of 32, at most NCOL) of NCOL fp32 values of the thread's
 // row (in registers), times mul, as bf16 to dst.
+// v8: dst is 32-byte aligned (then 32-byte stores).
 template <int NCOL>
 __device__ __forceinline__ void store_regs_bf16(__nv_bfloat16* dst, const uint32_t (&v)[NCOL], float mul,
-                                                int ncols) {
+                                                int ncols, bool v8) {
 #pragma unroll
   for (int cc = 0; cc < NCOL / 32; ++cc) {
     if (cc * 32 >= ncols) break;
-    uint4 o4[4];
-    uint32_t* w = reinterpret_cast<uint32_t*>(o4);
+    uint32_t w[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t)
       w[t] = pack_bf16(__uint_as_float(v[cc * 32 + 2 * t]) * mul, __uint_as_float(v[cc * 32 + 2 * t + 1]) * mul);
-    uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) d4[t] = o4[t];
+    store_row64(dst + cc * 32, w, v8);
   }
 }
 
@@ -606,7 +605,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
       if (j * 128 + r < p.Nk)  // key rows past N_k (last tile, N_k % 128 != 0) do not exist
-        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row, acc, h == 0 ? p.scale : 1.f, p.ds);
+        store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row, acc, h == 0 ? p.scale : 1.f, p.ds, p.v8 != 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -812,15 +811,24 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float c2 = p.scale * 1.4426950408889634f;
     bool ok = true;
     int it = 0;  // key tiles processed so far (continues across items)
+    // The row values of an item (-lse log2 e and D) are loaded ahead, during the previous
+    // item's epilogue, so that they do not queue behind its row stores.
+    auto row_vals = [&](const BwdItem& x, float& l2_, float& dv_) {
+      const size_t prow = (size_t(x.bh) * p.n_tiles + size_t(x.tile)) * 128 + r;  // padded row arrays
+      l2_ = p.lse2[prow];
+      dv_ = p.Drow[prow];
+    };
     BwdItem item;
-    for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
+    bool have = bwd_item<CAUSAL, false>(p.n_tiles, p.BH, 0, item);
+    float l2_next = 0.f, dv_next = 0.f;
+    if (have) row_vals(item, l2_next, dv_next);
+    for (int kk = 0; ok && have; ++kk) {
       const int i = item.tile;
       QuerySched<CAUSAL, SPARSE, XQK> sch{i, p.n_ktiles, off_, p.tile_mask};
       const int ib = item.bh / p.H, ih = item.bh - ib * p.H;
       const size_t row = seq_row_offset(ib, ih, i * 128 + r, p.N, p.H, p.ds, p.bnhd != 0);  // query row (elements)
-      const size_t prow = (size_t(item.bh) * p.n_tiles + size_t(i)) * 128 + r;  // padded row arrays
-      const float l2 = p.lse2[prow];
-      const float Dv = p.Drow[prow];
+      const float l2 = l2_next;
+      const float Dv = dv_next;
       int local = 0;
       for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it, ++local) {
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
@@ -905,8 +913,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
-      if (i * 128 + r < p.N)  // query rows past N (last tile, N % 128 != 0) do not exist
-        store_regs_bf16<D / 2>(p.dq + row + h * (D / 2), acc, p.scale, p.ds - h * (D / 2));
+      const bool row_ok = i * 128 + r < p.N;  // query rows past N (last tile, N % 128 != 0) do not exist
+      have = bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk + 1, item);
+      if (have) row_vals(item, l2_next, dv_next);
+      if (row_ok) store_regs_bf16<D / 2>(p.dq + row + h * (D / 2), acc, p.scale, p.ds - h * (D / 2), p.v8 != 0);
     }
     tc_fence_before();
     __syncthreads();

@@ -45,6 +45,7 @@ struct FwdParams {
   int BH;                    // B * H
   int H;                     // heads (item bh = b * H + h)
   int bnhd;                  // 1: q, k, v, o are [B, N, H, d]; 0: [B, H, N, d] (lse is [B, H, N] either way)
+  int v8;                    // 1: o is 32-byte aligned (32-byte row stores)
   int n_tiles;               // query tiles ceil(N_q / 128); the last may be partial
   int n_ktiles;              // key tiles ceil(N_k / 128)
   int off;                   // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
@@ -603,15 +604,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             if (cc * 32 >= DS) break;
-            uint4 pk[4];
-            uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+            uint32_t pw[16];
 #pragma unroll
             for (int t = 0; t < 16; ++t)
               pw[t] = pack_bf16(__uint_as_float(ov[cc * 32 + 2 * t]) * inv_l,
                                 __uint_as_float(ov[cc * 32 + 2 * t + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) dst[t] = pk[t];
+            store_row64(orow + cc * 32, pw, p.v8 != 0);
           }
         }
         if (row_ok) p.lse[row] = (!XQK || l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;

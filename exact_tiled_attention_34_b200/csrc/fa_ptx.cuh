@@ -308,6 +308,26 @@ __device__ __forceinline__ void regs_inc() {
 
 // ------------------------------------------------------------------ row stores
 
+// 32 bytes to global memory in one instruction (sm_100); p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// 16 packed words (32 bf16 columns, 64 bytes) of one row: two 32-byte stores when the
+// destination is 32-byte aligned (v8), else four 16-byte stores.
+__device__ __forceinline__ void store_row64(void* dst, const uint32_t (&w)[16], bool v8) {
+  if (v8) {
+    st_global_v8(dst, &w[0]);
+    st_global_v8(static_cast<uint8_t*>(dst) + 32, &w[8]);
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) d4[t] = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+  }
+}
+
 // Stores the calling warp's 32 rows (lane = row) of 2 * NW bf16 values, given as NW
 // packed words per lane, to global rows row0 + lane * ld (ld in elements); rows at or
 // past `nrows` are not written (the tail of the last tile). Each lane's
