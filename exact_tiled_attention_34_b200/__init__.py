@@ -68,6 +68,8 @@ _SIGS = {
     "fa_bwd_dkdv": ([_vp] * 7 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_dq": ([_vp] * 6 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
     "fa_debug_exp2": ([_vp, _vp, _i, _i, _vp], _i),
+    "fa_debug_wait_timeout": ([_i, _vp, _vp], _i),
+    "fa_debug_stall_producer": ([_i, _i], _i),
 }
 
 
@@ -304,6 +306,26 @@ def debug_exp2(x, mode: int):
         st = lib().fa_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), mode, _stream_ptr(x.device))
     _check(st, "fa_debug_exp2")
     return y
+
+
+def debug_wait_timeout(timeout_us: int, device=None):
+    """Run the bounded-wait self-test kernel and return (status, detail, out):
+    the status word after it (as device_status) and out = [warp 0 gave up at its
+    limit, warp 1 left on the abort flag, warp 0's wait in microseconds]."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = torch.full((3,), -1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().fa_debug_wait_timeout(int(timeout_us), out.data_ptr(), _stream_ptr(dev))
+    _check(st, "fa_debug_wait_timeout")
+    status, detail = device_status(dev)
+    return status, detail, out.tolist()
+
+
+def debug_stall_producer(on: bool, timeout_us: int = 2000):
+    """Test hook: while on, attention launches run with an idle TMA producer and a
+    wait limit of timeout_us, so that they end through their timeout path."""
+    _check(lib().fa_debug_stall_producer(1 if on else 0, int(timeout_us)), "fa_debug_stall_producer")
 
 
 # ---------------------------------------------------------------- autograd

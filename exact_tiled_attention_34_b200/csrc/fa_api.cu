@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -21,6 +22,17 @@ constexpr unsigned long long kTimeoutNs = 4000000000ull;  // 4 s per device-side
 
 // Library status word, one per device (module globals are per device).
 __device__ int g_fa_status[2];
+
+// Test hook set by fa_debug_stall_producer: attention launches made while it is on run
+// with an idle TMA producer and this wait limit instead of kTimeoutNs.
+std::atomic<int> g_stall{0};
+std::atomic<unsigned long long> g_stall_limit_ns{kTimeoutNs};
+
+void set_wait_limit(unsigned long long* timeout_ns, int* stall) {
+  const int on = g_stall.load(std::memory_order_acquire);
+  *stall = on;
+  *timeout_ns = on ? g_stall_limit_ns.load(std::memory_order_relaxed) : kTimeoutNs;
+}
 
 // ------------------------------------------------------------------ argument checks
 
@@ -177,7 +189,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.lse = lse;
   p.tile_mask = mask;
   p.status = status;
-  p.timeout_ns = kTimeoutNs;
+  set_wait_limit(&p.timeout_ns, &p.stall);
   p.N = N;
   p.Nk = Nk;
   p.BH = BH;
@@ -344,7 +356,7 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.dv = stage == BwdStage::kDkdv ? static_cast<__nv_bfloat16*>(out1) : nullptr;
   p.tile_mask = mask;
   p.status = status;
-  p.timeout_ns = kTimeoutNs;
+  set_wait_limit(&p.timeout_ns, &p.stall);
   p.N = N;
   p.Nk = Nk;
   p.BH = a.BH;
@@ -406,6 +418,39 @@ __global__ void fa_debug_exp2_kernel(const float* __restrict__ x, float* __restr
   if (i + 1 < n) y[i + 1] = r.y;
 }
 
+// Self-test of the bounded waits: warp w waits on barrier w, which nothing ever
+// completes. Warp 0 has the short limit and so records the timeout (site
+// kSiteDebugWait) and raises the abort flag; warp 1 has a limit 64 times longer and
+// honours the flag, as the kernels' other roles do. No copy, MMA or tensor memory
+// is involved, so nothing is left to drain.
+constexpr int kSiteDebugWait = 901;
+
+__global__ void fa_debug_wait_kernel(unsigned long long timeout_ns, int* status, int* out) {
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int abort_flag;
+  const int w = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar[0], 1);
+    fa::mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    fa::fence_mbar_init();
+  }
+  __syncthreads();
+  const unsigned long long limit = w == 0 ? timeout_ns : 64ull * timeout_ns;
+  const fa::WaitCtl wc{&abort_flag, status, limit};
+  const uint64_t t0 = fa::global_ns();
+  const bool done = __any_sync(0xffffffffu, fa::mbar_wait(&bar[w], 0, wc, kSiteDebugWait + w));
+  const uint64_t dt = fa::global_ns() - t0;
+  if ((threadIdx.x & 31) == 0 && out != nullptr) {
+    if (w == 0) {
+      out[0] = (!done && dt >= limit) ? 1 : 0;
+      out[2] = static_cast<int>(dt / 1000 < INT_MAX ? dt / 1000 : INT_MAX);
+    } else {
+      out[1] = (!done && dt < limit) ? 1 : 0;
+    }
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -417,6 +462,26 @@ fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, void* stream)
   const int pairs = (n + 1) / 2;
   fa_debug_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_wait_timeout(int timeout_us, int* out, void* stream) {
+  if (timeout_us < 1 || timeout_us > 100000) return FA_ERR_INVALID_ARG;
+  if (out != nullptr && (reinterpret_cast<uintptr_t>(out) & 3u) != 0) return FA_ERR_ALIGNMENT;
+  int* status;
+  if (device_status_ptr(&status) != FA_OK) return FA_ERR_CUDA;
+  fa_debug_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * timeout_us, status, out);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_stall_producer(int mode, int timeout_us) {
+  if (mode == 0) {
+    g_stall.store(0, std::memory_order_release);
+    return FA_OK;
+  }
+  if (mode != 1 || timeout_us < 1 || timeout_us > 100000) return FA_ERR_INVALID_ARG;
+  g_stall_limit_ns.store(1000ull * timeout_us, std::memory_order_relaxed);
+  g_stall.store(1, std::memory_order_release);
+  return FA_OK;
 }
 
 const char* fa_status_string(fa_status s) {

@@ -99,6 +99,7 @@ struct BwdParams {
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;
   unsigned long long timeout_ns;
+  int stall;            // test hook: 1 = the producer issues no copies, so every wait runs out
   int N;                // query rows N_q (any N >= 1)
   int Nk;               // key rows N_k
   int BH;
@@ -367,7 +368,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const uint64_t keep = policy_evict_last();
       int it = 0;  // Q/dO tiles loaded so far (ring position, continues across items)
       int nkv = 0;
-      bool ok = true;
+      bool ok = p.stall == 0;
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
         const int j = item.tile, bh = item.bh;
@@ -691,7 +692,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const uint64_t keep = policy_evict_last();
       int it = 0;  // K/V tiles loaded so far (ring position, continues across items)
       int nq = 0;
-      bool ok = true;
+      bool ok = p.stall == 0;
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, false>(p.n_tiles, p.BH, kk, item); ++kk) {
         const int i = item.tile, bh = item.bh;

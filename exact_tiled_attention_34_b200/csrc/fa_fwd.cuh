@@ -40,6 +40,7 @@ struct FwdParams {
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;               // library status word (global)
   unsigned long long timeout_ns;
+  int stall;                 // test hook: 1 = the producer issues no copies, so every wait runs out
   int N;                     // query rows N_q (any N >= 1)
   int Nk;                    // key rows N_k (any N_k >= 1)
   int BH;                    // B * H
@@ -309,7 +310,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const uint64_t keep = policy_evict_last();
       int it = 0;   // K/V tiles loaded so far (ring position, continues across items)
       int nq = 0;   // Q blocks loaded so far
-      bool ok = true;
+      bool ok = p.stall == 0;
       FwdItem item;
       for (int k = 0; ok && fwd_item<CAUSAL>(p.n_items, p.n_qblocks, p.BH, k, item); ++k) {
         const auto sch = sched_of(item);

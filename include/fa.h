@@ -249,6 +249,37 @@ fa_status fa_device_status(void* stream, int* detail);
  */
 fa_status fa_debug_exp2(const float* x, float* y, int n, int mode, void* stream);
 
+/*
+ * Diagnostic for the bounded waits behind FA_ERR_DEVICE_TIMEOUT: launches one block
+ * of two warps on `stream`. Warp 0 waits, with a limit of timeout_us microseconds,
+ * on a shared-memory barrier that nothing completes; when the limit passes it
+ * records FA_ERR_DEVICE_TIMEOUT with detail 901 in the status word and raises the
+ * block's abort flag. Warp 1 waits on a second such barrier with a limit 64 times
+ * longer and leaves when it sees the flag, as the kernels' other roles do. Nothing
+ * traps and the context stays usable; read the result with fa_device_status().
+ *   timeout_us : 1 .. 100000, else FA_ERR_INVALID_ARG (nothing launched).
+ *   out        : device array of 3 ints, or NULL (4-byte aligned, else
+ *                FA_ERR_ALIGNMENT). out[0] = 1 if warp 0 gave up at its limit;
+ *                out[1] = 1 if warp 1 left on the flag before its own limit;
+ *                out[2] = how long warp 0 waited, in microseconds.
+ */
+fa_status fa_debug_wait_timeout(int timeout_us, int* out, void* stream);
+
+/*
+ * Test hook for the bounded waits of the attention kernels themselves. mode 1: every
+ * forward, dK/dV and dQ launch made after this call, by any host thread on any
+ * stream, runs with a TMA producer that issues no copies and with a wait limit of
+ * timeout_us microseconds (1 .. 100000) instead of the usual 4 s. Its other roles
+ * wait for tiles that never arrive, give up at the limit, record
+ * FA_ERR_DEVICE_TIMEOUT and the site of the wait (forward 101..110, backward
+ * 201..211) in the status word, and the kernel returns through its normal teardown
+ * with its outputs unwritten. No copy or matrix product is in flight at any time.
+ * The backward pre-pass has no waits and runs normally. mode 0: normal launches
+ * again (timeout_us ignored). Any other mode or limit: FA_ERR_INVALID_ARG, the
+ * setting unchanged. Never call this while other threads launch work they need.
+ */
+fa_status fa_debug_stall_producer(int mode, int timeout_us);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int fa_version(void);
 

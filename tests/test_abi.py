@@ -23,7 +23,8 @@ def test_exports_every_declared_symbol(L):
     names = fa.exported_names()
     assert {"fa_fwd", "fa_bwd", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_bwd_workspace_bytes",
             "fa_status_string", "fa_device_status", "fa_version", "fa_bwd_preprocess", "fa_bwd_dkdv",
-            "fa_bwd_dq", "fa_bwd_noalloc"} <= set(names)
+            "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_wait_timeout",
+            "fa_debug_stall_producer"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True,
                          check=True).stdout
     defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -106,6 +107,19 @@ def test_workspace_bytes(L):
         assert L.fa_bwd_workspace_bytes(B, H, N, d) == 2 * up(rows * 4)
     assert L.fa_bwd_workspace_bytes(0, 1, 128, 64) == 0
     assert L.fa_bwd_workspace_bytes(1, 1, -128, 64) == 0
+
+
+def test_wait_timeout_argument_checks(L):
+    f = L.fa_debug_wait_timeout
+    assert f(0, A, None) == INVALID
+    assert f(-5, None, None) == INVALID
+    assert f(100001, A, None) == INVALID
+    assert f(1000, A + 2, None) == ALIGN
+    g = L.fa_debug_stall_producer
+    assert g(2, 1000) == INVALID
+    assert g(1, 0) == INVALID
+    assert g(1, 100001) == INVALID
+    assert g(0, -7) == OK  # off: the limit is ignored
 
 
 def test_binding_rejects_cpu_tensors():
