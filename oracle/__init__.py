@@ -11,3 +11,10 @@ from .attention import (  # noqa: F401
     attn_probs_ref,
     attn_scores_ref,
 )
+from .dropout import (  # noqa: F401
+    attn_dropout_bwd_ref,
+    attn_dropout_fwd_ref,
+    dropout_keep_mask,
+    keep_threshold,
+    philox4x32_10,
+)
