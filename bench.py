@@ -60,7 +60,8 @@ def workload(name: str):
     else:
         for c in w["causal"]:
             variants.append(("causal" if c else "noncausal", c, None))
-    return dict(B=w["B"], H=w["H"], N=w["N"], Nk=w.get("Nk", w["N"]), d=w["d"], variants=variants, do_scale=1.0)
+    return dict(B=w["B"], H=w["H"], N=w["N"], Nk=w.get("Nk", w["N"]), d=w["d"], variants=variants, do_scale=1.0,
+                dropout_p=w.get("dropout_p", 0.0))
 
 
 # ---------------------------------------------------------------- multi-rank helpers
@@ -509,7 +510,8 @@ def run_table(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse", "b8h16n2000d64_ragged",
-             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal", "b4h16n4096d96"]
+             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal", "b4h16n4096d96", "b8h16n2048d64_dropout",
+             "b2h16n8192d128_causal_dropout"]
     names += [f"sweep_N{N}_d{d}{c}" for d in SWEEP_D for N in SWEEP_N for c in ("", "_causal")]
     if args.only:
         names = [n for n in names if any(o in n for o in args.only.split(","))]
@@ -533,8 +535,13 @@ def run_table(args):
             kept = 1.0 if mask is None else float(mask.float().mean())
             F = fwd_flops(B, H, N, d, causal, kept, Nk)
 
+            pdrop = wl.get("dropout_p", 0.0)
+
             def fwd():
-                if mask is None:
+                if pdrop:
+                    fa.forward_dropout(t["q"], t["k"], t["v"], pdrop, 1234, 0, causal=causal, scale=sc, out=o,
+                                       lse=lse)
+                elif mask is None:
                     fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc, out=o, lse=lse)
                 else:
                     fa.forward_blocksparse(t["q"], t["k"], t["v"], mask, scale=sc, out=o, lse=lse)
@@ -566,13 +573,18 @@ def run_table(args):
             row = {"workload": name, "variant": label, "B": B, "H": H, "N": N, "d": d, "kept": round(kept, 4),
                    "fwd_ms": round(t_f, 4), "fwd_tflops": round(F / t_f / 1e9, 1),
                    "fwd_pct_peak": round(100 * F / t_f / 1e9 / pk["bf16_tflops"], 1)}
-            if Nk != N:
-                # The staged calls are for Nq = Nk; time the whole backward through the API.
+            if Nk != N or pdrop:
+                # The staged calls are for Nq = Nk without dropout; time the whole backward.
                 def bwd_all():
-                    fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=causal, scale=sc, workspace=ws,
-                                grads=(dq, dk, dv))
+                    if pdrop:
+                        fa.backward_dropout(t["q"], t["k"], t["v"], o, lse, t["do"], pdrop, 1234, 0, causal=causal,
+                                            scale=sc, workspace=ws, grads=(dq, dk, dv))
+                    else:
+                        fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=causal, scale=sc,
+                                    workspace=ws, grads=(dq, dk, dv))
                 t_b = timed([bwd_all])
-                row.update({"Nk": Nk, "bwd_ms": round(t_b, 4), "bwd_tflops": round(2.5 * F / t_b / 1e9, 1),
+                row.update({"Nk": Nk, "dropout_p": pdrop, "bwd_ms": round(t_b, 4),
+                            "bwd_tflops": round(2.5 * F / t_b / 1e9, 1),
                             "bwd_pct_peak": round(100 * 2.5 * F / t_b / 1e9 / pk["bf16_tflops"], 1),
                             "fwd_bwd_tflops": round(3.5 * F / (t_f + t_b) / 1e9, 1)})
             elif name != "pr1":
@@ -612,6 +624,8 @@ def main():
     if args.table:
         return run_table(args)
     wl = workload(args.workload)
+    if wl["dropout_p"]:
+        raise SystemExit("dropout workloads are measured by --table only")
     if args.impl == "reference":
         return run_reference(args, args.workload, wl)
     return run_ours(args, args.workload, wl)

@@ -27,7 +27,7 @@ import re
 __all__ = [
     "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
     "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_dkdv",
-    "bwd_dq", "attention", "attention_blocksparse",
+    "bwd_dq", "attention", "attention_blocksparse", "forward_dropout", "backward_dropout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -51,6 +51,7 @@ def lib_path() -> str:
 
 _lib = None
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_u64, _u32 = ctypes.c_uint64, ctypes.c_uint32
 _SIGS = {
     "fa_status_string": ([_i], ctypes.c_char_p),
     "fa_version": ([], _i),
@@ -67,6 +68,8 @@ _SIGS = {
     "fa_bwd_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
     "fa_bwd_dkdv": ([_vp] * 7 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_dq": ([_vp] * 6 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
+    "fa_fwd_dropout": ([_vp] * 5 + [_i] * 5 + [_f, _f, _u64, _u32, _vp], _i),
+    "fa_bwd_dropout": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _f, _u64, _u32, _vp], _i),
     "fa_debug_exp2": ([_vp, _vp, _i, _i, _vp], _i),
     "fa_debug_wait_timeout": ([_i, _vp, _vp], _i),
     "fa_debug_stall_producer": ([_i, _i], _i),
@@ -192,6 +195,33 @@ def forward_blocksparse(q, k, v, tile_mask, scale=None, mask_block: int = 128, o
     return o, l
 
 
+def _seed_args(p, seed, offset):
+    p = float(p)
+    if not (0.0 <= p < 1.0):
+        raise ValueError("dropout probability must be in [0, 1)")
+    return p, int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF
+
+
+def forward_dropout(q, k, v, p: float, seed: int, offset: int = 0, causal: bool = False, scale=None, out=None,
+                    lse=None):
+    """Forward with dropout on the attention probabilities (keep mask from Philox,
+    seeded by (seed, offset)): O = (P * M * 256/t) V with t = round(256 (1 - p)); lse is
+    that of the softmax before dropout. q, k, v [B, H, N, d], d 64 or 128."""
+    import torch
+    _check_qkv(q, k, v)
+    if k.shape != q.shape:
+        raise ValueError("dropout needs equal query and key lengths")
+    p, seed, offset = _seed_args(p, seed, offset)
+    B, H, N, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    with torch.cuda.device(q.device):
+        st = lib().fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
+                                  int(bool(causal)), _scale(scale, d), p, seed, offset, _stream_ptr(q.device))
+    _check(st, "fa_fwd_dropout")
+    return o, l
+
+
 def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
 
@@ -232,6 +262,24 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=No
                                  workspace.numel(), B, H, N, Nk, d, int(bool(causal)), _scale(scale, d),
                                  _stream_ptr(q.device))
     _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def backward_dropout(q, k, v, o, lse, do, p: float, seed: int, offset: int = 0, causal: bool = False, scale=None,
+                     workspace=None, grads=None):
+    """Gradients of sum(O * dO) for ``forward_dropout`` with the same p, seed and offset."""
+    import torch
+    if k.shape != q.shape:
+        raise ValueError("dropout needs equal query and key lengths")
+    p, seed, offset = _seed_args(p, seed, offset)
+    workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
+    B, H, N, d = q.shape
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel(), B, H, N, d, int(bool(causal)), _scale(scale, d), p, seed,
+                                  offset, _stream_ptr(q.device))
+    _check(st, "fa_bwd_dropout")
     return dq, dk, dv
 
 
@@ -337,13 +385,15 @@ def _autograd_fn():
 
     class _Attention(torch.autograd.Function):
         @staticmethod
-        def forward(ctx, q, k, v, causal, scale, tile_mask, layout):
-            if tile_mask is None:
+        def forward(ctx, q, k, v, causal, scale, tile_mask, layout, drop):
+            if drop is not None:
+                o, lse = forward_dropout(q, k, v, *drop, causal=causal, scale=scale)
+            elif tile_mask is None:
                 o, lse = forward(q, k, v, causal=causal, scale=scale, layout=layout)
             else:
                 o, lse = forward_blocksparse(q, k, v, tile_mask, scale=scale)
             ctx.save_for_backward(q, k, v, o, lse)
-            ctx.causal, ctx.scale, ctx.tile_mask, ctx.layout = causal, scale, tile_mask, layout
+            ctx.causal, ctx.scale, ctx.tile_mask, ctx.layout, ctx.drop = causal, scale, tile_mask, layout, drop
             ctx.mark_non_differentiable(lse)
             return o, lse
 
@@ -351,11 +401,13 @@ def _autograd_fn():
         def backward(ctx, do, _dlse):
             q, k, v, o, lse = ctx.saved_tensors
             do = do.contiguous()
-            if ctx.tile_mask is None:
+            if ctx.drop is not None:
+                dq, dk, dv = backward_dropout(q, k, v, o, lse, do, *ctx.drop, causal=ctx.causal, scale=ctx.scale)
+            elif ctx.tile_mask is None:
                 dq, dk, dv = backward(q, k, v, o, lse, do, causal=ctx.causal, scale=ctx.scale, layout=ctx.layout)
             else:
                 dq, dk, dv = backward_blocksparse(q, k, v, o, lse, do, ctx.tile_mask, scale=ctx.scale)
-            return dq, dk, dv, None, None, None, None
+            return dq, dk, dv, None, None, None, None, None
 
     return _Attention
 
@@ -363,13 +415,25 @@ def _autograd_fn():
 _ATTN = None
 
 
-def attention(q, k, v, causal: bool = False, scale=None, layout: str = "bhnd"):
+def attention(q, k, v, causal: bool = False, scale=None, layout: str = "bhnd", dropout_p: float = 0.0,
+              seed=None, offset: int = 0):
     """Differentiable O = softmax(scale q k^T [causal]) v for torch.autograd: the
-    forward and backward run in the library (q, k, v and layout as for ``forward``)."""
+    forward and backward run in the library (q, k, v and layout as for ``forward``).
+    dropout_p > 0 applies dropout to the probabilities (see ``forward_dropout``); the
+    seed is drawn from torch's default CPU generator when not given, and the backward
+    reuses it."""
     global _ATTN
     if _ATTN is None:
         _ATTN = _autograd_fn()
-    o, _ = _ATTN.apply(q, k, v, bool(causal), scale, None, layout)
+    drop = None
+    if dropout_p:
+        if layout != "bhnd":
+            raise ValueError("dropout is implemented for the [B, H, N, d] layout")
+        if seed is None:
+            import torch
+            seed = int(torch.randint(0, 2 ** 62, (1,), dtype=torch.int64).item())
+        drop = (float(dropout_p), int(seed), int(offset))
+    o, _ = _ATTN.apply(q, k, v, bool(causal), scale, None, layout, drop)
     return o
 
 
@@ -378,5 +442,5 @@ def attention_blocksparse(q, k, v, tile_mask, scale=None):
     global _ATTN
     if _ATTN is None:
         _ATTN = _autograd_fn()
-    o, _ = _ATTN.apply(q, k, v, False, scale, tile_mask, "bhnd")
+    o, _ = _ATTN.apply(q, k, v, False, scale, tile_mask, "bhnd", None)
     return o

@@ -57,6 +57,20 @@ fa_status check_ptrs(std::initializer_list<const void*> ptrs) {
 
 fa_status check_scale(float scale) { return std::isfinite(scale) ? FA_OK : FA_ERR_INVALID_ARG; }
 
+// Dropout settings: keep threshold t = round(256 (1 - p)) in 1..256 (computed in double
+// from the float argument), kept probabilities scaled by 256 / t.
+fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, fa::DropParams* dp) {
+  if (!std::isfinite(p_drop) || p_drop < 0.f || p_drop >= 1.f) return FA_ERR_INVALID_ARG;
+  const double t = std::nearbyint(256.0 * (1.0 - static_cast<double>(p_drop)));
+  if (t < 1.0) return FA_ERR_INVALID_ARG;
+  dp->seed_lo = static_cast<uint32_t>(seed);
+  dp->seed_hi = static_cast<uint32_t>(seed >> 32);
+  dp->offset = offset;
+  dp->tm1 = static_cast<uint32_t>(t) - 1u;
+  dp->rs = static_cast<float>(256.0 / t);
+  return FA_OK;
+}
+
 // ------------------------------------------------------------------ per-device state
 
 struct DeviceState {
@@ -139,13 +153,13 @@ fa_status set_smem(K kernel, int bytes, std::once_flag (&flags)[kMaxDevices], cu
 }
 
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, int DS = D>
-fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
-                     cudaStream_t stream) {
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, int DS = D, bool DROP = false>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const fa::FwdParamsT<DROP>& p, cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK, DS>;
+  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK, DS, DROP>;
   constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
   // The kernel re-divides its register pool between warpgroups: refuse to launch a
@@ -166,8 +180,10 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// drop: dropout settings, or nullptr (dropout needs d 64 or 128, N_q = N_k and no tile mask).
 fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
-                     int B, int H, int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
+                     int B, int H, int N, int Nk, int d, int layout, int causal, float scale, void* stream,
+                     const fa::DropParams* drop = nullptr) {
   fa_status s;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
   const bool bnhd = layout == FA_LAYOUT_BNHD;
@@ -175,6 +191,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
+  if (drop != nullptr && (mask != nullptr || Nk != N || d == 96)) return FA_ERR_UNSUPPORTED;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
   int* status;
@@ -203,6 +220,16 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (drop) {
+    fa::FwdParamsDrop pd;
+    static_cast<fa::FwdParams&>(pd) = p;
+    pd.drop = *drop;
+    if (causal)
+      return d == 64 ? launch_fwd<64, true, false, false, 64, true>(mq, mk, mv, pd, st)
+                     : launch_fwd<128, true, false, false, 128, true>(mq, mk, mv, pd, st);
+    return d == 64 ? launch_fwd<64, false, false, false, 64, true>(mq, mk, mv, pd, st)
+                   : launch_fwd<128, false, false, false, 128, true>(mq, mk, mv, pd, st);
+  }
   if (d == 96) {  // the 128-wide kernels with 96 stored columns
     if (mask) return launch_fwd<128, false, true, false, 96>(mq, mk, mv, p, st);
     if (causal && Nk != N) return launch_fwd<128, true, false, true, 96>(mq, mk, mv, p, st);
@@ -236,9 +263,9 @@ size_t bwd_ws_bytes(int B, int H, int N, int d) {
 // Launch one of the two 384-thread backward kernels. They re-divide their register
 // pool between warpgroups; refuse to launch if the build gave them fewer registers
 // per thread than that split needs.
-template <typename K>
+template <typename K, typename P>
 fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid /* work items */, const CUtensorMap& mq, const CUtensorMap& mk,
-                            const CUtensorMap& mv, const CUtensorMap& mdo, const fa::BwdParams& p,
+                            const CUtensorMap& mv, const CUtensorMap& mdo, const P& p,
                             cudaStream_t stream, std::once_flag (&flags)[kMaxDevices],
                             cudaError_t (&errs)[kMaxDevices], int (&regs)[kMaxDevices]) {
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
@@ -258,23 +285,23 @@ fa_status launch_bwd_kernel(K kernel, int smem, unsigned grid /* work items */, 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, bool DROP = false>
 fa_status launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                      const fa::BwdParams& p, cudaStream_t stream) {
+                      const fa::BwdParamsT<DROP>& p, cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  return launch_bwd_kernel(fa::fa_bwd_dkdv_kernel<D, CAUSAL, SPARSE, XQK>, fa::BwdCfg<D>::kSmemBytes,
+  return launch_bwd_kernel(fa::fa_bwd_dkdv_kernel<D, CAUSAL, SPARSE, XQK, DROP>, fa::BwdCfg<D>::kSmemBytes,
                            unsigned(p.n_ktiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
 }
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, bool DROP = false>
 fa_status launch_dq(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                    const fa::BwdParams& p, cudaStream_t stream) {
+                    const fa::BwdParamsT<DROP>& p, cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  return launch_bwd_kernel(fa::fa_bwd_dq_kernel<D, CAUSAL, SPARSE, XQK>, fa::BwdCfg<D>::kQSmemBytes,
+  return launch_bwd_kernel(fa::fa_bwd_dq_kernel<D, CAUSAL, SPARSE, XQK, DROP>, fa::BwdCfg<D>::kQSmemBytes,
                            unsigned(p.n_tiles) * unsigned(p.BH), mq, mk, mv, mdo, p, stream, flags, errs, regs);
 }
 
@@ -328,7 +355,8 @@ enum class BwdStage { kDkdv, kDq };
 // N: query rows (the workspace's rows), Nk: key rows.
 fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v, const void* dO, void* out0,
                     void* out1, const void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H,
-                    int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
+                    int N, int Nk, int d, int layout, int causal, float scale, void* stream,
+                    const fa::DropParams* drop = nullptr) {
   fa_status s;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
   const bool bnhd = layout == FA_LAYOUT_BNHD;
@@ -338,6 +366,7 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   BwdArgs a;
   if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
+  if (drop != nullptr && (mask != nullptr || Nk != N || d == 96)) return FA_ERR_UNSUPPORTED;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
   int* status;
@@ -369,7 +398,17 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.off = Nk - N;
   p.ds = d;
   p.scale = scale;
+  fa::BwdParamsDrop pd;  // the dropout kernels' parameter block
+  if (drop) {
+    static_cast<fa::BwdParams&>(pd) = p;
+    pd.drop = *drop;
+  }
 #define FA_BWD_DISPATCH(LAUNCH)                                                                  \
+  if (drop)                                                                                      \
+    return causal ? (d == 64 ? LAUNCH<64, true, false, false, true>(mq, mk, mv, mdo, pd, st)     \
+                             : LAUNCH<128, true, false, false, true>(mq, mk, mv, mdo, pd, st))   \
+                  : (d == 64 ? LAUNCH<64, false, false, false, true>(mq, mk, mv, mdo, pd, st)    \
+                             : LAUNCH<128, false, false, false, true>(mq, mk, mv, mdo, pd, st)); \
   if (mask)                                                                                      \
     return d == 64 ? LAUNCH<64, false, true>(mq, mk, mv, mdo, p, st)                             \
                    : LAUNCH<128, false, true>(mq, mk, mv, mdo, p, st);                           \
@@ -390,7 +429,8 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
 
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int B, int H,
-                     int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
+                     int N, int Nk, int d, int layout, int causal, float scale, void* stream,
+                     const fa::DropParams* drop = nullptr) {
   fa_status s;
   // Validate everything before the first launch so that an error writes nothing.
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
@@ -400,12 +440,13 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
+  if (drop != nullptr && (mask != nullptr || Nk != N || d == 96)) return FA_ERR_UNSUPPORTED;
   if ((s = bwd_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, layout, stream)) != FA_OK) return s;
   if ((s = bwd_stage(BwdStage::kDkdv, q, k, v, dO, dk, dv, ws, ws_bytes, mask, 128, B, H, N, Nk, d, layout, causal,
-                     scale, stream)) != FA_OK)
+                     scale, stream, drop)) != FA_OK)
     return s;
   return bwd_stage(BwdStage::kDq, q, k, v, dO, dq, nullptr, ws, ws_bytes, mask, 128, B, H, N, Nk, d, layout, causal,
-                   scale, stream);
+                   scale, stream, drop);
 }
 
 __global__ void fa_debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int mode) {
@@ -522,6 +563,14 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
   return fwd_common(q, k, v, o, lse, tile_mask, B, H, N, N, d, FA_LAYOUT_BHND, 0, scale, stream);
 }
 
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                         int d, int causal, float scale, float p_drop, uint64_t seed, uint32_t offset, void* stream) {
+  fa::DropParams dp;
+  const fa_status s = make_drop(p_drop, seed, offset, &dp);
+  if (s != FA_OK) return s;
+  return fwd_common(q, k, v, o, lse, nullptr, B, H, N, N, d, FA_LAYOUT_BHND, causal != 0, scale, stream, &dp);
+}
+
 fa_status fa_device_status(void* stream, int* detail) {
   int* status;
   if (detail) *detail = 0;
@@ -546,6 +595,17 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int causal, float scale, void* stream) {
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, N, d,
                     FA_LAYOUT_BHND, causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                         int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, uint32_t offset,
+                         void* stream) {
+  fa::DropParams dp;
+  const fa_status s = make_drop(p_drop, seed, offset, &dp);
+  if (s != FA_OK) return s;
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, N, d,
+                    FA_LAYOUT_BHND, causal != 0, scale, stream, &dp);
 }
 
 fa_status fa_bwd_qk(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,

@@ -35,6 +35,9 @@
 // first finish reading (bounded mbarrier handshake).
 #pragma once
 
+#include <type_traits>
+
+#include "fa_dropout.cuh"
 #include "fa_ptx.cuh"
 
 namespace fa {
@@ -112,6 +115,13 @@ struct BwdParams {
   int v8;               // 1: the gradient outputs are 32-byte aligned (32-byte row stores)
   float scale;          // softmax scale
 };
+
+// The dropout kernels' parameters (the others keep the plain block unchanged).
+struct BwdParamsDrop : BwdParams {
+  DropParams drop;
+};
+template <bool DROP>
+using BwdParamsT = std::conditional_t<DROP, BwdParamsDrop, BwdParams>;
 
 // Register split of both 384-thread kernels: the producer/MMA warpgroup drops to 80,
 // the two compute warpgroups rise to 200 -> 128 * (80 + 2 * 200) = 61,440 registers,
@@ -306,11 +316,12 @@ struct DkdvBars {
   int abort;
 };
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK>
+// DROP: dropout on P (dV takes the dropped P^T, dS the kept part of dP^T).
+template <int D, bool CAUSAL, bool SPARSE, bool XQK, bool DROP = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const BwdParams p) {
+                   const BwdParamsT<DROP> p) {
   using Cfg = BwdCfg<D>;
   // Causal offset N_k - N_q: a compile-time 0 in the N_q = N_k kernels (XQK false).
   const int off_ = XQK ? p.off : 0;
@@ -502,6 +513,11 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int local = 0;
       for (int i = sch.first(); i >= 0; i = sch.next(i), ++it, ++local) {
         const int st = it & 1;
+        // Keep bits of this key over query columns [64h, 64h + 64) of tile i.
+        uint32_t kb[2] = {0u, 0u};
+        if constexpr (DROP)
+          drop_bits_cols<16>(kb, uint32_t(j * 32 + quarter * 8 + (lane >> 2)), uint32_t(i * 32 + h * 16),
+                             uint32_t(item.bh), p.drop);
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->t_full[st], (it >> 1) & 1, wc, kSiteBwdTFull)) ||
             !__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
           ok = false;
@@ -547,7 +563,19 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             pk[t] = pack_bf16(v.x, v.y);
           }
         }
-        tmem_st32(trow + Cfg::kTmS + h * 32, pk);
+        if constexpr (DROP) {
+          // dV = P~^T dO takes the dropped probabilities; dS below the undropped ones.
+          uint32_t pd[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float2 pp = unpack_bf16(pk[t]);
+            const float2 w = drop_pair(pp.x, pp.y, kb[t >> 4] >> ((2 * t) & 31), p.drop.rs);
+            pd[t] = pack_bf16(w.x, w.y);
+          }
+          tmem_st32(trow + Cfg::kTmS + h * 32, pd);
+        } else {
+          tmem_st32(trow + Cfg::kTmS + h * 32, pk);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
@@ -571,8 +599,14 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int t = 0; t < 32; ++t) {
             const float2 pp = unpack_bf16(pk[t]);
             const float2 dd = *reinterpret_cast<const float2*>(Dr + 2 * t);
-            const uint64_t diff =
-                f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), f2(dd.x, dd.y));
+            uint64_t diff;
+            if constexpr (DROP) {
+              const float2 dpv = drop_pair(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1]),
+                                           kb[t >> 4] >> ((2 * t) & 31), p.drop.rs);
+              diff = f2_sub(f2(dpv.x, dpv.y), f2(dd.x, dd.y));
+            } else {
+              diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), f2(dd.x, dd.y));
+            }
             const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
             ds[t] = pack_bf16(v.x, v.y);
           }
@@ -634,11 +668,12 @@ struct DqBars {
   int abort;
 };
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK>
+// DROP: dropout on P (dS takes the kept part of dP).
+template <int D, bool CAUSAL, bool SPARSE, bool XQK, bool DROP = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const BwdParams p) {
+                 const BwdParamsT<DROP> p) {
   using Cfg = BwdCfg<D>;
   // Causal offset N_k - N_q: a compile-time 0 in the N_q = N_k kernels (XQK false).
   const int off_ = XQK ? p.off : 0;
@@ -832,6 +867,11 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float Dv = dv_next;
       int local = 0;
       for (int jj = sch.first(); jj >= 0; jj = sch.next(jj), ++it, ++local) {
+        // Keep bits of this query row over key columns [64h, 64h + 64) of tile jj.
+        uint32_t kb[2] = {0u, 0u};
+        if constexpr (DROP)
+          drop_bits_rows<16>(kb, uint32_t(i * 32 + quarter * 8 + (lane >> 2)), uint32_t(jj * 32 + h * 16),
+                             uint32_t(item.bh), p.drop);
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, it & 1, wc, kSiteBwdSFull))) {
           ok = false;
           break;
@@ -885,7 +925,14 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             const float2 pp = unpack_bf16(pk[t]);
-            const uint64_t diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), dv2);
+            uint64_t diff;
+            if constexpr (DROP) {
+              const float2 dpv = drop_pair(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1]),
+                                           kb[t >> 4] >> ((2 * t) & 31), p.drop.rs);
+              diff = f2_sub(f2(dpv.x, dpv.y), dv2);
+            } else {
+              diff = f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), dv2);
+            }
             const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
             ds[t] = pack_bf16(v.x, v.y);
           }

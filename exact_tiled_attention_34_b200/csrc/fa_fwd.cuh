@@ -30,6 +30,9 @@
 // max, so skipping is exact (a deferred normalisation).
 #pragma once
 
+#include <type_traits>
+
+#include "fa_dropout.cuh"
 #include "fa_ptx.cuh"
 
 namespace fa {
@@ -54,6 +57,13 @@ struct FwdParams {
   int n_items;               // n_qblocks * BH work items (query block, batch*head)
   float c_log2;              // scale * log2(e)
 };
+
+// The dropout kernels' parameters (the others keep the plain block unchanged).
+struct FwdParamsDrop : FwdParams {
+  DropParams drop;
+};
+template <bool DROP>
+using FwdParamsT = std::conditional_t<DROP, FwdParamsDrop, FwdParams>;
 
 template <int D>
 struct FwdCfg {
@@ -182,9 +192,11 @@ enum FwdSite : int {
 // MASK: only columns t < lim are visible, for the tile on the causal diagonal
 // (lim = r + 1) or the last K/V tile of a sequence whose length is not a multiple of
 // 128 (lim = number of keys in it).
-template <bool MASK, int POLY8>
+// DROP: the probabilities written for P V are dropped where bit t of kb is clear and
+// scaled by rs where it is set; the returned sum is that of the undropped row.
+template <bool MASK, int POLY8, bool DROP = false>
 __device__ __forceinline__ void softmax_row(float (&s)[128], int lim, float c, float m, uint32_t tp, float& sum,
-                                            float& alpha, float& m_use) {
+                                            float& alpha, float& m_use, const uint32_t (&kb)[4], float rs) {
   // Four independent accumulators keep the reduction chains short.
   float mx;
   if (c >= 0.f) {
@@ -223,7 +235,12 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int lim, float c, f
       }
       acc[t & 3] = f2_add(acc[t & 3], pv);
       const float2 v = f2_split(pv);
-      pk[t] = pack_bf16(v.x, v.y);
+      if constexpr (DROP) {
+        const float2 w = drop_pair(v.x, v.y, kb[c0 >> 5] >> (c0 & 31), rs);
+        pk[t] = pack_bf16(w.x, w.y);
+      } else {
+        pk[t] = pack_bf16(v.x, v.y);
+      }
     }
     tmem_st32(tp + h * 32, pk);
   }
@@ -241,10 +258,11 @@ constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 
 // DS: the head dim as stored (row length of q, k, v, o): D, or 96 on the D = 128 kernels
 // (the loads read zeros for columns 96..127; only DS columns of O are written).
-template <int D, bool CAUSAL, bool SPARSE, bool XQK, int DS>
+// DROP: dropout on the probabilities that multiply V (keep masks regenerated per tile).
+template <int D, bool CAUSAL, bool SPARSE, bool XQK, int DS, bool DROP = false>
 __global__ void __launch_bounds__(384, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+              const __grid_constant__ CUtensorMap tm_v, const FwdParamsT<DROP> p) {
   using Cfg = FwdCfg<D>;
   constexpr int S = Cfg::kStages;
   // Causal offset N_k - N_q: a compile-time 0 in the N_q = N_k kernels (XQK false).
@@ -484,6 +502,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int r = quarter * 32 + lane;
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
     const float c = p.c_log2;
+    float drop_rs = 1.f;  // scale of the kept probabilities
+    if constexpr (DROP) drop_rs = p.drop.rs;
     int cnt = 0;  // S_i tiles consumed so far (continues across items)
     bool ok = true;
     FwdItem item;
@@ -497,6 +517,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint32_t b;
         for (int j = sch.first(b); j >= 0; j = sch.next(j, b)) {
           if (!(b & (1u << i))) continue;
+          // Keep bits of this row over key tile j, drawn while S is being computed.
+          uint32_t kb[4] = {0u, 0u, 0u, 0u};
+          if constexpr (DROP)
+            drop_bits_rows<32>(kb, uint32_t(tile * 32 + quarter * 8 + (lane >> 2)), uint32_t(j * 32),
+                               uint32_t(item.bh), p.drop);
           if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], cnt & 1, wc, kSiteFwdSFull))) {
             ok = false;
             break;
@@ -529,9 +554,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (diag || tail) {
             int lim = diag ? r + 1 + dbase : nk_last;
             if (XQK && lim < 0) lim = 0;  // (only an offset makes a row see none of a scheduled tile)
-            softmax_row<true, PolyShare<D>::kFwd>(s, lim, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+            softmax_row<true, PolyShare<D>::kFwd, DROP>(s, lim, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use, kb,
+                                                        drop_rs);
           } else {
-            softmax_row<false, PolyShare<D>::kFwd>(s, 128, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use);
+            softmax_row<false, PolyShare<D>::kFwd, DROP>(s, 128, c, m, trow + Cfg::tm_p(i), sum, alpha, m_use, kb,
+                                                         drop_rs);
           }
           const bool rescale = m_use != m;
           l = l * alpha + sum;

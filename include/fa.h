@@ -126,6 +126,27 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                              int B, int H, int N, int d, float scale, void* stream);
 
 /*
+ * Forward with dropout on the attention probabilities (dropout is named among the
+ * element-wise O(N^2) operations of standard attention on the PagedAttention page,
+ * section on bandwidth constraints; what follows is this library's definition).
+ *   P = softmax(scale q k^T [causal]) as in fa_fwd; O = (P * M * 256 / t) V, where
+ *   M is a 0/1 keep mask and t = round(256 (1 - p_drop)) in 1..256 (computed in
+ *   double from p_drop): the drop probability is p_drop rounded to a multiple of
+ *   1/256 and the kept entries are scaled so that E[O] is exact. lse is that of the
+ *   softmax before dropout.
+ *   M: element (b, h, i, j) is kept iff byte (j % 4) (least significant first) of
+ *   word (i % 4) of Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy
+ *   as 1, 2, 3", SC 2011) with counter (j / 4, i / 4, b H + h, offset) and key
+ *   (seed mod 2^32, seed / 2^32) is below t. The same (seed, offset) passed to
+ *   fa_bwd_dropout gives the gradients of the same function.
+ *   p_drop : 0 <= p_drop < 1 with t >= 1, else FA_ERR_INVALID_ARG.
+ *   d      : 64 or 128 (96: FA_ERR_UNSUPPORTED). Other arguments as for fa_fwd.
+ */
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                         int d, int causal, float scale, float p_drop, uint64_t seed, uint32_t offset,
+                         void* stream);
+
+/*
  * Bytes of device scratch that fa_bwd / fa_bwd_blocksparse need for these sizes:
  * two fp32 [B,H,Npad] row arrays (D_i = sum_c dO_ic O_ic, and lse_i * log2 e;
  * Npad = 128 * ceil(N / 128), so each tile's rows are one run), each rounded up to
@@ -230,6 +251,17 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const void* dO, void* dq, void* dk, void* dv,
                          const uint8_t* tile_mask, int mask_block,
                          int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Backward of fa_fwd_dropout (same p_drop, seed and offset, and its o and lse):
+ * dV = P~^T dO, dP = (dO V^T) * M * 256 / t, dS = P * (dP - D), dQ = scale dS K,
+ * dK = scale dS^T Q with P~ = P * M * 256 / t and D = rowsum(dO * O). Arguments,
+ * workspace and rules as for fa_bwd, plus those of fa_fwd_dropout.
+ */
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                         int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, uint32_t offset,
+                         void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the library's device status

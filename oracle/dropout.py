@@ -37,7 +37,8 @@ its backward see the same mask without storing it:
 Parity status: pinned by tests/test_oracle_dropout.py (the generator against its
 published known-answer vectors; the mask layout against a scalar re-derivation; p = 0
 against plain attention; keep statistics; finite differences of the loss with the
-mask held fixed; the expectation over seeds).
+mask held fixed; the expectation over seeds; single-head slices against the full
+problem).
 """
 from __future__ import annotations
 
@@ -95,13 +96,15 @@ def keep_threshold(p: float) -> int:
 
 
 def dropout_keep_mask(B: int, H: int, n_q: int, n_k: int, p: float, seed: int, offset: int = 0,
-                      rows=None) -> np.ndarray:
+                      rows=None, bh0: int = 0) -> np.ndarray:
     """Boolean keep mask [B, H, R, n_k] (R = n_q, or len(rows) for the given absolute
-    query rows), following the block layout in the module docstring."""
+    query rows), following the block layout in the module docstring. bh0 is added to
+    the head counter b * H + h: a single-head slice of a larger problem passes the
+    head's own index b * H + h there."""
     t = keep_threshold(p)
     qi = np.arange(n_q, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     kj = np.arange(n_k, dtype=np.int64)
-    bh = np.arange(B * H, dtype=np.int64).reshape(B, H, 1, 1)
+    bh = int(bh0) + np.arange(B * H, dtype=np.int64).reshape(B, H, 1, 1)
     shape = (B, H, qi.shape[0], n_k)
     c0 = np.broadcast_to((kj // 4)[None, None, None, :], shape)
     c1 = np.broadcast_to((qi // 4)[None, None, :, None], shape)
@@ -117,16 +120,17 @@ def dropout_keep_mask(B: int, H: int, n_q: int, n_k: int, p: float, seed: int, o
 
 
 def attn_dropout_fwd_ref(q, k, v, p: float, seed: int, offset: int = 0, causal: bool = False,
-                         scale: float | None = None):
+                         scale: float | None = None, bh0: int = 0):
     """Forward with dropout for q [B, H, N_q, d], k, v [B, H, N_k, d]: (O, lse) in fp64.
-    lse is that of the softmax before dropout (what the backward needs)."""
+    lse is that of the softmax before dropout (what the backward needs). bh0: as for
+    ``dropout_keep_mask``."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     n_k = k.shape[2]
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     t = keep_threshold(p)
-    keep = dropout_keep_mask(B, H, N, n_k, p, seed, offset)
+    keep = dropout_keep_mask(B, H, N, n_k, p, seed, offset, bh0=bh0)
     o = np.zeros((B, H, N, v.shape[-1]))
     lse = np.zeros((B, H, N))
     for b in range(B):
@@ -140,16 +144,17 @@ def attn_dropout_fwd_ref(q, k, v, p: float, seed: int, offset: int = 0, causal: 
 
 
 def attn_dropout_bwd_ref(q, k, v, do, p: float, seed: int, offset: int = 0, causal: bool = False,
-                         scale: float | None = None):
+                         scale: float | None = None, bh0: int = 0):
     """Gradients of L = sum(O * dO) with dropout (the mask fixed by seed and offset).
-    Returns dq, dk, dv, the forward's o and lse, and D = sum_j P_ij dP_ij."""
+    Returns dq, dk, dv, the forward's o and lse, and D = sum_j P_ij dP_ij. bh0: as for
+    ``dropout_keep_mask``."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, N, d = q.shape
     n_k = k.shape[2]
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     t = keep_threshold(p)
-    keep = dropout_keep_mask(B, H, N, n_k, p, seed, offset)
+    keep = dropout_keep_mask(B, H, N, n_k, p, seed, offset, bh0=bh0)
     out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
            "o": np.zeros((B, H, N, v.shape[-1])), "lse": np.zeros((B, H, N)), "D": np.zeros((B, H, N))}
     for b in range(B):

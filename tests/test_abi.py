@@ -24,7 +24,7 @@ def test_exports_every_declared_symbol(L):
     assert {"fa_fwd", "fa_bwd", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_bwd_workspace_bytes",
             "fa_status_string", "fa_device_status", "fa_version", "fa_bwd_preprocess", "fa_bwd_dkdv",
             "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_wait_timeout",
-            "fa_debug_stall_producer"} <= set(names)
+            "fa_debug_stall_producer", "fa_fwd_dropout", "fa_bwd_dropout"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True,
                          check=True).stdout
     defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -107,6 +107,20 @@ def test_workspace_bytes(L):
         assert L.fa_bwd_workspace_bytes(B, H, N, d) == 2 * up(rows * 4)
     assert L.fa_bwd_workspace_bytes(0, 1, 128, 64) == 0
     assert L.fa_bwd_workspace_bytes(1, 1, -128, 64) == 0
+
+
+def test_dropout_argument_checks(L):
+    f = lambda p=0.1, d=64, N=128, q=A: L.fa_fwd_dropout(q, A, A, A, A, 1, 1, N, d, 0, 0.125, p, 5, 0, None)
+    b = lambda p=0.1, d=64: L.fa_bwd_dropout(A, A, A, A, A, A, A, A, A, A, 1 << 20, 1, 1, 128, d, 0, 0.125, p, 5,
+                                             0, None)
+    for bad in (-0.1, 1.0, 2.0, float("nan"), float("inf"), 0.999):  # 0.999: keep threshold rounds to 0
+        assert f(p=bad) == INVALID and b(p=bad) == INVALID
+    assert f(d=96) == UNSUPPORTED and b(d=96) == UNSUPPORTED
+    assert f(d=80) == UNSUPPORTED
+    assert f(q=None) == INVALID and f(q=A + 2) == ALIGN
+    assert f(N=0) == INVALID
+    assert f() == _fwd(L)  # valid arguments get as far as a plain forward does here
+    assert f(p=0.0) == _fwd(L) and f(p=0.998) == _fwd(L)  # t = 256 and t = 1 are valid
 
 
 def test_wait_timeout_argument_checks(L):

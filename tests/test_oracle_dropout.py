@@ -78,6 +78,11 @@ def pin_mask_layout(mod):
     # sampled rows give the same mask rows
     rows = np.array([8, 0, 5])
     assert np.array_equal(mod.dropout_keep_mask(B, H, N, Nk, p, seed, off, rows=rows), m[:, :, rows])
+    # a single-head slice with its head index gives that head's mask
+    for b in range(B):
+        for h in range(H):
+            one = mod.dropout_keep_mask(1, 1, N, Nk, p, seed, off, bh0=b * H + h)
+            assert np.array_equal(one[0, 0], m[b, h])
 
 
 def pin_p_zero_is_plain_attention(mod):
@@ -148,6 +153,20 @@ def pin_dropout_finite_differences(mod):
             assert err < 1e-6, (name, N, causal, err)
 
 
+def pin_head_slices_match_full(mod):
+    """Forward and backward of one (b, h) slice with its head index equal the full
+    problem's (b, h) results."""
+    q, k, v, do = (_rand((2, 3, 9, 4), s) for s in (61, 62, 63, 64))
+    full = mod.attn_dropout_bwd_ref(q, k, v, do, 0.4, 555, 2, True, 0.7)
+    for b, h in ((0, 0), (1, 2), (0, 2)):
+        sl = lambda x: x[b:b + 1, h:h + 1]
+        one = mod.attn_dropout_bwd_ref(sl(q), sl(k), sl(v), sl(do), 0.4, 555, 2, True, 0.7, bh0=b * 3 + h)
+        for name in ("dq", "dk", "dv", "o", "lse"):
+            assert np.max(np.abs(one[name][0, 0] - full[name][b, h])) < 1e-13, (name, b, h)
+        o, _ = mod.attn_dropout_fwd_ref(sl(q), sl(k), sl(v), 0.4, 555, 2, True, 0.7, bh0=b * 3 + h)
+        assert np.max(np.abs(o[0, 0] - full["o"][b, h])) < 1e-13
+
+
 def pin_expectation_over_seeds(mod):
     """Dropout is unbiased: the mean of O over seeds tends to plain attention's O
     (within 5 standard errors of the sample)."""
@@ -176,6 +195,7 @@ DROPOUT_PINS = [
     pin_dropout_finite_differences,
     pin_expectation_over_seeds,
     pin_threshold_rule,
+    pin_head_slices_match_full,
 ]
 
 
@@ -199,6 +219,7 @@ MUTATIONS = {
                          "    c1 = np.broadcast_to((qi // 4)[None, None, :, None], shape)",
                          "c1 = np.broadcast_to((kj // 4)[None, None, None, :], shape)\n"
                          "    c0 = np.broadcast_to((qi // 4)[None, None, :, None], shape)"),
+    "head_offset_ignored": ("bh = int(bh0) + np.arange(B * H", "bh = 0 * int(bh0) + np.arange(B * H"),
     "offset_ignored": ("c3 = np.full(shape, int(offset) & 0xFFFFFFFF, dtype=np.int64)",
                        "c3 = np.full(shape, 0, dtype=np.int64)"),
     "keep_le": ("return byte < np.uint64(t)", "return byte <= np.uint64(t)"),
