@@ -27,7 +27,8 @@ import re
 __all__ = [
     "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
     "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_dkdv",
-    "bwd_dq", "attention", "attention_blocksparse", "forward_dropout", "backward_dropout",
+    "bwd_dq", "attention", "attention_blocksparse", "forward_dropout", "backward_dropout", "merge_partial",
+    "accumulate_bf16", "to_bf16",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +71,9 @@ _SIGS = {
     "fa_bwd_dq": ([_vp] * 6 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
     "fa_fwd_dropout": ([_vp] * 5 + [_i] * 5 + [_f, _f, _u64, _u32, _vp], _i),
     "fa_bwd_dropout": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _f, _u64, _u32, _vp], _i),
+    "fa_merge_partial": ([_vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _vp], _i),
+    "fa_accumulate_bf16": ([_vp, _vp, ctypes.c_longlong, _i, _vp], _i),
+    "fa_to_bf16": ([_vp, _vp, ctypes.c_longlong, _vp], _i),
     "fa_debug_exp2": ([_vp, _vp, _i, _i, _vp], _i),
     "fa_debug_wait_timeout": ([_i, _vp, _vp], _i),
     "fa_debug_stall_producer": ([_i, _i], _i),
@@ -374,6 +378,52 @@ def debug_stall_producer(on: bool, timeout_us: int = 2000):
     """Test hook: while on, attention launches run with an idle TMA producer and a
     wait limit of timeout_us, so that they end through their timeout path."""
     _check(lib().fa_debug_stall_producer(1 if on else 0, int(timeout_us)), "fa_debug_stall_producer")
+
+
+# ---------------------------------------------------------------- key-block merging
+# Element-wise kernels for attention split over key blocks (see ``ring``).
+
+def merge_partial(o_acc, lse_acc, o_part, lse_part):
+    """In place: (o_acc fp32, lse_acc fp32) <- the log-sum-exp merge with one key block's
+    partial result (o_part bf16, lse_part fp32), all [B, H, N, d] / [B, H, N]."""
+    import torch
+    if o_acc.dtype != torch.float32 or o_part.dtype != torch.bfloat16 or o_acc.shape != o_part.shape:
+        raise ValueError("o_acc must be fp32 and o_part bf16 of one shape")
+    if lse_acc.dtype != torch.float32 or lse_part.dtype != torch.float32 or lse_acc.shape != lse_part.shape:
+        raise ValueError("lse_acc and lse_part must be fp32 of one shape")
+    for t in (o_acc, lse_acc, o_part, lse_part):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("contiguous CUDA tensors expected")
+    d = o_acc.shape[-1]
+    with torch.cuda.device(o_acc.device):
+        st = lib().fa_merge_partial(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                                    lse_acc.numel(), d, _stream_ptr(o_acc.device))
+    _check(st, "fa_merge_partial")
+
+
+def accumulate_bf16(acc, x, overwrite: bool = False):
+    """In place: acc (fp32) <- (0 if overwrite else acc) + x (bf16), same shape."""
+    import torch
+    if acc.dtype != torch.float32 or x.dtype != torch.bfloat16 or acc.shape != x.shape:
+        raise ValueError("acc must be fp32 and x bf16 of one shape")
+    if not (acc.is_cuda and x.is_cuda and acc.is_contiguous() and x.is_contiguous()):
+        raise ValueError("contiguous CUDA tensors expected")
+    with torch.cuda.device(acc.device):
+        st = lib().fa_accumulate_bf16(acc.data_ptr(), x.data_ptr(), acc.numel(), int(bool(overwrite)),
+                                      _stream_ptr(acc.device))
+    _check(st, "fa_accumulate_bf16")
+
+
+def to_bf16(x, out=None):
+    """bf16 copy of an fp32 CUDA tensor (round to nearest even), through the library."""
+    import torch
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else out
+    with torch.cuda.device(x.device):
+        st = lib().fa_to_bf16(out.data_ptr(), x.data_ptr(), x.numel(), _stream_ptr(x.device))
+    _check(st, "fa_to_bf16")
+    return out
 
 
 # ---------------------------------------------------------------- autograd

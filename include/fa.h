@@ -264,6 +264,34 @@ fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void
                          void* stream);
 
 /*
+ * Attention over a key sequence split into blocks (the sequence-parallel ring, where
+ * each GPU holds one block of queries, keys and values and the key/value blocks
+ * travel around the GPUs). Softmax attention over the union of two key sets is the
+ * log-sum-exp-weighted mean of the two partial results, which is what the online
+ * softmax of the method does tile by tile; these calls do it block by block.
+ *
+ * fa_merge_partial: merges a partial result (o_part bf16 [rows, d], lse_part fp32
+ * [rows], as written by fa_fwd for one key block) into the running one (o_acc fp32
+ * [rows, d], lse_acc fp32 [rows], updated in place):
+ *   lse' = ln(e^lse_acc + e^lse_part),
+ *   o'   = o_acc e^(lse_acc - lse') + o_part e^(lse_part - lse').
+ * Start from o_acc = 0 and lse_acc = -INFINITY; a row with both -INFINITY stays
+ * o = 0, lse = -INFINITY. rows = B*H*N_q; d 64 or 128 (else FA_ERR_UNSUPPORTED);
+ * o_acc and o_part 16-byte aligned (FA_ERR_ALIGNMENT). Device pointers; async.
+ */
+fa_status fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows,
+                           int d, void* stream);
+
+/*
+ * acc[i] = (overwrite ? 0 : acc[i]) + x[i] for i < n: fp32 accumulation of a bf16
+ * partial gradient (device pointers, both 16-byte aligned; n a multiple of 8).
+ */
+fa_status fa_accumulate_bf16(float* acc, const void* x, long long n, int overwrite, void* stream);
+
+/* out[i] = bf16(in[i]), round to nearest even (n a multiple of 8; 16-byte aligned). */
+fa_status fa_to_bf16(void* out, const float* in, long long n, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the library's device status
  * word for the current device: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel since
  * the last call gave up on a wait. *detail (if non-NULL, host pointer) receives

@@ -4,8 +4,10 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
 ``bench.py`` may import this package. It is independent of the CUDA library.
 """
 from .attention import (  # noqa: F401
+    attn_bwd_block_ref,
     attn_bwd_ref,
     attn_dq_rows_ref,
+    attn_fwd_block_ref,
     attn_fwd_ref,
     attn_fwd_rows_ref,
     attn_probs_ref,

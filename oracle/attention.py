@@ -57,6 +57,8 @@ __all__ = [
     "attn_fwd_rows_ref",
     "attn_bwd_ref",
     "attn_dq_rows_ref",
+    "attn_fwd_block_ref",
+    "attn_bwd_block_ref",
 ]
 
 
@@ -215,3 +217,43 @@ def attn_dq_rows_ref(q_rows, rows, k, v, do_rows, causal: bool, scale: float,
     D = np.sum(p * dp, axis=1)
     ds = p * (dp - D[:, None])
     return scale * (ds @ k)
+
+
+# ---------------------------------------------------------------- key blocks
+# Attention over a key sequence split into blocks (one block per GPU of a ring). With
+# the causal mask the rule is the global one: key j is visible to query i iff j <= i,
+# for absolute positions i = q_off + row and j = k_off + column.
+
+def _block_scores(q, k, scale: float, causal: bool, q_off: int, k_off: int) -> np.ndarray:
+    s = float(scale) * (_f64(q) @ _f64(k).T)
+    if causal:
+        rows = q_off + np.arange(s.shape[0])[:, None]
+        cols = k_off + np.arange(s.shape[1])[None, :]
+        s = np.where(cols <= rows, s, -np.inf)
+    return s
+
+
+def attn_fwd_block_ref(q, k, v, scale: float, causal: bool = False, q_off: int = 0, k_off: int = 0):
+    """One head's partial result over one key block: (O_b, lse_b), the softmax taken over
+    the block's visible keys only (O_b = 0, lse_b = -inf for a row that sees none of
+    them). q [R, d] at positions q_off.., k and v [C, d] at positions k_off..."""
+    p, lse = _softmax_rows(_block_scores(q, k, scale, causal, q_off, k_off))
+    return p @ _f64(v), lse
+
+
+def attn_bwd_block_ref(q, k, v, do, lse, D, scale: float, causal: bool = False, q_off: int = 0, k_off: int = 0):
+    """One head's share of the gradients from one key block, given each query row's
+    log-sum-exp and D_i = sum_c dO_ic O_ic over the WHOLE key sequence: with
+    P = exp(S - lse) on the block, dV_b = P^T dO, dP = dO V_b^T, dS = P (dP - D),
+    dQ += scale dS K_b, dK_b = scale dS^T Q. Summed over the blocks these are the
+    full gradients (the sum over j of the definition splits along the key blocks).
+    Returns (dq_part, dk_b, dv_b)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    s = _block_scores(q, k, scale, causal, q_off, k_off)
+    lse = _f64(lse)[:, None]
+    with np.errstate(invalid="ignore"):
+        p = np.where(np.isfinite(s) & np.isfinite(lse), np.exp(s - np.where(np.isfinite(lse), lse, 0.0)), 0.0)
+    dp = do @ v.T
+    ds = p * (dp - _f64(D)[:, None])
+    return scale * (ds @ k), scale * (ds.T @ q), p.T @ do
+

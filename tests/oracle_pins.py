@@ -362,6 +362,73 @@ def pin_cross_rows_match_full(mod):
     assert np.allclose(dqr, g["dq"][0, 0][rows], atol=1e-12)
 
 
+# ---------------------------------------------------------------- key-block pins
+
+def _split(n, sizes):
+    out, o = [], 0
+    for c in sizes:
+        out.append((o, o + c))
+        o += c
+    assert o == n
+    return out
+
+
+def pin_blocks_merge_to_full(mod):
+    """Partial results over a partition of the keys, merged by the textbook log-sum-exp
+    rule (weights e^(lse_b - lse)), give the full attention (causal and not)."""
+    N, d, scale = 11, 4, 0.6
+    q, k, v = (_rand((N, d), s) for s in (81, 82, 83))
+    for causal in (False, True):
+        o_ref, lse_ref = mod.attn_fwd_ref(q[None, None], k[None, None], v[None, None], causal, scale)
+        for q0, q1 in _split(N, (5, 6)):
+            parts = [mod.attn_fwd_block_ref(q[q0:q1], k[k0:k1], v[k0:k1], scale, causal, q0, k0)
+                     for (k0, k1) in _split(N, (4, 4, 3))]
+            lse = np.logaddexp.reduce(np.stack([l for _, l in parts]), axis=0)
+            w = [np.where(np.isfinite(l), np.exp(l - lse), 0.0)[:, None] for _, l in parts]
+            o = sum(wi * oi for wi, (oi, _) in zip(w, parts))
+            assert np.max(np.abs(lse - lse_ref[0, 0, q0:q1])) < 1e-12
+            assert np.max(np.abs(o - o_ref[0, 0, q0:q1])) < 1e-12
+
+
+def pin_block_grads_sum_to_full(mod):
+    """Block gradients with the whole row's lse and D: the dQ shares sum to dQ, and each
+    block's dK, dV shares summed over the query blocks are that block's rows of dK, dV."""
+    N, d, scale = 10, 3, 0.8
+    q, k, v, do = (_rand((N, d), s) for s in (84, 85, 86, 87))
+    for causal in (False, True):
+        full = mod.attn_bwd_ref(q[None, None], k[None, None], v[None, None], do[None, None], causal, scale)
+        lse, D = full["lse"][0, 0], full["D"][0, 0]
+        dq = np.zeros_like(q)
+        dk = np.zeros_like(k)
+        dv = np.zeros_like(v)
+        for q0, q1 in _split(N, (3, 7)):
+            for k0, k1 in _split(N, (6, 4)):
+                a, b, c = mod.attn_bwd_block_ref(q[q0:q1], k[k0:k1], v[k0:k1], do[q0:q1], lse[q0:q1], D[q0:q1],
+                                                 scale, causal, q0, k0)
+                dq[q0:q1] += a
+                dk[k0:k1] += b
+                dv[k0:k1] += c
+        for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+            assert np.max(np.abs(g - full[name][0, 0])) < 1e-12, (name, causal)
+
+
+def pin_block_above_diagonal_is_empty(mod):
+    """With the causal mask a key block entirely after the query block contributes
+    nothing: lse -inf, O = 0, zero gradients."""
+    q, k, v, do = (_rand((4, 3), s) for s in (88, 89, 90, 91))
+    o, lse = mod.attn_fwd_block_ref(q, k, v, 0.5, True, 0, 4)
+    assert np.all(np.isneginf(lse)) and np.all(o == 0)
+    g = mod.attn_bwd_block_ref(q, k, v, do, np.zeros(4), np.zeros(4), 0.5, True, 0, 4)
+    assert all(np.all(x == 0) for x in g)
+
+
+BLOCK_PINS = [
+    pin_blocks_merge_to_full,
+    pin_block_grads_sum_to_full,
+    pin_block_above_diagonal_is_empty,
+]
+
+
 FORWARD_PINS = [
     pin_probs_rows_sum_to_one,
     pin_equal_keys_mean_of_v,
@@ -390,4 +457,4 @@ CROSS_PINS = [
     pin_cross_brute_force,
     pin_cross_rows_match_full,
 ]
-ALL_PINS = FORWARD_PINS + BACKWARD_PINS + CROSS_PINS
+ALL_PINS = FORWARD_PINS + BACKWARD_PINS + CROSS_PINS + BLOCK_PINS

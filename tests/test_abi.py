@@ -24,7 +24,8 @@ def test_exports_every_declared_symbol(L):
     assert {"fa_fwd", "fa_bwd", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_bwd_workspace_bytes",
             "fa_status_string", "fa_device_status", "fa_version", "fa_bwd_preprocess", "fa_bwd_dkdv",
             "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_wait_timeout",
-            "fa_debug_stall_producer", "fa_fwd_dropout", "fa_bwd_dropout"} <= set(names)
+            "fa_debug_stall_producer", "fa_fwd_dropout", "fa_bwd_dropout", "fa_merge_partial",
+            "fa_accumulate_bf16", "fa_to_bf16"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True,
                          check=True).stdout
     defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -121,6 +122,22 @@ def test_dropout_argument_checks(L):
     assert f(N=0) == INVALID
     assert f() == _fwd(L)  # valid arguments get as far as a plain forward does here
     assert f(p=0.0) == _fwd(L) and f(p=0.998) == _fwd(L)  # t = 256 and t = 1 are valid
+
+
+def test_merge_argument_checks(L):
+    m = lambda oa=A, la=A, op=A, lp=A, rows=128, d=64: L.fa_merge_partial(oa, la, op, lp, rows, d, None)
+    assert m(rows=0) == OK and m(oa=None, rows=0) == OK  # nothing to do
+    assert m(rows=-1) == INVALID
+    assert m(d=96) == UNSUPPORTED and m(d=32) == UNSUPPORTED
+    assert m(oa=None) == INVALID and m(lp=None) == INVALID
+    assert m(oa=A + 8) == ALIGN and m(op=A + 4) == ALIGN and m(la=A + 2) == ALIGN
+    assert m(rows=1 << 41) == UNSUPPORTED
+    acc = L.fa_accumulate_bf16
+    assert acc(A, A, 12, 0, None) == INVALID and acc(A, A, -8, 0, None) == INVALID
+    assert acc(None, A, 8, 0, None) == INVALID and acc(A + 8, A, 8, 0, None) == ALIGN
+    assert acc(A, A, 0, 0, None) == OK
+    cv = L.fa_to_bf16
+    assert cv(A, A, 7, None) == INVALID and cv(A, None, 8, None) == INVALID and cv(A + 2, A, 8, None) == ALIGN
 
 
 def test_wait_timeout_argument_checks(L):

@@ -51,6 +51,12 @@ MUTATIONS = {
     "dq_dropped_scale": ('out["dq"][b, h] = scale * (ds @ k[b, h])', 'out["dq"][b, h] = (ds @ k[b, h])'),
     "dk_wrong_operand": ('out["dk"][b, h] = scale * (ds.T @ q[b, h])', 'out["dk"][b, h] = scale * (ds.T @ k[b, h])'),
     "dp_wrong_operand": ("dp = do[b, h] @ v[b, h].T", "dp = do[b, h] @ k[b, h].T"),
+    "block_causal_strict": ("s = np.where(cols <= rows, s, -np.inf)", "s = np.where(cols < rows, s, -np.inf)"),
+    "block_offsets_swapped": ("rows = q_off + np.arange(s.shape[0])[:, None]",
+                              "rows = k_off + np.arange(s.shape[0])[:, None]"),
+    "block_ds_dropped_D": ("ds = p * (dp - _f64(D)[:, None])", "ds = p * dp"),
+    "block_dv_from_q": ("return scale * (ds @ k), scale * (ds.T @ q), p.T @ do",
+                        "return scale * (ds @ k), scale * (ds.T @ q), p.T @ q"),
 }
 
 
