@@ -168,17 +168,17 @@ def _autograd_fn():
 
     class _Ring(torch.autograd.Function):
         @staticmethod
-        def forward(ctx, q, k, v, causal, scale, ring):
-            o, lse = ring_forward(q, k, v, causal, scale, ring)
+        def forward(ctx, q, k, v, causal, scale, ring, ops):
+            o, lse = ring_forward(q, k, v, causal, scale, ring, ops)
             ctx.save_for_backward(q, k, v, o, lse)
-            ctx.causal, ctx.scale, ctx.ring = causal, scale, ring
+            ctx.causal, ctx.scale, ctx.ring, ctx.ops = causal, scale, ring, ops
             return o
 
         @staticmethod
         def backward(ctx, do):
             q, k, v, o, lse = ctx.saved_tensors
-            dq, dk, dv = ring_backward(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale, ctx.ring)
-            return dq, dk, dv, None, None, None
+            dq, dk, dv = ring_backward(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale, ctx.ring, ctx.ops)
+            return dq, dk, dv, None, None, None, None
 
     return _Ring
 
@@ -186,10 +186,11 @@ def _autograd_fn():
 _RING = None
 
 
-def ring_attention(q, k, v, causal=False, scale=None, ring=None):
+def ring_attention(q, k, v, causal=False, scale=None, ring=None, ops=None):
     """Differentiable sequence-parallel attention over the ranks of `ring` (default: the
-    default process group); q, k, v are this rank's [B, H, n, d] sequence blocks."""
+    default process group); q, k, v are this rank's [B, H, n, d] sequence blocks. `ops`
+    are the per-block steps (default: the library's kernels)."""
     global _RING
     if _RING is None:
         _RING = _autograd_fn()
-    return _RING.apply(q, k, v, bool(causal), scale, ProcessGroupRing() if ring is None else ring)
+    return _RING.apply(q, k, v, bool(causal), scale, ProcessGroupRing() if ring is None else ring, ops)

@@ -100,6 +100,13 @@ def _worker(rank, world, port, causal, out):
         for name, x in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
             ref = full[name][:, :, rank * n:(rank + 1) * n]
             errs[name] = float(np.max(np.abs(x.numpy() - ref)))
+        # the autograd wrapper: same blocks, gradients through torch.autograd
+        qa, ka, va = (blk(x).requires_grad_(True) for x in (q, k, v))
+        oa = ring.ring_attention(qa, ka, va, causal, scale, rg, ops)
+        oa.backward(blk(do))
+        errs["autograd_o"] = float((oa.detach() - o).abs().max())
+        for name, x in (("autograd_dq", qa), ("autograd_dk", ka), ("autograd_dv", va)):
+            errs[name] = float(np.max(np.abs(x.grad.numpy() - full[name[-2:]][:, :, rank * n:(rank + 1) * n])))
         out[rank] = errs
     finally:
         dist.barrier()
