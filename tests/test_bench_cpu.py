@@ -1,0 +1,72 @@
+"""CPU tests of bench.py's measurement logic: the FLOP convention against a brute
+count of visible (query, key) pairs, the workload table, the peak source, and the
+rule that a committed ncu traffic figure is used only while the kernel sources it
+was taken from are unchanged."""
+import numpy as np
+import pytest
+
+import bench
+
+
+def _visible_pairs(nq, nk, causal):
+    """Brute force: key j visible to query i iff j <= i + (nk - nq) under the causal mask."""
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    return int(np.sum(j <= i + (nk - nq))) if causal else nq * nk
+
+
+@pytest.mark.parametrize("nq,nk", [(128, 128), (300, 300), (512, 8192), (1, 1000), (77, 300)])
+def test_fwd_flops_counts_visible_pairs(nq, nk):
+    B, H, d = 2, 3, 64
+    assert bench.fwd_flops(B, H, nq, d, False, 1.0, nk) == 4.0 * B * H * d * _visible_pairs(nq, nk, False)
+    # causal: the exact count minus the diagonal's half (N^2 / 2 for a square problem,
+    # the convention of the pages' FLOP figures)
+    assert bench.fwd_flops(B, H, nq, d, True, 1.0, nk) == 4.0 * B * H * d * (_visible_pairs(nq, nk, True) - nq / 2)
+
+
+def test_fwd_flops_density_and_square_default():
+    assert bench.fwd_flops(1, 16, 16384, 64, False, 0.25) == 0.25 * 4.0 * 16 * 16384 ** 2 * 64
+    assert bench.fwd_flops(8, 16, 2048, 64, True) == 0.5 * bench.fwd_flops(8, 16, 2048, 64, False)
+
+
+def test_workload_table():
+    w = bench.workload("b8h16n2048d64")
+    assert (w["B"], w["H"], w["N"], w["Nk"], w["d"]) == (8, 16, 2048, 2048, 64)
+    assert [v[0] for v in w["variants"]] == ["noncausal", "causal"] and w["dropout_p"] == 0.0
+    c = bench.workload("b4h16q512k8192d128_causal")
+    assert (c["N"], c["Nk"], c["d"]) == (512, 8192, 128)
+    s = bench.workload("sweep_N4096_d128_causal")
+    assert (s["B"], s["H"], s["N"], s["d"]) == (4, 16, 4096, 128) and s["variants"][0][1] is True
+    sp = bench.workload("b1h16n16384d64_sparse")
+    assert sp["variants"] == [("blocksparse", False, 0.25)]
+    dr = bench.workload("b8h16n2048d64_dropout")
+    assert dr["dropout_p"] == 0.1
+
+
+def test_peaks_come_from_the_measured_file():
+    p, kind = bench.peaks()
+    assert kind == "measured" and p["bf16_tflops"] > 1000 and p["hbm_gbs"] > 1000
+
+
+def test_traffic_only_while_sources_unchanged(monkeypatch):
+    t = bench.profiled_traffic("fa_bwd_dkdv_kernel", "b8h16n2048d64")
+    assert t is not None and 1e8 < t < 3e8  # the committed figure for the current sources
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
+    assert bench.profiled_traffic("fa_bwd_dkdv_kernel", "b8h16n2048d64") is None
+    assert bench.profiled_traffic("fa_bwd_dkdv_kernel", "no_such_workload") is None
+
+
+def test_source_hash_covers_the_kernel_files(tmp_path, monkeypatch):
+    import os
+    import shutil
+    csrc = tmp_path / "exact_tiled_attention_34_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for fn in bench.KERNEL_SOURCES:
+        shutil.copy(os.path.join(bench.ROOT, "exact_tiled_attention_34_b200", "csrc", fn), csrc / fn)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    (csrc / "unrelated.cu").write_text("// not part of the profiled kernels\n")
+    assert bench.kernel_source_hash() == h0
+    with open(csrc / "fa_bwd.cuh", "a") as f:
+        f.write("\n")
+    assert bench.kernel_source_hash() != h0
