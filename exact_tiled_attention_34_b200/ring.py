@@ -147,19 +147,29 @@ def ring_backward(q, k, v, o, lse, do, causal=False, scale=None, ring=None, ops=
     state = ops.bwd_prepare(q, o, lse, do)
     dq = ops.zeros_f32(q)
     kv = [k, v]
-    dkv = [ops.zeros_f32(k), ops.zeros_f32(v)]  # accumulators of the block held now
+    dkv = [ops.zeros_f32(k), ops.zeros_f32(v)]  # accumulators of the block held at step 0 (own)
+    moving = None  # accumulators in flight to rank r + 1 (this step's arrive from rank r - 1)
     for s in range(R):
         src = (r - s) % R
         pending = ring.start(kv) if s < R - 1 else None
+        shares = None
         if _visible(causal, src, r):
-            dq_p, dk_p, dv_p = ops.bwd_block(state, q, kv[0], kv[1], do, causal and src == r)
-            ops.accumulate(dq, dq_p)
-            ops.accumulate(dkv[0], dk_p)
-            ops.accumulate(dkv[1], dv_p)
-        if R > 1:  # the accumulators follow their block; the last hop takes them home
-            dkv = ring.exchange(dkv)
+            shares = ops.bwd_block(state, q, kv[0], kv[1], do, causal and src == r)
+            ops.accumulate(dq, shares[0])
+        # The accumulators of block src travel with it: they arrive while this block's
+        # kernels run, take its shares, and leave for the next rank; after the last
+        # step that hop takes every block's accumulators home.
+        if moving is not None:
+            dkv = ring.finish(moving)
+        if shares is not None:
+            ops.accumulate(dkv[0], shares[1])
+            ops.accumulate(dkv[1], shares[2])
+        if R > 1:
+            moving = ring.start(dkv)
         if pending is not None:
             kv = ring.finish(pending)
+    if moving is not None:
+        dkv = ring.finish(moving)
     return ops.to_out(dq), ops.to_out(dkv[0]), ops.to_out(dkv[1])
 
 
