@@ -2,7 +2,12 @@
 emulated by host threads that hand each other tensors through queues (no kernel waits
 for another; all launches share one stream in the order the ranks make them). The
 output blocks are compared with the fp64 oracle on the whole sequence. Also the merge
-kernel on its own: two key halves merged equal attention over all keys."""
+kernel on its own: two key halves merged equal attention over all keys.
+
+The autograd wrapper is not run here: torch's autograd engine executes CUDA backward
+nodes on one worker thread per device, so emulated ranks blocking on each other inside
+their backward would wait forever; separate processes (the real setting) do not share
+that thread, and the wrapper is tested that way on gloo ranks."""
 import math
 import queue
 import threading
