@@ -267,8 +267,12 @@ fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void
  * Attention over a key sequence split into blocks (the sequence-parallel ring, where
  * each GPU holds one block of queries, keys and values and the key/value blocks
  * travel around the GPUs). Softmax attention over the union of two key sets is the
- * log-sum-exp-weighted mean of the two partial results, which is what the online
- * softmax of the method does tile by tile; these calls do it block by block.
+ * log-sum-exp-weighted mean of the two partial results: the combination the review's
+ * "Proposed method" performs tile by tile with its online softmax, and that the
+ * summary's saved normalisation factor makes possible afterwards; these calls do it
+ * block by block. Splitting one sequence across GPUs is not on the pages (they split
+ * it across the thread blocks of one GPU); fa_accumulate_bf16 and fa_to_bf16 are its
+ * plumbing and have no counterpart there.
  *
  * fa_merge_partial: merges a partial result (o_part bf16 [rows, d], lse_part fp32
  * [rows], as written by fa_fwd for one key block) into the running one (o_acc fp32
