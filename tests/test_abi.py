@@ -152,6 +152,14 @@ def test_merge_argument_checks(L):
     assert cv(A, A, 7, None) == INVALID and cv(A, None, 8, None) == INVALID and cv(A + 2, A, 8, None) == ALIGN
 
 
+def test_exp2_diagnostic_argument_checks(L):
+    e = L.fa_debug_exp2
+    assert e(A, A, -1, 0, None) == INVALID
+    assert e(A, A, 16, 2, None) == INVALID  # mode 0 (special-function unit) or 1 (polynomial)
+    assert e(None, None, 0, 1, None) == OK  # nothing to do
+    assert e(None, A, 16, 0, None) == INVALID
+
+
 def test_wait_timeout_argument_checks(L):
     f = L.fa_debug_wait_timeout
     assert f(0, A, None) == INVALID
