@@ -391,6 +391,9 @@ def merge_partial(o_acc, lse_acc, o_part, lse_part):
         raise ValueError("o_acc must be fp32 and o_part bf16 of one shape")
     if lse_acc.dtype != torch.float32 or lse_part.dtype != torch.float32 or lse_acc.shape != lse_part.shape:
         raise ValueError("lse_acc and lse_part must be fp32 of one shape")
+    # The kernel indexes O at row * d for every lse row: one lse entry per row of O.
+    if o_acc.dim() < 1 or tuple(lse_acc.shape) != tuple(o_acc.shape[:-1]):
+        raise ValueError("lse_acc must have the shape of o_acc without its last dimension")
     for t in (o_acc, lse_acc, o_part, lse_part):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError("contiguous CUDA tensors expected")

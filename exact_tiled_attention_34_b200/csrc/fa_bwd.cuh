@@ -49,6 +49,10 @@ namespace fa {
 // row arrays hold Npad = 128 * ceil(N / 128) rows per (batch, head): a tile's rows are
 // one 512-byte run. The pad rows of the last tile (n >= N, when N % 128 != 0) get
 // D = 0 and nl2 = -inf, so their recomputed P is 0 and they add nothing to dK or dV.
+// A row that sees no key (lse = -inf: an empty tile row of a block mask, or the causal
+// mask with N_q > N_k) also gets nl2 = -inf rather than +inf, so its exponents are
+// never +inf (2^(+inf) is not finite on either exponential path); its P is then 0
+// without relying on the element mask of the tiles it meets.
 // D / 8 threads per row, 16 bytes each; rows hold ds <= D columns (96 with D = 128).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
@@ -87,7 +91,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   for (int w = TPR / 2; w > 0; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
   if (inrange && part == 0) {
     Drow[prow] = s;
-    lse2[prow] = valid ? -lse[row] * 1.4426950408889634f : -INFINITY;
+    const float l = valid ? lse[row] : -INFINITY;
+    lse2[prow] = l > -INFINITY ? -l * 1.4426950408889634f : -INFINITY;
   }
 }
 

@@ -121,11 +121,22 @@ def _visible(causal, src, r):
     return (not causal) or src <= r
 
 
+def _check_block_shapes(q, k, v, ops):
+    """Reject, before any exchange is posted, what the library's per-block steps cannot
+    take: the merge kernel handles head dims 64 and 128 only (the attention kernels also
+    take 96), and every rank's key block must have the query block's shape."""
+    if tuple(k.shape) != tuple(q.shape) or tuple(v.shape) != tuple(q.shape):
+        raise ValueError("the ring needs q, k, v blocks of one shape [B, H, n, d]")
+    if isinstance(ops, CudaBlockOps) and q.shape[-1] not in (64, 128):
+        raise ValueError(f"head dim {q.shape[-1]}: the ring's merge step supports head dims 64 and 128")
+
+
 def ring_forward(q, k, v, causal=False, scale=None, ring=None, ops=None):
     """(O_r, lse_r) for this rank's query block against every rank's key block.
     q, k, v: this rank's [B, H, n, d] blocks (n equal on all ranks)."""
     ring = ProcessGroupRing() if ring is None else ring
     ops = CudaBlockOps(1.0 / math.sqrt(q.shape[-1]) if scale is None else scale) if ops is None else ops
+    _check_block_shapes(q, k, v, ops)
     R, r = ring.world, ring.rank
     acc = ops.new_acc(q)
     kv = [k, v]
@@ -143,6 +154,7 @@ def ring_backward(q, k, v, o, lse, do, causal=False, scale=None, ring=None, ops=
     """(dQ_r, dK_r, dV_r) for this rank's blocks, given the ring forward's O_r, lse_r."""
     ring = ProcessGroupRing() if ring is None else ring
     ops = CudaBlockOps(1.0 / math.sqrt(q.shape[-1]) if scale is None else scale) if ops is None else ops
+    _check_block_shapes(q, k, v, ops)
     R, r = ring.world, ring.rank
     state = ops.bwd_prepare(q, o, lse, do)
     dq = ops.zeros_f32(q)

@@ -25,7 +25,8 @@
  *    d innermost; element (b, h, n, c) at offset ((b*H + h)*N + n)*d + c.
  *  - lse: float32 [B, H, N]; lse[b,h,i] = ln sum_j exp(scale * q_i . k_j) over the
  *    keys visible to row i (natural log, scale and mask included); -INFINITY for
- *    a row that sees no key (possible only with a block mask).
+ *    a row that sees no key (a block mask whose tile row keeps nothing, or the
+ *    causal mask with N_q > N_k, where the first N_q - N_k queries see no key).
  *  - All pointers are DEVICE pointers on the current device, except where noted.
  *    Every base pointer must be 16-byte aligned.
  *  - Supported sizes: B, H, N >= 1 (any N; the kernels work on 128-row tiles and

@@ -6,6 +6,7 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
 from .attention import (  # noqa: F401
     attn_bwd_block_ref,
     attn_bwd_ref,
+    attn_dkdv_cols_ref,
     attn_dq_rows_ref,
     attn_fwd_block_ref,
     attn_fwd_ref,

@@ -57,6 +57,7 @@ __all__ = [
     "attn_fwd_rows_ref",
     "attn_bwd_ref",
     "attn_dq_rows_ref",
+    "attn_dkdv_cols_ref",
     "attn_fwd_block_ref",
     "attn_bwd_block_ref",
 ]
@@ -73,12 +74,13 @@ def _f64(x) -> np.ndarray:
 
 
 def _visible(n_q_rows: np.ndarray, n_k: int, causal: bool, block_mask, mask_block: int,
-             causal_offset: int = 0) -> np.ndarray:
-    """Boolean [len(rows), n_k] visibility for the given absolute query rows; with the
-    causal mask key j is visible to row i iff j <= i + causal_offset."""
+             causal_offset: int = 0, key_cols=None) -> np.ndarray:
+    """Boolean [len(rows), n_k] visibility for the given absolute query rows (or
+    [len(rows), len(key_cols)] for the given absolute key columns); with the causal mask
+    key j is visible to row i iff j <= i + causal_offset."""
     rows = np.asarray(n_q_rows, dtype=np.int64)
-    cols = np.arange(n_k, dtype=np.int64)
-    vis = np.ones((rows.shape[0], n_k), dtype=bool)
+    cols = np.arange(n_k, dtype=np.int64) if key_cols is None else np.asarray(key_cols, dtype=np.int64)
+    vis = np.ones((rows.shape[0], cols.shape[0]), dtype=bool)
     if causal:
         vis &= cols[None, :] <= rows[:, None] + causal_offset
     if block_mask is not None:
@@ -217,6 +219,38 @@ def attn_dq_rows_ref(q_rows, rows, k, v, do_rows, causal: bool, scale: float,
     D = np.sum(p * dp, axis=1)
     ds = p * (dp - D[:, None])
     return scale * (ds @ k)
+
+
+def attn_dkdv_cols_ref(q, k, v, do, cols, causal: bool, scale: float, block_mask=None,
+                       mask_block: int = 128, row_block: int = 1024):
+    """dK and dV for a sample of key rows (columns of S) of ONE head, same definition as
+    attn_bwd_ref, for sizes where the N x N matrices are too large to hold at once.
+
+    Column j of the gradients needs every query row's lse_i and D_i = sum_c dO_ic O_ic
+    over ALL keys, so those row statistics are computed first, row by row (``row_block``
+    rows at a time only to bound memory; each row is the plain softmax of its own
+    scores). Then, for the chosen keys j: P_ij = exp(S_ij - lse_i) (0 where masked or
+    where row i sees nothing), dP_ij = dO_i . v_j, dS_ij = P_ij (dP_ij - D_i),
+    dK_j = scale sum_i dS_ij q_i and dV_j = sum_i P_ij dO_i.
+    q, do [N_q, d]; k, v [N_k, d]; cols: absolute key indices. Returns (dK [C, d], dV [C, d]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    n_q, n_k = q.shape[0], k.shape[0]
+    cols = np.asarray(cols, dtype=np.int64)
+    lse = np.empty(n_q)
+    D = np.empty(n_q)
+    for r0 in range(0, n_q, row_block):
+        rows = np.arange(r0, min(n_q, r0 + row_block))
+        p, lse[rows] = _softmax_rows(attn_scores_ref(q[rows], k, scale, causal, block_mask, mask_block,
+                                                     rows=rows, n_q=n_q))
+        D[rows] = np.sum(do[rows] * (p @ v), axis=1)
+    vis = _visible(np.arange(n_q), n_k, causal, block_mask, mask_block, n_k - n_q, key_cols=cols)
+    s_c = np.where(vis, float(scale) * (q @ k[cols].T), -np.inf)
+    fin = np.isfinite(lse)[:, None]
+    p_c = np.where(vis & fin, np.exp(s_c - np.where(fin, lse[:, None], 0.0)), 0.0)
+    dp_c = do @ v[cols].T
+    ds_c = p_c * (dp_c - D[:, None])
+    return scale * (ds_c.T @ q), p_c.T @ do
 
 
 # ---------------------------------------------------------------- key blocks

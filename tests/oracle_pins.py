@@ -281,6 +281,35 @@ def pin_dq_rows_match_full(mod):
         assert np.allclose(dq, g["dq"][0, 0, rows], atol=1e-12)
 
 
+def pin_dkdv_cols_match_full(mod):
+    """The sampled-key dK, dV equal the corresponding rows of the full backward: square
+    problems (dense, causal, block mask with an empty tile row, so some rows see nothing)
+    and N_q != N_k with the causal mask (more keys than queries, and more queries than
+    keys, where the leading rows see nothing); row statistics taken in blocks of 3 rows
+    and in one block give the same result."""
+    T = 4
+    cases = []
+    N = 16
+    q, k, v, do = (_rand((N, 4), s) for s in (62, 63, 64, 65))
+    mask = _tiny_mask(N, T, seed=66)
+    mask[1, :] = 0  # query tile 1 sees no key
+    cases += [(q, k, v, do, False, None), (q, k, v, do, True, None), (q, k, v, do, False, mask)]
+    for nq, nk in ((6, 11), (11, 6)):
+        qx, dox = _rand((nq, 4), 67 + nq), _rand((nq, 4), 68 + nq)
+        kx, vx = _rand((nk, 4), 69 + nk), _rand((nk, 4), 70 + nk)
+        cases.append((qx, kx, vx, dox, True, None))
+    for (qq, kk, vv, dd, causal, m) in cases:
+        g = mod.attn_bwd_ref(qq[None, None], kk[None, None], vv[None, None], dd[None, None], causal, 0.7, m, T)
+        nk = kk.shape[0]
+        cols = np.array(sorted({0, 1, nk // 2, nk - 2, nk - 1}))
+        for rb in (3, 1024):
+            dk, dv = mod.attn_dkdv_cols_ref(qq, kk, vv, dd, cols, causal, 0.7, m, T, row_block=rb)
+            assert np.allclose(dk, g["dk"][0, 0, cols], atol=1e-12), (causal, rb)
+            assert np.allclose(dv, g["dv"][0, 0, cols], atol=1e-12), (causal, rb)
+        dk_all, dv_all = mod.attn_dkdv_cols_ref(qq, kk, vv, dd, np.arange(nk), causal, 0.7, m, T, row_block=5)
+        assert np.allclose(dk_all, g["dk"][0, 0], atol=1e-12) and np.allclose(dv_all, g["dv"][0, 0], atol=1e-12)
+
+
 # ---------------------------------------------------------------- N_q != N_k (bottom-right causal)
 
 def pin_cross_decode_sees_every_key(mod):
@@ -449,6 +478,7 @@ BACKWARD_PINS = [
     pin_D_two_ways,
     pin_gradient_invariants,
     pin_dq_rows_match_full,
+    pin_dkdv_cols_match_full,
 ]
 CROSS_PINS = [
     pin_cross_decode_sees_every_key,

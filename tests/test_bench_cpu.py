@@ -55,12 +55,29 @@ def test_peaks_come_from_the_measured_file():
     assert p["bf16_tflops"] > 1000 and p["hbm_gbs"] > 1000
 
 
-def test_traffic_only_while_sources_unchanged(monkeypatch):
-    t = bench.profiled_traffic("fa_bwd_dkdv_kernel", "b8h16n2048d64")
-    assert t is not None and 1e8 < t < 3e8  # the committed figure for the current sources
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
-    assert bench.profiled_traffic("fa_bwd_dkdv_kernel", "b8h16n2048d64") is None
+def test_traffic_only_while_sources_unchanged(tmp_path, monkeypatch):
+    """A committed ncu figure is reported only while the kernel sources hash to the value
+    stored with it."""
+    h = bench.kernel_source_hash()
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "fa_bwd_dkdv_kernel_wl.txt").write_text(
+        "# capture notes\nsource_hash: %s\ndram_bytes_per_launch: 123456789\n" % h)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: h)
+    assert bench.profiled_traffic("fa_bwd_dkdv_kernel", "wl") == 123456789.0
     assert bench.profiled_traffic("fa_bwd_dkdv_kernel", "no_such_workload") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
+    assert bench.profiled_traffic("fa_bwd_dkdv_kernel", "wl") is None
+
+
+def test_default_workload_is_the_long_context_config():
+    """The default bench line is the largest single-GPU workload, the one the head-dim-128
+    targets are stated on: B=2, H=16, N=8192, d=128, causal, forward + backward."""
+    args = bench.build_parser().parse_args([])
+    w = bench.workload(args.workload)
+    assert (w["B"], w["H"], w["N"], w["d"]) == (2, 16, 8192, 128)
+    assert [v[0] for v in w["variants"]] == ["causal"]
+    assert args.gpus == 1 and args.warmup >= 3
 
 
 def test_source_hash_covers_the_kernel_files(tmp_path, monkeypatch):

@@ -46,6 +46,10 @@ def test_merge_and_accumulate_check_dtypes_and_devices():
         fa.merge_partial(acc, lse.double(), part, lse)
     with pytest.raises(ValueError):
         fa.merge_partial(acc, lse, part, lse)  # CPU tensors
+    with pytest.raises(ValueError):  # more lse rows than rows of O: the kernel would run past O
+        fa.merge_partial(acc, torch.zeros(1, 1, 256), part, torch.zeros(1, 1, 256))
+    with pytest.raises(ValueError):  # fewer lse rows than rows of O
+        fa.merge_partial(acc, torch.zeros(1, 1, 64), part, torch.zeros(1, 1, 64))
     with pytest.raises(ValueError):
         fa.accumulate_bf16(acc, acc)
     with pytest.raises(ValueError):
@@ -58,3 +62,29 @@ def test_ring_visibility_rule():
     # causal: key block src is visible to query block r iff src <= r; all without the mask
     assert [ring._visible(True, s, 2) for s in range(4)] == [True, True, True, False]
     assert all(ring._visible(False, s, 0) for s in range(4))
+
+
+class _RingThatMustNotExchange:
+    """A two-rank ring whose exchange fails the test if it is ever started."""
+    rank, world = 0, 2
+
+    def start(self, tensors):
+        raise AssertionError("an exchange was posted before the arguments were checked")
+
+    finish = exchange = start
+
+
+def test_ring_rejects_head_dim_96_before_any_exchange():
+    q = _bf16(1, 1, 128, 96)
+    ops = ring.CudaBlockOps(0.1)
+    with pytest.raises(ValueError):
+        ring.ring_forward(q, q, q, ring=_RingThatMustNotExchange(), ops=ops)
+    lse = torch.zeros(1, 1, 128)
+    with pytest.raises(ValueError):
+        ring.ring_backward(q, q, q, q, lse, q, ring=_RingThatMustNotExchange(), ops=ops)
+
+
+def test_ring_rejects_blocks_of_different_shapes():
+    q, k = _bf16(1, 1, 128, 64), _bf16(1, 1, 256, 64)
+    with pytest.raises(ValueError):
+        ring.ring_forward(q, k, k, ring=_RingThatMustNotExchange(), ops=ring.CudaBlockOps(0.1))

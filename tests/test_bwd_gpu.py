@@ -115,6 +115,24 @@ def test_workspace_too_small_is_rejected(cuda_device):
     assert e.value.status == 4
 
 
+def _sampled_bwd_check(t, grads, causal, sc, heads, rows, cols, mask=None, what=""):
+    """Element-wise comparison with the oracle on sampled query rows (dQ) and sampled key
+    rows (dK, dV) of the given heads; each tensor's bound is 2e-2 times the largest
+    oracle value among its samples."""
+    dq, dk, dv = grads
+    mk = None if mask is None else mask.cpu().numpy()
+    ridx, cidx = torch.as_tensor(rows), torch.as_tensor(cols)
+    for (b, h) in heads:
+        c = {k: x[b, h].cpu() for k, x in t.items()}
+        w = f"{what} (b={b}, h={h})"
+        ref_dq = oracle.attn_dq_rows_ref(f64(c["q"])[rows], rows, c["k"], c["v"], f64(c["do"])[rows], causal, sc,
+                                         mk, 128)
+        assert_grad_close(dq[b, h].cpu()[ridx], ref_dq, "dq", w)
+        ref_dk, ref_dv = oracle.attn_dkdv_cols_ref(c["q"], c["k"], c["v"], c["do"], cols, causal, sc, mk, 128)
+        assert_grad_close(dk[b, h].cpu()[cidx], ref_dk, "dk", w)
+        assert_grad_close(dv[b, h].cpu()[cidx], ref_dv, "dv", w)
+
+
 def _invariants(t, dk, dv):
     """sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i for every head (any size)."""
     dk64 = dk.double()
@@ -139,24 +157,22 @@ def test_b2h16n8192d128_causal(cuda_device):
 
 
 def test_b1h16n16384d64_sparse(cuda_device):
-    """Full size: sampled dQ rows from the oracle, gradient invariants on every head,
-    and the full oracle on a 2048-token case with the same mask density."""
+    """Full size with the 128 x 128 tile mask: element-wise oracle comparison of sampled
+    dQ rows and sampled dK, dV key rows (tile boundaries, keys of tiles that few query
+    tiles keep, random keys) on three heads, gradient invariants on every head, and the
+    full oracle on a 2048-token case with the same mask density."""
     B, H, N, d = 1, 16, 16384, 64
     mask = make_tile_mask(N // 128, seed=0, density=0.25)
     t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, N, d, seed=0).items()}
     sc = 1.0 / math.sqrt(d)
-    o, lse, (dq, dk, dv) = _run(t, False, sc, mask.to(cuda_device))
-    _invariants(t, dk, dv)
-    rows = sample_rows(N, n_random=16)
-    idx = torch.as_tensor(rows)
-    mk = mask.numpy()
-    for h in (0, 9, 15):
-        c = {k: x[0, h].cpu() for k, x in t.items()}
-        ref = oracle.attn_dq_rows_ref(f64(c["q"])[rows], rows, c["k"], c["v"], f64(c["do"])[rows], False, sc, mk,
-                                      128)
-        full_scale = float(np.max(np.abs(ref)))
-        err = float(np.max(np.abs(f64(dq[0, h].cpu()[idx]) - ref)))
-        assert err <= TOL_GRAD_REL * full_scale, (h, err, full_scale)
+    o, lse, grads = _run(t, False, sc, mask.to(cuda_device))
+    _invariants(t, grads[1], grads[2])
+    rows = sample_rows(N, n_random=24)
+    # key tiles kept by the fewest and by the most query tiles, plus boundaries and random keys
+    kept = mask.sum(dim=0).numpy()
+    extra = [int(np.argmin(kept)) * 128 + 5, int(np.argmax(kept)) * 128 + 64]
+    cols = np.array(sorted(set(sample_rows(N, n_random=24, seed=1).tolist()) | set(extra)))
+    _sampled_bwd_check(t, grads, False, sc, [(0, 0), (0, 9), (0, 15)], rows, cols, mask, "B1 H16 N16384 d64 sparse")
     small = make_tile_mask(16, seed=0, density=0.25)
     _full_check(1, 2, 2048, 64, False, cuda_device, mask=small)
 
@@ -169,6 +185,24 @@ def test_sweep_points(cuda_device, N, d):
         t, (dq, dk, dv), _ = _full_check(B, H, N, d, causal, cuda_device, do_scale=0.5,
                                           heads=[(0, 0), (B - 1, H - 1)])
         _invariants(t, dk, dv)
+
+
+@pytest.mark.parametrize("N", [1024, 2048, 8192, 16384])
+@pytest.mark.parametrize("d", [64, 128])
+def test_sweep_points_sampled(cuda_device, N, d):
+    """The other sweep lengths at full size (B N = 16384 tokens, H = 2048 / d), causal and
+    not: sampled dQ rows and dK, dV key rows of two heads against the oracle, and the
+    gradient invariants on every head."""
+    B, H = sweep_shape(N, d)
+    sc = 1.0 / math.sqrt(d)
+    t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, N, d, seed=0, do_scale=0.5).items()}
+    rows = sample_rows(N, n_random=16)
+    cols = sample_rows(N, n_random=16, seed=1)
+    for causal in (False, True):
+        _, _, grads = _run(t, causal, sc)
+        _invariants(t, grads[1], grads[2])
+        _sampled_bwd_check(t, grads, causal, sc, [(0, 0), (B - 1, H - 1)], rows, cols, None,
+                           f"B{B} H{H} N{N} d{d} causal={causal}")
 
 
 @pytest.mark.parametrize("d", [64, 128])

@@ -39,6 +39,12 @@ def _check(B, H, Nq, Nk, d, causal, dev, seed=0):
     for (big, _), n in ((gq, math.prod(qs)), (gk, math.prod(ks)), (gv, math.prod(ks))):
         assert _tail_untouched(big, n, float("nan")), "gradient written past its end"
     what = f"B{B} H{H} Nq{Nq} Nk{Nk} d{d} causal={causal}"
+    if causal and Nq > Nk:
+        # the first Nq - Nk queries see no key: lse -inf, O and dQ exactly 0 (finite)
+        blind = slice(0, Nq - Nk)
+        assert torch.all(torch.isneginf(lse[:, :, blind]))
+        assert torch.all(torch.isfinite(dq[:, :, blind])) and torch.all(dq[:, :, blind] == 0)
+        assert torch.all(o[:, :, blind] == 0)
     for b in range(B):
         for h in range(H):
             sl = lambda x: x[b:b + 1, h:h + 1].cpu()

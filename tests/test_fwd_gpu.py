@@ -130,8 +130,8 @@ def _sampled(B, H, N, d, causal, dev, mask=None, do_scale=1.0):
         o, lse = fa.forward_blocksparse(t["q"], t["k"], t["v"], mask.to(dev), scale=sc)
     torch.cuda.synchronize()
     assert fa.device_status() == (0, 0)
-    heads = sorted({(0, 0), (B - 1, H - 1), (B // 2, H // 2)})
-    rows = sample_rows(N)
+    heads = sorted({(0, 0), (B - 1, H - 1), (B // 2, H // 2), (0, H - 1), (B - 1, 0)})
+    rows = sample_rows(N, n_random=48)
     o_c, lse_c = o.cpu(), lse.cpu()
     t_c = {k: x.cpu() for k, x in t.items()}
     return sampled_fwd_check(t_c["q"], t_c["k"], t_c["v"], o_c, lse_c, causal, sc, heads, rows,
@@ -153,7 +153,7 @@ def test_b1h16n16384d64_sparse(cuda_device):
     _sampled(1, 16, 16384, 64, False, cuda_device, mask=mask)
 
 
-@pytest.mark.parametrize("N", [512, 1024, 4096, 16384])
+@pytest.mark.parametrize("N", [512, 1024, 2048, 4096, 8192, 16384])
 @pytest.mark.parametrize("d", [64, 128])
 def test_sweep_points(cuda_device, N, d):
     B, H = sweep_shape(N, d)

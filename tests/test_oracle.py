@@ -55,6 +55,13 @@ MUTATIONS = {
     "block_offsets_swapped": ("rows = q_off + np.arange(s.shape[0])[:, None]",
                               "rows = k_off + np.arange(s.shape[0])[:, None]"),
     "block_ds_dropped_D": ("ds = p * (dp - _f64(D)[:, None])", "ds = p * dp"),
+    "cols_p_without_lse": ("np.exp(s_c - np.where(fin, lse[:, None], 0.0))", "np.exp(s_c)"),
+    "cols_ds_dropped_D": ("ds_c = p_c * (dp_c - D[:, None])", "ds_c = p_c * dp_c"),
+    "cols_dp_wrong_operand": ("dp_c = do @ v[cols].T", "dp_c = do @ k[cols].T"),
+    "cols_dk_dropped_scale": ("return scale * (ds_c.T @ q), p_c.T @ do", "return (ds_c.T @ q), p_c.T @ do"),
+    "cols_D_without_o": ("D[rows] = np.sum(do[rows] * (p @ v), axis=1)", "D[rows] = np.sum(do[rows] * v[rows], axis=1)"),
+    "cols_causal_offset_dropped": ("mask_block, n_k - n_q, key_cols=cols)", "mask_block, 0, key_cols=cols)"),
+    "cols_last_row_block_skipped": ("for r0 in range(0, n_q, row_block):", "for r0 in range(0, n_q - row_block, row_block):"),
     "block_dv_from_q": ("return scale * (ds @ k), scale * (ds.T @ q), p.T @ do",
                         "return scale * (ds @ k), scale * (ds.T @ q), p.T @ q"),
 }
