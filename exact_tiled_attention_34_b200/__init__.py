@@ -27,7 +27,7 @@ import re
 __all__ = [
     "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
     "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_dkdv",
-    "bwd_dq", "attention", "attention_blocksparse", "forward_dropout", "backward_dropout", "merge_partial",
+    "bwd_dq", "bwd_fused_preprocess", "bwd_fused_main", "bwd_fused_dq", "attention", "attention_blocksparse", "forward_dropout", "backward_dropout", "merge_partial",
     "accumulate_bf16", "to_bf16",
 ]
 
@@ -74,6 +74,12 @@ _SIGS = {
     "fa_merge_partial": ([_vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _vp], _i),
     "fa_accumulate_bf16": ([_vp, _vp, ctypes.c_longlong, _i, _vp], _i),
     "fa_to_bf16": ([_vp, _vp, ctypes.c_longlong, _vp], _i),
+    "fa_bwd_fused_workspace_bytes": ([_i] * 4, _sz),
+    "fa_bwd_fused": ([_vp] * 10 + [_sz] + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_fused_ex": ([_vp] * 10 + [_sz, _vp, _i] + [_i] * 7 + [_f, _vp], _i),
+    "fa_bwd_fused_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
+    "fa_bwd_fused_main": ([_vp] * 7 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_fused_dq": ([_vp, _vp, _sz] + [_i] * 4 + [_f, _vp], _i),
     "fa_debug_exp2": ([_vp, _vp, _i, _i, _vp], _i),
     "fa_debug_wait_timeout": ([_i, _vp, _vp], _i),
     "fa_debug_stall_producer": ([_i, _i], _i),
@@ -226,17 +232,21 @@ def forward_dropout(q, k, v, p: float, seed: int, offset: int = 0, causal: bool 
     return o, l
 
 
-def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
-    return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int, deterministic: bool = True) -> int:
+    """Workspace bytes of the deterministic backward, or (deterministic=False) of the
+    fused backward, which also holds an fp32 dQ accumulator."""
+    if deterministic:
+        return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+    return int(lib().fa_bwd_fused_workspace_bytes(B, H, N, d))
 
 
-def _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout="bhnd"):
+def _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout="bhnd", deterministic=True):
     import torch
     _check_qkv(q, k, v, o, do, layout=layout)
     B, H, N, _, d = _dims(q, k, layout)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
         raise ValueError("lse must be contiguous fp32 [B, H, N]")
-    need = bwd_workspace_bytes(B, H, N, d)
+    need = bwd_workspace_bytes(B, H, N, d, deterministic)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if grads is None:
@@ -244,10 +254,30 @@ def _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout="bhnd"):
     return workspace, grads
 
 
-def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None, grads=None,
-             layout: str = "bhnd"):
-    """Gradients (dq, dk, dv) of sum(O * dO) given the forward's o and lse."""
+def _bwd_fused(q, k, v, o, lse, do, causal, scale, workspace, grads, layout, tile_mask, mask_block):
     import torch
+    workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout, deterministic=False)
+    B, H, N, Nk, d = _dims(q, k, layout)
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_fused_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel(), None if tile_mask is None else tile_mask.data_ptr(),
+                                   mask_block, B, H, N, Nk, d, _LAYOUTS[layout], int(bool(causal)),
+                                   _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_bwd_fused_ex")
+    return dq, dk, dv
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None, grads=None,
+             layout: str = "bhnd", deterministic: bool = True):
+    """Gradients (dq, dk, dv) of sum(O * dO) given the forward's o and lse.
+
+    deterministic=True: the two-kernel backward (bit-reproducible). False: the fused
+    single kernel (five products per tile pair instead of seven; dq accumulated in fp32
+    in an order that varies from run to run)."""
+    import torch
+    if not deterministic:
+        return _bwd_fused(q, k, v, o, lse, do, causal, scale, workspace, grads, layout, None, 128)
     workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout)
     B, H, N, Nk, d = _dims(q, k, layout)
     with torch.cuda.device(q.device):
@@ -288,10 +318,12 @@ def backward_dropout(q, k, v, o, lse, do, p: float, seed: int, offset: int = 0, 
 
 
 def backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None, mask_block: int = 128, workspace=None,
-                         grads=None):
-    """Block-sparse backward (same mask as the forward)."""
+                         grads=None, deterministic: bool = True):
+    """Block-sparse backward (same mask as the forward); deterministic as for backward."""
     import torch
     _check_mask(tile_mask, q, mask_block)
+    if not deterministic:
+        return _bwd_fused(q, k, v, o, lse, do, False, scale, workspace, grads, "bhnd", tile_mask, mask_block)
     workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
     B, H, N, d = q.shape
     with torch.cuda.device(q.device):
@@ -345,6 +377,38 @@ def bwd_dq(q, k, v, do, dq, workspace, causal=False, scale=None, tile_mask=None,
                              None if tile_mask is None else tile_mask.data_ptr(), mask_block,
                              B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
     _check(st, "fa_bwd_dq")
+
+
+# The three launches of ``backward(..., deterministic=False)`` as separate calls
+# (workspace of bwd_workspace_bytes(..., deterministic=False), the same for all three).
+
+def bwd_fused_preprocess(o, do, lse, workspace):
+    import torch
+    B, H, N, d = o.shape
+    with torch.cuda.device(o.device):
+        st = lib().fa_bwd_fused_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel(), B, H, N, d, _stream_ptr(o.device))
+    _check(st, "fa_bwd_fused_preprocess")
+
+
+def bwd_fused_main(q, k, v, do, dk, dv, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
+    import torch
+    B, H, N, d = q.shape
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_fused_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
+                                     dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                     None if tile_mask is None else tile_mask.data_ptr(), mask_block,
+                                     B, H, N, d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_bwd_fused_main")
+
+
+def bwd_fused_dq(dq, workspace, scale=None):
+    import torch
+    B, H, N, d = dq.shape
+    with torch.cuda.device(dq.device):
+        st = lib().fa_bwd_fused_dq(dq.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, N, d,
+                                   _scale(scale, d), _stream_ptr(dq.device))
+    _check(st, "fa_bwd_fused_dq")
 
 
 def debug_exp2(x, mode: int):

@@ -13,6 +13,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_fused.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -329,7 +330,7 @@ fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d,
 }
 
 fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, size_t ws_bytes, int B, int H, int N,
-                  int d, int layout, void* stream) {
+                  int d, int layout, void* stream, float* dqacc = nullptr) {
   fa_status s;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
   const int bnhd = layout == FA_LAYOUT_BNHD ? 1 : 0;
@@ -343,9 +344,10 @@ fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, siz
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   const long long rows = static_cast<long long>(a.rows);
   if (d == 64)
-    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows);
+    fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows, dqacc);
   else  // 96 or 128 (16 threads per row)
-    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows);
+    fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows,
+                                                     dqacc);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -649,6 +651,224 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
   if (mask_block != 128) return FA_ERR_UNSUPPORTED;
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, B, H, N, N, d,
                     FA_LAYOUT_BHND, 0, scale, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------- fused backward
+// One kernel for dK, dV and dQ (five products per tile pair instead of seven), with
+// dQ reduced in fp32 into the workspace and converted to bf16 by a last launch.
+namespace {
+
+int dq_width(int d) { return d == 64 ? 64 : 128; }  // columns of the fp32 dQ accumulator
+
+// Workspace: the two row arrays of the deterministic backward, then the fp32 dQ
+// accumulator [B*H, Npad, 64 or 128], 256-byte aligned.
+size_t fused_ws_bytes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  const size_t rows = size_t(B) * H * ((size_t(N) + 127) / 128 * 128);
+  return bwd_ws_bytes(B, H, N, d) + round256(rows * size_t(dq_width(d)) * 4);
+}
+
+float* fused_dqacc(const void* ws, int B, int H, int N, int d) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(const_cast<void*>(ws)) + bwd_ws_bytes(B, H, N, d));
+}
+
+fa_status fused_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a) {
+  fa_status s;
+  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, a)) != FA_OK) return s;
+  return ws_bytes < fused_ws_bytes(B, H, N, d) ? FA_ERR_WORKSPACE : FA_OK;
+}
+
+// The fp32 accumulator [BH, Npad, Dk] as a 3-D tensor (column, row, batch*head) for
+// 32 x 32 reduce-add boxes with 128-byte swizzle (a box row is 32 fp32 = 128 bytes).
+fa_status make_acc_map(CUtensorMap* m, const float* base, int BH, int Npad, int Dk) {
+  cuuint64_t dims[3] = {cuuint64_t(Dk), cuuint64_t(Npad), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(Dk) * 4, cuuint64_t(Npad) * cuuint64_t(Dk) * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false>
+fa_status launch_fused(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                       const CUtensorMap& macc, const fa::BwdParams& p, cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  static int regs[kMaxDevices];
+  auto kernel = fa::fa_bwd_fused_kernel<D, CAUSAL, SPARSE, XQK>;
+  constexpr int smem = fa::FusedCfg<D>::kSmemBytes;
+  if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  if (regs[dev] == 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+    regs[dev] = attr.numRegs;
+  }
+  // The kernel re-divides its register pool between warpgroups.
+  if (regs[dev] * fa::kBwdThreads < fa::kFusedRegsNeeded) return FA_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return FA_ERR_CUDA;
+  unsigned grid = unsigned(p.n_ktiles) * unsigned(p.BH);
+  if (grid > unsigned(sms)) grid = unsigned(sms);  // persistent: at most one CTA per SM
+  kernel<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, macc, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// D and -lse log2 e rows, and the zeroed dQ accumulator.
+fa_status fused_pre(const void* o, const void* dO, const float* lse, void* ws, size_t ws_bytes, int B, int H, int N,
+                    int d, int layout, void* stream) {
+  BwdArgs a;
+  fa_status s;
+  if (ws == nullptr) return FA_ERR_INVALID_ARG;
+  if ((s = fused_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  return bwd_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, layout, stream, fused_dqacc(ws, B, H, N, d));
+}
+
+// The fused kernel: dk, dv written, dQ added into the accumulator (which the
+// pre-pass must have zeroed).
+fa_status fused_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const void* ws,
+                     size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H, int N, int Nk, int d,
+                     int layout, int causal, float scale, void* stream) {
+  fa_status s;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
+  const bool bnhd = layout == FA_LAYOUT_BNHD;
+  if ((s = check_ptrs({q, k, v, dO, dk, dv})) != FA_OK) return s;
+  if (mask != nullptr && (mask_block != 128 || causal || Nk != N)) return FA_ERR_UNSUPPORTED;
+  if (ws == nullptr) return FA_ERR_INVALID_ARG;
+  BwdArgs a;
+  if ((s = fused_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if ((s = encoder()) != FA_OK) return s;
+  int* status;
+  if ((s = device_status_ptr(&status)) != FA_OK) return s;
+  CUtensorMap mq, mk, mv, mdo, macc;
+  if ((s = make_map(&mq, q, B, H, N, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mk, k, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mv, v, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_map(&mdo, dO, B, H, N, d, bnhd, 128)) != FA_OK) return s;
+  if ((s = make_acc_map(&macc, fused_dqacc(ws, B, H, N, d), a.BH, a.Npad, dq_width(d))) != FA_OK) return s;
+  fa::BwdParams p;
+  p.lse2 = a.lse2;
+  p.Drow = a.Drow;
+  p.dq = nullptr;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.tile_mask = mask;
+  p.status = status;
+  set_wait_limit(&p.timeout_ns, &p.stall);
+  p.N = N;
+  p.Nk = Nk;
+  p.BH = a.BH;
+  p.H = H;
+  p.bnhd = bnhd ? 1 : 0;
+  p.v8 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
+  p.n_tiles = (N + 127) / 128;
+  p.n_ktiles = (Nk + 127) / 128;
+  p.off = Nk - N;
+  p.ds = d;
+  p.scale = scale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mask)
+    return d == 64 ? launch_fused<64, false, true>(mq, mk, mv, mdo, macc, p, st)
+                   : launch_fused<128, false, true>(mq, mk, mv, mdo, macc, p, st);
+  if (causal && Nk != N)
+    return d == 64 ? launch_fused<64, true, false, true>(mq, mk, mv, mdo, macc, p, st)
+                   : launch_fused<128, true, false, true>(mq, mk, mv, mdo, macc, p, st);
+  if (causal)
+    return d == 64 ? launch_fused<64, true, false>(mq, mk, mv, mdo, macc, p, st)
+                   : launch_fused<128, true, false>(mq, mk, mv, mdo, macc, p, st);
+  return d == 64 ? launch_fused<64, false, false>(mq, mk, mv, mdo, macc, p, st)
+                 : launch_fused<128, false, false>(mq, mk, mv, mdo, macc, p, st);
+}
+
+// dq = bf16(scale * accumulator) for the N real rows of every (batch, head).
+fa_status fused_dq(void* dq, const void* ws, size_t ws_bytes, int B, int H, int N, int d, int layout, float scale,
+                   void* stream) {
+  fa_status s;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
+  if ((s = check_ptrs({dq})) != FA_OK) return s;
+  if (ws == nullptr) return FA_ERR_INVALID_ARG;
+  BwdArgs a;
+  if ((s = fused_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  const long long rows = static_cast<long long>(a.BH) * N;
+  const int Dk = dq_width(d);
+  const long long threads = rows * (Dk / 8);
+  const unsigned grid = unsigned((threads + 255) / 256);
+  const float* acc = fused_dqacc(ws, B, H, N, d);
+  auto* out = static_cast<__nv_bfloat16*>(dq);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bnhd = layout == FA_LAYOUT_BNHD ? 1 : 0;
+  if (Dk == 64)
+    fa::fa_dq_convert_kernel<64><<<grid, 256, 0, st>>>(acc, out, N, a.Npad, d, H, bnhd, rows, scale);
+  else
+    fa::fa_dq_convert_kernel<128><<<grid, 256, 0, st>>>(acc, out, N, a.Npad, d, H, bnhd, rows, scale);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fused_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                       void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const uint8_t* mask, int mask_block,
+                       int B, int H, int N, int Nk, int d, int layout, int causal, float scale, void* stream) {
+  fa_status s;
+  // Validate everything before the first launch so that an error writes nothing.
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
+  if ((s = check_ptrs({q, k, v, o, lse, dO, dq, dk, dv})) != FA_OK) return s;
+  if (ws == nullptr) return FA_ERR_INVALID_ARG;
+  BwdArgs a;
+  if ((s = fused_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if (mask != nullptr && (mask_block != 128 || causal || Nk != N)) return FA_ERR_UNSUPPORTED;
+  if ((s = fused_pre(o, dO, lse, ws, ws_bytes, B, H, N, d, layout, stream)) != FA_OK) return s;
+  if ((s = fused_main(q, k, v, dO, dk, dv, ws, ws_bytes, mask, mask_block, B, H, N, Nk, d, layout, causal, scale,
+                      stream)) != FA_OK)
+    return s;
+  return fused_dq(dq, ws, ws_bytes, B, H, N, d, layout, scale, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_bwd_fused_workspace_bytes(int B, int H, int N, int d) { return fused_ws_bytes(B, H, N, d); }
+
+fa_status fa_bwd_fused(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                       void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N,
+                       int d, int causal, float scale, void* stream) {
+  return fused_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, nullptr, 128, B, H, N, N, d,
+                      FA_LAYOUT_BHND, causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_fused_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                          const uint8_t* tile_mask, int mask_block, int B, int H, int Nq, int Nk, int d, int layout,
+                          int causal, float scale, void* stream) {
+  return fused_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, Nq,
+                      Nk, d, layout, causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_fused_preprocess(const void* o, const void* dO, const float* lse, void* workspace,
+                                  size_t workspace_bytes, int B, int H, int N, int d, void* stream) {
+  return fused_pre(o, dO, lse, workspace, workspace_bytes, B, H, N, d, FA_LAYOUT_BHND, stream);
+}
+
+fa_status fa_bwd_fused_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, const uint8_t* tile_mask, int mask_block, int B,
+                            int H, int N, int d, int causal, float scale, void* stream) {
+  return fused_main(q, k, v, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N, N, d,
+                    FA_LAYOUT_BHND, causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_fused_dq(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                          float scale, void* stream) {
+  return fused_dq(dq, workspace, workspace_bytes, B, H, N, d, FA_LAYOUT_BHND, scale, stream);
 }
 
 }  // extern "C"

@@ -54,12 +54,15 @@ namespace fa {
 // never +inf (2^(+inf) is not finite on either exponential path); its P is then 0
 // without relying on the element mask of the tiles it meets.
 // D / 8 threads per row, 16 bytes each; rows hold ds <= D columns (96 with D = 128).
+// dqacc (or nullptr): an fp32 [rows_pad, D] accumulator that the fused backward adds
+// dQ into; it is zeroed here (pad rows included), each thread 8 columns of its row.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse, float* __restrict__ Drow,
                                                          float* __restrict__ lse2, int N, int Npad, int ds,
-                                                         int H, int bnhd, long long rows_pad) {
+                                                         int H, int bnhd, long long rows_pad,
+                                                         float* __restrict__ dqacc) {
   constexpr int TPR = D / 8;
   const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long prow = g / TPR;  // padded row index: bh * Npad + n
@@ -86,6 +89,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
       s = fmaf(x.x, y.x, s);
       s = fmaf(x.y, y.y, s);
     }
+  }
+  if (dqacc != nullptr && inrange) {
+    float4* z = reinterpret_cast<float4*>(dqacc + static_cast<size_t>(prow) * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int w = TPR / 2; w > 0; w >>= 1) s += __shfl_xor_sync(0xffffffffu, s, w);

@@ -224,6 +224,60 @@ fa_status fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
                     int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * Fused backward: the same gradients as fa_bwd from ONE kernel per call instead of two,
+ * executing five matrix products per (key tile, query tile) pair instead of seven (the
+ * summary's recomputation: S and dP are formed once per pair; the deterministic path
+ * forms them a second time for dq). dQ_i's share from each key tile is added in fp32
+ * into an accumulator in the workspace with the tensor memory accelerator's bulk
+ * reduce-add, then converted: dq = bf16(scale * accumulator).
+ *   NOT bit-reproducible: the key tiles add into a dq row in an order that varies from
+ *   run to run (fp32 sums; dk and dv are deterministic). Use fa_bwd when run-to-run
+ *   identical gradients are required.
+ *   workspace : at least fa_bwd_fused_workspace_bytes(B,H,N,d) bytes, 256-byte
+ *               aligned (the two row arrays of fa_bwd, then the fp32 accumulator
+ *               [B*H, Npad, 64 (d = 64) or 128 (d = 96, 128)]); contents on entry do
+ *               not matter; not to be shared with a concurrent call.
+ * Other arguments, results and rules as for fa_bwd. No dropout variant.
+ */
+size_t fa_bwd_fused_workspace_bytes(int B, int H, int N, int d);
+fa_status fa_bwd_fused(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv,
+                       void* workspace, size_t workspace_bytes,
+                       int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_bwd_fused with query and key lengths of their own (as fa_bwd_qk), a memory layout
+ * (as fa_bwd_ex) and an optional block mask (tile_mask NULL, or as fa_bwd_blocksparse
+ * with causal = 0, Nq = Nk and mask_block = 128; else FA_ERR_UNSUPPORTED). The
+ * workspace holds per-query rows: fa_bwd_fused_workspace_bytes(B, H, Nq, d).
+ */
+fa_status fa_bwd_fused_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes,
+                          const uint8_t* tile_mask, int mask_block,
+                          int B, int H, int Nq, int Nk, int d, int layout, int causal, float scale,
+                          void* stream);
+
+/*
+ * The three launches that make up fa_bwd_fused (tile_mask NULL) or its block-sparse
+ * form, for callers that schedule or time them separately; same workspace for all
+ * three, in this order on one stream:
+ *   fa_bwd_fused_preprocess : the row arrays of fa_bwd_preprocess, and the fp32 dQ
+ *                             accumulator set to zero.
+ *   fa_bwd_fused_main       : dk and dv written; dq's shares added into the
+ *                             accumulator (mask rules as fa_bwd_dkdv).
+ *   fa_bwd_fused_dq         : dq [B,H,N,d] bf16 = bf16(scale * accumulator).
+ */
+fa_status fa_bwd_fused_preprocess(const void* o, const void* dO, const float* lse, void* workspace,
+                                  size_t workspace_bytes, int B, int H, int N, int d, void* stream);
+fa_status fa_bwd_fused_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes,
+                            const uint8_t* tile_mask, int mask_block,
+                            int B, int H, int N, int d, int causal, float scale, void* stream);
+fa_status fa_bwd_fused_dq(void* dq, const void* workspace, size_t workspace_bytes,
+                          int B, int H, int N, int d, float scale, void* stream);
+
+/*
  * Backward without caller-provided scratch (no counterpart on the pages: this is
  * an interface convenience, not part of the method).
  *
