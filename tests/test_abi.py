@@ -25,7 +25,8 @@ def test_exports_every_declared_symbol(L):
             "fa_status_string", "fa_device_status", "fa_version", "fa_bwd_preprocess", "fa_bwd_dkdv",
             "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_wait_timeout",
             "fa_debug_stall_producer", "fa_fwd_dropout", "fa_bwd_dropout", "fa_merge_partial",
-            "fa_accumulate_bf16", "fa_to_bf16"} <= set(names)
+            "fa_accumulate_bf16", "fa_to_bf16", "fa_bwd_fused_workspace_bytes", "fa_bwd_fused", "fa_bwd_fused_ex",
+            "fa_bwd_fused_preprocess", "fa_bwd_fused_main", "fa_bwd_fused_dq"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True,
                          check=True).stdout
     defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -118,6 +119,46 @@ def test_workspace_bytes(L):
         assert L.fa_bwd_workspace_bytes(B, H, N, d) == 2 * up(rows * 4)
     assert L.fa_bwd_workspace_bytes(0, 1, 128, 64) == 0
     assert L.fa_bwd_workspace_bytes(1, 1, -128, 64) == 0
+
+
+def test_fused_workspace_bytes(L):
+    """Row arrays of the deterministic backward, then the fp32 dQ accumulator
+    [B*H, Npad, 64 or 128] (d = 96 and 128 share the 128-column width)."""
+    up = lambda x: (x + 255) // 256 * 256
+    for (B, H, N, d) in ((1, 1, 128, 64), (8, 16, 2048, 64), (2, 16, 8192, 128), (2, 3, 130, 96), (1, 1, 1, 128)):
+        rows = B * H * ((N + 127) // 128 * 128)
+        dk = 64 if d == 64 else 128
+        assert L.fa_bwd_fused_workspace_bytes(B, H, N, d) == 2 * up(rows * 4) + up(rows * dk * 4)
+    assert L.fa_bwd_fused_workspace_bytes(0, 1, 128, 64) == 0
+
+
+def test_fused_argument_checks(L):
+    need = L.fa_bwd_fused_workspace_bytes(1, 1, 128, 64)
+    det = L.fa_bwd_workspace_bytes(1, 1, 128, 64)
+    f = lambda ws=A, wsb=need, mask=None, mb=128, causal=0, Nq=128, Nk=128, d=64, layout=0, dq=A, scale=0.1: \
+        L.fa_bwd_fused_ex(A, A, A, A, A, A, dq, A, A, ws, wsb, mask, mb, 1, 1, Nq, Nk, d, layout, causal, scale, None)
+    assert f(wsb=det) == WORKSPACE  # the deterministic path's workspace is too small here
+    assert f(ws=None) == INVALID and f(ws=A + 16) == ALIGN  # workspace 256-byte aligned
+    assert f(dq=None) == INVALID and f(dq=A + 2) == ALIGN
+    assert f(mask=A, causal=1) == UNSUPPORTED  # block mask with the causal flag
+    assert f(mask=A, mb=64) == UNSUPPORTED
+    assert f(mask=A, Nk=256) == UNSUPPORTED  # block mask needs Nq = Nk
+    assert f(d=80) == UNSUPPORTED and f(Nq=0) == INVALID and f(layout=5) == INVALID
+    assert f(scale=float("nan")) == INVALID
+    g = L.fa_bwd_fused
+    assert g(A, A, A, A, A, A, A, A, A, A, det, 1, 1, 128, 64, 0, 0.1, None) == WORKSPACE
+    pre = L.fa_bwd_fused_preprocess
+    assert pre(A, A, A, A, det, 1, 1, 128, 64, None) == WORKSPACE
+    assert pre(A, A, A, None, need, 1, 1, 128, 64, None) == INVALID
+    main = L.fa_bwd_fused_main
+    assert main(A, A, A, A, A, A, A, det, None, 128, 1, 1, 128, 64, 0, 0.1, None) == WORKSPACE
+    assert main(A, A, A, A, None, A, A, need, None, 128, 1, 1, 128, 64, 0, 0.1, None) == INVALID
+    conv = L.fa_bwd_fused_dq
+    assert conv(A, A, det, 1, 1, 128, 64, 0.1, None) == WORKSPACE
+    assert conv(None, A, need, 1, 1, 128, 64, 0.1, None) == INVALID
+    assert conv(A, A, need, 1, 1, 128, 64, float("inf"), None) == INVALID
+    if NO_GPU:  # valid arguments get as far as the first CUDA call, as a forward does
+        assert f() == _fwd(L)
 
 
 def test_dropout_argument_checks(L):
