@@ -15,6 +15,7 @@
 #include "fa_bwd.cuh"
 #include "fa_bwd_fused.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd256.cuh"
 
 namespace {
 
@@ -41,7 +42,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 fa_status check_sizes(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 96 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   // Padded rows (N rounded up to whole 128-row tiles) index the backward's row arrays.
   const long long rows = static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128 * 128);
   if (rows > INT_MAX || static_cast<long long>(B) * H > INT_MAX / 2) return FA_ERR_UNSUPPORTED;
@@ -181,6 +182,23 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <bool CAUSAL, bool SPARSE, bool XQK = false>
+fa_status launch_fwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
+                        cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  auto kernel = fa::fa_fwd256_kernel<CAUSAL, SPARSE, XQK>;
+  constexpr int smem = fa::Fwd256Cfg::kSmemBytes;
+  if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  int dev, sms = 0;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return FA_ERR_CUDA;
+  const unsigned grid = unsigned(p.n_items < sms ? p.n_items : sms);  // persistent: one CTA per SM
+  kernel<<<grid, fa::Fwd256Cfg::kThreads, smem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 // drop: dropout settings, or nullptr (dropout needs d 64 or 128, N_q = N_k and no tile mask).
 fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
                      int B, int H, int N, int Nk, int d, int layout, int causal, float scale, void* stream,
@@ -192,7 +210,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
-  if (drop != nullptr && (mask != nullptr || Nk != N || d == 96)) return FA_ERR_UNSUPPORTED;
+  if (drop != nullptr && (mask != nullptr || Nk != N || d == 96 || d == 256)) return FA_ERR_UNSUPPORTED;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
   int* status;
@@ -221,6 +239,14 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 256) {  // one Q tile per work item
+    p.n_qblocks = p.n_tiles;
+    p.n_items = p.n_tiles * BH;
+    if (mask) return launch_fwd256<false, true>(mq, mk, mv, p, st);
+    if (causal && Nk != N) return launch_fwd256<true, false, true>(mq, mk, mv, p, st);
+    if (causal) return launch_fwd256<true, false>(mq, mk, mv, p, st);
+    return launch_fwd256<false, false>(mq, mk, mv, p, st);
+  }
   if (drop) {
     fa::FwdParamsDrop pd;
     static_cast<fa::FwdParams&>(pd) = p;
@@ -320,6 +346,7 @@ fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d,
   if (ws == nullptr) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FA_ERR_ALIGNMENT;
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
+  if (d == 256) return FA_ERR_UNSUPPORTED;  // head dim 256: forward only
   if (ws_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
   a->BH = B * H;
   a->Npad = (N + 127) / 128 * 128;

@@ -67,7 +67,9 @@ def test_fwd_argument_checks(L):
     if NO_GPU:
         assert _fwd(L, d=96) == _fwd(L)  # head dim 96 runs on the 128-wide kernels
     assert _fwd(L, d=80) == UNSUPPORTED
-    assert _fwd(L, d=256) == UNSUPPORTED
+    if NO_GPU:
+        assert _fwd(L, d=256) == _fwd(L)  # head dim 256 has a forward kernel of its own
+    assert _fwd(L, d=192) == UNSUPPORTED and _fwd(L, d=512) == UNSUPPORTED
     # Any N >= 1 passes validation (the last 128-row tile may be partial): such a call
     # gets as far as a valid one, which on a machine without a GPU is FA_ERR_CUDA.
     if NO_GPU:
