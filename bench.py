@@ -176,7 +176,7 @@ def peaks():
 
 # The files the profiled attention kernels and their launches are compiled from: a
 # committed ncu figure stays valid while none of them changes.
-KERNEL_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_bwd_fused.cuh", "fa_dropout.cuh", "fa_fwd.cuh", "fa_fwd256.cuh", "fa_ptx.cuh")
+KERNEL_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_bwd_fused.cuh", "fa_bwd256.cuh", "fa_dropout.cuh", "fa_fwd.cuh", "fa_fwd256.cuh", "fa_ptx.cuh")
 
 
 def kernel_source_hash() -> str:

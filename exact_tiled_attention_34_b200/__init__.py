@@ -268,15 +268,26 @@ def _bwd_fused(q, k, v, o, lse, do, causal, scale, workspace, grads, layout, til
     return dq, dk, dv
 
 
+def _deterministic(deterministic, d):
+    """The backward to use: True (two-kernel, bit-reproducible) unless asked otherwise;
+    head dim 256 has only the fused backward."""
+    if deterministic is None:
+        return d != 256
+    if deterministic and d == 256:
+        raise ValueError("head dim 256 has only the fused backward (deterministic=False)")
+    return bool(deterministic)
+
+
 def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None, grads=None,
-             layout: str = "bhnd", deterministic: bool = True):
+             layout: str = "bhnd", deterministic=None):
     """Gradients (dq, dk, dv) of sum(O * dO) given the forward's o and lse.
 
-    deterministic=True: the two-kernel backward (bit-reproducible). False: the fused
+    deterministic=True (the default for head dims 64, 96, 128): the two-kernel backward
+    (bit-reproducible). False (the default, and only choice, at head dim 256): the fused
     single kernel (five products per tile pair instead of seven; dq accumulated in fp32
     in an order that varies from run to run)."""
     import torch
-    if not deterministic:
+    if not _deterministic(deterministic, q.shape[-1]):
         return _bwd_fused(q, k, v, o, lse, do, causal, scale, workspace, grads, layout, None, 128)
     workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout)
     B, H, N, Nk, d = _dims(q, k, layout)
@@ -318,11 +329,11 @@ def backward_dropout(q, k, v, o, lse, do, p: float, seed: int, offset: int = 0, 
 
 
 def backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None, mask_block: int = 128, workspace=None,
-                         grads=None, deterministic: bool = True):
+                         grads=None, deterministic=None):
     """Block-sparse backward (same mask as the forward); deterministic as for backward."""
     import torch
     _check_mask(tile_mask, q, mask_block)
-    if not deterministic:
+    if not _deterministic(deterministic, q.shape[-1]):
         return _bwd_fused(q, k, v, o, lse, do, False, scale, workspace, grads, "bhnd", tile_mask, mask_block)
     workspace, (dq, dk, dv) = _bwd_prep(q, k, v, o, lse, do, workspace, grads)
     B, H, N, d = q.shape

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libfa.so")
 
 SOURCES = ["fa_api.cu", "fa_merge.cu"]
-DEPS = ["fa_api.cu", "fa_merge.cu", "fa_fwd.cuh", "fa_fwd256.cuh", "fa_bwd.cuh", "fa_bwd_fused.cuh", "fa_dropout.cuh", "fa_ptx.cuh"]
+DEPS = ["fa_api.cu", "fa_merge.cu", "fa_fwd.cuh", "fa_fwd256.cuh", "fa_bwd.cuh", "fa_bwd_fused.cuh", "fa_bwd256.cuh", "fa_dropout.cuh", "fa_ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

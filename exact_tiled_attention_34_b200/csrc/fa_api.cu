@@ -14,6 +14,7 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_bwd_fused.cuh"
+#include "fa_bwd256.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd256.cuh"
 
@@ -341,12 +342,13 @@ struct BwdArgs {
 };
 
 // Checks shared by the backward stages; fills the workspace views.
-fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a) {
+// allow256: head dim 256 has only the fused backward (fa_bwd_fused*).
+fa_status bwd_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a, bool allow256 = false) {
   fa_status s;
   if (ws == nullptr) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FA_ERR_ALIGNMENT;
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
-  if (d == 256) return FA_ERR_UNSUPPORTED;  // head dim 256: forward only
+  if (d == 256 && !allow256) return FA_ERR_UNSUPPORTED;
   if (ws_bytes < bwd_ws_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
   a->BH = B * H;
   a->Npad = (N + 127) / 128 * 128;
@@ -363,15 +365,18 @@ fa_status bwd_pre(const void* o, const void* dO, const float* lse, void* ws, siz
   const int bnhd = layout == FA_LAYOUT_BNHD ? 1 : 0;
   if ((s = check_ptrs({o, dO, lse})) != FA_OK) return s;
   BwdArgs a;
-  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a)) != FA_OK) return s;
+  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, &a, dqacc != nullptr)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long threads = static_cast<long long>(a.rows) * (d == 64 ? 8 : 16);  // D / 8 per row
+  const long long threads = static_cast<long long>(a.rows) * (d == 64 ? 8 : (d == 256 ? 32 : 16));  // D / 8 per row
   const unsigned grid = unsigned((threads + 255) / 256);
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   const long long rows = static_cast<long long>(a.rows);
   if (d == 64)
     fa::fa_bwd_pre_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows, dqacc);
+  else if (d == 256)
+    fa::fa_bwd_pre_kernel<256><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows,
+                                                     dqacc);
   else  // 96 or 128 (16 threads per row)
     fa::fa_bwd_pre_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, a.Drow, a.lse2, N, a.Npad, d, H, bnhd, rows,
                                                      dqacc);
@@ -687,7 +692,7 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
 // dQ reduced in fp32 into the workspace and converted to bf16 by a last launch.
 namespace {
 
-int dq_width(int d) { return d == 64 ? 64 : 128; }  // columns of the fp32 dQ accumulator
+int dq_width(int d) { return d == 64 ? 64 : (d == 256 ? 256 : 128); }  // columns of the fp32 dQ accumulator
 
 // Workspace: the two row arrays of the deterministic backward, then the fp32 dQ
 // accumulator [B*H, Npad, 64 or 128], 256-byte aligned.
@@ -703,16 +708,16 @@ float* fused_dqacc(const void* ws, int B, int H, int N, int d) {
 
 fa_status fused_check(const void* ws, size_t ws_bytes, int B, int H, int N, int d, BwdArgs* a) {
   fa_status s;
-  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, a)) != FA_OK) return s;
+  if ((s = bwd_check(ws, ws_bytes, B, H, N, d, a, true)) != FA_OK) return s;
   return ws_bytes < fused_ws_bytes(B, H, N, d) ? FA_ERR_WORKSPACE : FA_OK;
 }
 
 // The fp32 accumulator [BH, Npad, Dk] as a 3-D tensor (column, row, batch*head) for
 // 32 x 32 reduce-add boxes with 128-byte swizzle (a box row is 32 fp32 = 128 bytes).
-fa_status make_acc_map(CUtensorMap* m, const float* base, int BH, int Npad, int Dk) {
+fa_status make_acc_map(CUtensorMap* m, const float* base, int BH, int Npad, int Dk, int box_rows = 32) {
   cuuint64_t dims[3] = {cuuint64_t(Dk), cuuint64_t(Npad), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(Dk) * 4, cuuint64_t(Npad) * cuuint64_t(Dk) * 4};
-  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t box[3] = {32, cuuint32_t(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -747,6 +752,32 @@ fa_status launch_fused(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <bool CAUSAL, bool SPARSE, bool XQK = false>
+fa_status launch_bwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                        const CUtensorMap& macc, const fa::BwdParams& p, cudaStream_t stream) {
+  static std::once_flag flags[kMaxDevices];
+  static cudaError_t errs[kMaxDevices];
+  static int regs[kMaxDevices];
+  auto kernel = fa::fa_bwd256_kernel<CAUSAL, SPARSE, XQK>;
+  constexpr int smem = fa::Bwd256Cfg::kSmemBytes;
+  if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
+  int dev;
+  if (current_device(&dev) != FA_OK) return FA_ERR_CUDA;
+  if (regs[dev] == 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+    regs[dev] = attr.numRegs;
+  }
+  if (regs[dev] * fa::kBwdThreads < fa::kFusedRegsNeeded) return FA_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return FA_ERR_CUDA;
+  unsigned grid = 2u * unsigned(p.n_ktiles) * unsigned(p.BH);  // (key tile, column half, batch*head) items
+  if (grid > unsigned(sms)) grid = unsigned(sms);
+  kernel<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, macc, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 // D and -lse log2 e rows, and the zeroed dQ accumulator.
 fa_status fused_pre(const void* o, const void* dO, const float* lse, void* ws, size_t ws_bytes, int B, int H, int N,
                     int d, int layout, void* stream) {
@@ -776,11 +807,15 @@ fa_status fused_main(const void* q, const void* k, const void* v, const void* dO
   int* status;
   if ((s = device_status_ptr(&status)) != FA_OK) return s;
   CUtensorMap mq, mk, mv, mdo, macc;
-  if ((s = make_map(&mq, q, B, H, N, d, bnhd, 128)) != FA_OK) return s;
+  // Head dim 256 visits queries in 64-row sub-tiles and reduces dQ in 32 x 16 boxes.
+  const int qrows = d == 256 ? 64 : 128;
+  if ((s = make_map(&mq, q, B, H, N, d, bnhd, qrows)) != FA_OK) return s;
   if ((s = make_map(&mk, k, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
   if ((s = make_map(&mv, v, B, H, Nk, d, bnhd, 128)) != FA_OK) return s;
-  if ((s = make_map(&mdo, dO, B, H, N, d, bnhd, 128)) != FA_OK) return s;
-  if ((s = make_acc_map(&macc, fused_dqacc(ws, B, H, N, d), a.BH, a.Npad, dq_width(d))) != FA_OK) return s;
+  if ((s = make_map(&mdo, dO, B, H, N, d, bnhd, qrows)) != FA_OK) return s;
+  if ((s = make_acc_map(&macc, fused_dqacc(ws, B, H, N, d), a.BH, a.Npad, dq_width(d), d == 256 ? 16 : 32)) !=
+      FA_OK)
+    return s;
   fa::BwdParams p;
   p.lse2 = a.lse2;
   p.Drow = a.Drow;
@@ -802,6 +837,12 @@ fa_status fused_main(const void* q, const void* k, const void* v, const void* dO
   p.ds = d;
   p.scale = scale;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 256) {
+    if (mask) return launch_bwd256<false, true>(mq, mk, mv, mdo, macc, p, st);
+    if (causal && Nk != N) return launch_bwd256<true, false, true>(mq, mk, mv, mdo, macc, p, st);
+    if (causal) return launch_bwd256<true, false>(mq, mk, mv, mdo, macc, p, st);
+    return launch_bwd256<false, false>(mq, mk, mv, mdo, macc, p, st);
+  }
   if (mask)
     return d == 64 ? launch_fused<64, false, true>(mq, mk, mv, mdo, macc, p, st)
                    : launch_fused<128, false, true>(mq, mk, mv, mdo, macc, p, st);
@@ -835,6 +876,8 @@ fa_status fused_dq(void* dq, const void* ws, size_t ws_bytes, int B, int H, int 
   const int bnhd = layout == FA_LAYOUT_BNHD ? 1 : 0;
   if (Dk == 64)
     fa::fa_dq_convert_kernel<64><<<grid, 256, 0, st>>>(acc, out, N, a.Npad, d, H, bnhd, rows, scale);
+  else if (Dk == 256)
+    fa::fa_dq_convert_kernel<256><<<grid, 256, 0, st>>>(acc, out, N, a.Npad, d, H, bnhd, rows, scale);
   else
     fa::fa_dq_convert_kernel<128><<<grid, 256, 0, st>>>(acc, out, N, a.Npad, d, H, bnhd, rows, scale);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
