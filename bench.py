@@ -320,7 +320,8 @@ def run_ours(args, wl_name, wl):
     for (_, _, dens) in wl["variants"]:
         if dens is not None:
             masks[dens] = make_tile_mask(-(-N // 128), seed=0, density=dens).to(dev)
-    ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    fused = args.backward == "fused"
+    ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d, deterministic=not fused), dtype=torch.uint8, device=dev)
     outs = {}
     for (label, _, _) in wl["variants"]:
         outs[label] = dict(o=torch.empty_like(t["q"]), lse=torch.empty((B, H, N), dtype=torch.float32, device=dev),
@@ -337,7 +338,9 @@ def run_ours(args, wl_name, wl):
         step_flops += 3.5 * f
 
     def one_step(ev=None):
-        # ev: dict label -> 5 events [start, after fwd, after pre, after dK/dV, after dQ]
+        # ev: dict label -> 5 events [start, after fwd, after pre, after main, after dQ]
+        # main: the fused kernel (dK, dV, dQ shares) or the dK/dV kernel; dQ: the
+        # accumulator's conversion or the dQ kernel.
         for (label, causal, _) in wl["variants"]:
             k = kinds[label]
             x = outs[label]
@@ -350,14 +353,25 @@ def run_ours(args, wl_name, wl):
                 fa.forward_blocksparse(t["q"], t["k"], t["v"], k["mask"], scale=sc, out=x["o"], lse=x["lse"])
             if e:
                 e[1].record(stream)
-            fa.bwd_preprocess(x["o"], t["do"], x["lse"], ws)
+            if fused:
+                fa.bwd_fused_preprocess(x["o"], t["do"], x["lse"], ws)
+            else:
+                fa.bwd_preprocess(x["o"], t["do"], x["lse"], ws)
             if e:
                 e[2].record(stream)
-            fa.bwd_dkdv(t["q"], t["k"], t["v"], t["do"], x["dk"], x["dv"], ws, causal=causal, scale=sc,
-                        tile_mask=k["mask"])
+            if fused:
+                fa.bwd_fused_main(t["q"], t["k"], t["v"], t["do"], x["dk"], x["dv"], ws, causal=causal, scale=sc,
+                                  tile_mask=k["mask"])
+            else:
+                fa.bwd_dkdv(t["q"], t["k"], t["v"], t["do"], x["dk"], x["dv"], ws, causal=causal, scale=sc,
+                            tile_mask=k["mask"])
             if e:
                 e[3].record(stream)
-            fa.bwd_dq(t["q"], t["k"], t["v"], t["do"], x["dq"], ws, causal=causal, scale=sc, tile_mask=k["mask"])
+            if fused:
+                fa.bwd_fused_dq(x["dq"], ws, scale=sc)
+            else:
+                fa.bwd_dq(t["q"], t["k"], t["v"], t["do"], x["dq"], ws, causal=causal, scale=sc,
+                          tile_mask=k["mask"])
             if e:
                 e[4].record(stream)
 
@@ -390,7 +404,7 @@ def run_ours(args, wl_name, wl):
         raise SystemExit(f"device status {st} (site {dt}) in the timed region")
 
     # per-kernel and per-step device times (ms)
-    per = {label: dict(fwd=0.0, pre=0.0, dkdv=0.0, dq=0.0) for (label, _, _) in wl["variants"]}
+    per = {label: dict(fwd=0.0, pre=0.0, main=0.0, dq=0.0) for (label, _, _) in wl["variants"]}
     step_ms = []
     for s in range(args.steps):
         tot = 0.0
@@ -399,7 +413,7 @@ def run_ours(args, wl_name, wl):
             a = [e[i].elapsed_time(e[i + 1]) for i in range(4)]
             per[label]["fwd"] += a[0]
             per[label]["pre"] += a[1]
-            per[label]["dkdv"] += a[2]
+            per[label]["main"] += a[2]
             per[label]["dq"] += a[3]
             tot += sum(a)
         step_ms.append(tot)
@@ -413,14 +427,14 @@ def run_ours(args, wl_name, wl):
     peak_label = ("sustained" if sustained else "burst") + f" bf16, {pk_kind}"
 
     breakdown = {}
-    dkdv_flops, dkdv_ms = 0.0, 0.0
+    main_flops, main_ms = 0.0, 0.0
     for (label, _, _) in wl["variants"]:
         k = kinds[label]
         p = {kk: v / K for kk, v in per[label].items()}
-        bwd_ms = p["pre"] + p["dkdv"] + p["dq"]
+        bwd_ms = p["pre"] + p["main"] + p["dq"]
         breakdown[label] = {
             "fwd_ms": round(p["fwd"], 4), "bwd_ms": round(bwd_ms, 4),
-            "bwd_pre_ms": round(p["pre"], 4), "bwd_dkdv_ms": round(p["dkdv"], 4), "bwd_dq_ms": round(p["dq"], 4),
+            "bwd_pre_ms": round(p["pre"], 4), "bwd_main_ms": round(p["main"], 4), "bwd_dq_ms": round(p["dq"], 4),
             "fwd_tflops": round(k["fwd"] / (p["fwd"] * 1e-3) / 1e12, 2),
             "bwd_tflops": round(k["bwd"] / (bwd_ms * 1e-3) / 1e12, 2),
             "fwd_bwd_tflops": round(3.5 * k["fwd"] / ((p["fwd"] + bwd_ms) * 1e-3) / 1e12, 2),
@@ -429,13 +443,17 @@ def run_ours(args, wl_name, wl):
             "fwd_pct_spec_peak": round(100 * k["fwd"] / (p["fwd"] * 1e-3) / 1e12 / SPEC_BF16_TFLOPS, 1),
             "bwd_pct_spec_peak": round(100 * k["bwd"] / (bwd_ms * 1e-3) / 1e12 / SPEC_BF16_TFLOPS, 1),
         }
-        # dK/dV kernel: S^T, dP^T, dV, dK = four N x N x d products = 2x the forward count
-        dkdv_flops += 2.0 * k["fwd"]
-        dkdv_ms += p["dkdv"]
-    achieved = dkdv_flops / (dkdv_ms * 1e-3) / 1e12
-    roofline = {"kernel": "fa_bwd_dkdv_kernel (backward dK/dV, 4 products per tile pair)", "bound": "tensor",
-                "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_label, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("fa_bwd_dkdv_kernel", wl_name)}
+        # The step's dominant kernel. Fused: S^T, dP^T, dV, dK, dQ = five N x N x d products =
+        # the whole backward's 2.5x the forward count. dK/dV kernel: four = 2x.
+        main_flops += (2.5 if fused else 2.0) * k["fwd"]
+        main_ms += p["main"]
+    achieved = main_flops / (main_ms * 1e-3) / 1e12
+    main_kernel = "fa_bwd_fused_kernel" if fused else "fa_bwd_dkdv_kernel"
+    roofline = {"kernel": main_kernel + (" (backward dK, dV and dQ shares, 5 products per tile pair)" if fused
+                                         else " (backward dK/dV, 4 products per tile pair)"),
+                "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_label,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": profiled_traffic(main_kernel, wl_name)}
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e_steps = max(3, min(K, 10))
@@ -451,11 +469,12 @@ def run_ours(args, wl_name, wl):
             k = kinds[label]
             if k["mask"] is None:
                 o, lse = fa.forward(x["q"], x["k"], x["v"], causal=causal, scale=sc)
-                g = fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, scale=sc, workspace=ws)
+                g = fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, scale=sc, workspace=ws,
+                                deterministic=not fused)
             else:
                 o, lse = fa.forward_blocksparse(x["q"], x["k"], x["v"], k["mask"], scale=sc)
                 g = fa.backward_blocksparse(x["q"], x["k"], x["v"], o, lse, x["do"], k["mask"], scale=sc,
-                                            workspace=ws)
+                                            workspace=ws, deterministic=not fused)
             for n, v in zip(("o", "lse", "dq", "dk", "dv"), (o, lse) + tuple(g)):
                 res_host[label][n].copy_(v, non_blocking=True)
 
@@ -480,7 +499,11 @@ def run_ours(args, wl_name, wl):
         "data": "synthetic (seeded N(0,1) inputs rounded to bf16; per-rank seeds)",
         "config": {"workload": wl_name, "B": B, "H": H, "N": N, "d": d,
                    "variants": [v[0] for v in wl["variants"]],
-                   "step": "per variant: forward, backward pre-pass, backward dK/dV, backward dQ",
+                   "step": ("per variant: forward, backward pre-pass (D, lse rows, dQ accumulator zeroed), fused "
+                            "backward kernel (dK, dV, dQ shares reduced in fp32), dQ conversion" if fused else
+                            "per variant: forward, backward pre-pass, backward dK/dV kernel, backward dQ kernel"),
+                   "backward": ("fused: one kernel, dQ reduced in fp32 by TMA reduce-add (run-to-run order varies)"
+                                if fused else "deterministic: dK/dV kernel + dQ kernel (bit-reproducible)"),
                    "l2": "flushed before every timed step (256 MiB write, outside the step events)",
                    "parallelism": f"replicas x{world} (independent (batch, head) shards, no collective)"},
         "pct_of_peak": round(100 * value / world / peak, 2),
@@ -520,8 +543,8 @@ def run_table(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     names = ["pr1", "b8h16n2048d64", "b2h16n8192d128_causal", "b1h16n16384d64_sparse", "b8h16n2000d64_ragged",
-             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal", "b4h16n4096d96", "b8h16n2048d64_dropout",
-             "b2h16n8192d128_causal_dropout"]
+             "b2h16n8000d128_ragged_causal", "b4h16q512k8192d128_causal", "b4h16n4096d96", "b2h8n8192d256",
+             "b8h16n2048d64_dropout", "b2h16n8192d128_causal_dropout"]
     names += [f"sweep_N{N}_d{d}{c}" for d in SWEEP_D for N in SWEEP_N for c in ("", "_causal")]
     if args.only:
         names = [n for n in names if any(o in n for o in args.only.split(","))]
@@ -536,7 +559,9 @@ def run_table(args):
         if Nk != N:  # keys and values of their own length
             kv = make_qkv(B, H, Nk, d, seed=1, with_do=False)
             t["k"], t["v"] = kv["k"].to(dev), kv["v"].to(dev)
-        ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+        det_ok = d != 256  # head dim 256 has only the fused backward
+        ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, min(d, 128)), dtype=torch.uint8, device=dev)
+        ws_f = torch.empty(fa.bwd_workspace_bytes(B, H, N, d, deterministic=False), dtype=torch.uint8, device=dev)
         o = torch.empty_like(t["q"])
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
@@ -586,7 +611,27 @@ def run_table(args):
             row = {"workload": name, "variant": label, "B": B, "H": H, "N": N, "d": d, "kept": round(kept, 4),
                    "fwd_ms": round(t_f, 4), "fwd_tflops": round(F / t_f / 1e9, 1),
                    "fwd_pct_peak": round(100 * F / t_f / 1e9 / pk["bf16_tflops"], 1)}
-            if Nk != N or pdrop:
+            if name != "pr1" and not pdrop:
+                # the fused backward (one kernel; dQ reduced in fp32), whole and its main kernel
+                def fbwd():
+                    if mask is None:
+                        fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=causal, scale=sc, workspace=ws_f,
+                                    grads=(dq, dk, dv), deterministic=False)
+                    else:
+                        fa.backward_blocksparse(t["q"], t["k"], t["v"], o, lse, t["do"], mask, scale=sc,
+                                                workspace=ws_f, grads=(dq, dk, dv), deterministic=False)
+                t_fb = timed([fbwd])
+                row.update({"fused_bwd_ms": round(t_fb, 4), "fused_bwd_tflops": round(2.5 * F / t_fb / 1e9, 1),
+                            "fused_bwd_pct_peak": round(100 * 2.5 * F / t_fb / 1e9 / pk["bf16_tflops"], 1),
+                            "fused_fwd_bwd_tflops": round(3.5 * F / (t_f + t_fb) / 1e9, 1)})
+                if Nk == N:
+                    fa.bwd_fused_preprocess(o, t["do"], lse, ws_f)
+                    t_fm = timed([lambda: fa.bwd_fused_main(t["q"], t["k"], t["v"], t["do"], dk, dv, ws_f,
+                                                            causal=causal, scale=sc, tile_mask=mask)])
+                    row.update({"fused_main_ms": round(t_fm, 4), "fused_main_tflops": round(2.5 * F / t_fm / 1e9, 1)})
+            if not det_ok:
+                pass
+            elif Nk != N or pdrop:
                 # The staged calls are for Nq = Nk without dropout; time the whole backward.
                 def bwd_all():
                     if pdrop:
@@ -615,11 +660,13 @@ def run_table(args):
             row["fwd_pct_spec_peak"] = round(100 * F / t_f / 1e9 / SPEC_BF16_TFLOPS, 1)
             if "bwd_ms" in row:
                 row["bwd_pct_spec_peak"] = round(100 * 2.5 * F / row["bwd_ms"] / 1e9 / SPEC_BF16_TFLOPS, 1)
+            if "fused_bwd_ms" in row:
+                row["fused_bwd_pct_spec_peak"] = round(100 * 2.5 * F / row["fused_bwd_ms"] / 1e9 / SPEC_BF16_TFLOPS, 1)
             st, site = fa.device_status(dev)
             row["status"] = st
             row["peak"] = f'{pk["bf16_tflops"]} ({pk_kind}, burst)'
             print(json.dumps(row), flush=True)
-        del t, ws, o, lse, dq, dk, dv
+        del t, ws, ws_f, o, lse, dq, dk, dv
         torch.cuda.empty_cache()
     return 0
 
@@ -631,6 +678,8 @@ def build_parser():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="b2h16n8192d128_causal")
+    ap.add_argument("--backward", choices=("fused", "deterministic"), default="fused",
+                    help="fused: one kernel for dK, dV, dQ (dQ reduced in fp32); deterministic: two kernels")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--table", action="store_true", help="per-workload fwd/bwd times (JSON lines), not the contract line")

@@ -32,6 +32,8 @@ WORKLOADS = {
     "b4h16q512k8192d128_causal": dict(B=4, H=16, N=512, Nk=8192, d=128, causal=(True,), backward=True),
     # Head dim 96 (runs on the 128-wide kernels).
     "b4h16n4096d96": dict(B=4, H=16, N=4096, d=96, causal=(False, True), backward=True),
+    # Head dim 256 (kernels of its own; the fused backward only).
+    "b2h8n8192d256": dict(B=2, H=8, N=8192, d=256, causal=(False, True), backward=True),
     # Dropout on the probabilities (p = 0.1) on the shapes above.
     "b8h16n2048d64_dropout": dict(B=8, H=16, N=2048, d=64, causal=(False, True), backward=True, dropout_p=0.1),
     "b2h16n8192d128_causal_dropout": dict(B=2, H=16, N=8192, d=128, causal=(True,), backward=True,

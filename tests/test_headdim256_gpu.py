@@ -101,9 +101,101 @@ def test_long_sequence_sampled(cuda_device, causal):
                       sample_rows(N, n_random=32), what=f"d256 N{N} causal={causal}")
 
 
-def test_backward_not_built_for_256(cuda_device):
-    t = {k: x.to(cuda_device) for k, x in make_qkv(1, 1, 128, D, seed=2630).items()}
+# ------------------------------------------------------------------ backward (fused kernel)
+
+def _bwd_check(B, H, Nq, Nk, causal, dev, seed, mask=None, scale=None, heads=None):
+    a = make_qkv(B, H, Nq, D, seed=seed)
+    kv = a if Nk == Nq else make_qkv(B, H, Nk, D, seed=seed + 1000)
+    t = {"q": a["q"].to(dev), "do": a["do"].to(dev), "k": kv["k"].to(dev), "v": kv["v"].to(dev)}
+    sc = 1.0 / math.sqrt(D) if scale is None else scale
+    m = None if mask is None else mask.to(dev)
+    if m is None:
+        o, lse = fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc)
+    else:
+        o, lse = fa.forward_blocksparse(t["q"], t["k"], t["v"], m, scale=sc)
+    bufs = [_padded(shape, torch.bfloat16, dev, float("nan")) for shape in
+            ((B, H, Nq, D), (B, H, Nk, D), (B, H, Nk, D))]
+    grads = tuple(b[1] for b in bufs)
+    if m is None:
+        dq, dk, dv = fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=causal, scale=sc, grads=grads)
+    else:
+        dq, dk, dv = fa.backward_blocksparse(t["q"], t["k"], t["v"], o, lse, t["do"], m, scale=sc, grads=grads)
+    torch.cuda.synchronize()
+    assert fa.device_status() == (0, 0)
+    for (big, g) in bufs:
+        assert _tail_untouched(big, g.numel(), float("nan")), "gradient written past its end"
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for (b, h) in heads:
+        sl = lambda x: x[b:b + 1, h:h + 1].cpu()
+        ref = oracle.attn_bwd_ref(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["do"]), causal, sc,
+                                  None if mask is None else mask.numpy(), 128)
+        for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+            assert_grad_close(sl(g), ref[name], name, f"d256 bwd B{B} H{H} Nq{Nq} Nk{Nk} causal={causal} (b={b}, h={h})")
+    return t, (dq, dk, dv)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 300, 1000])
+def test_backward_lengths(cuda_device, N, causal):
+    _bwd_check(2, 2, N, N, causal, cuda_device, seed=2640 + N)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(1, 700), (77, 300), (300, 77), (256, 640)])
+def test_backward_cross_lengths(cuda_device, nq, nk, causal):
+    _, (dq, _, _) = _bwd_check(1, 2, nq, nk, causal, cuda_device, seed=2650 + nq)
+    if causal and nq > nk:
+        assert torch.all(dq[:, :, : nq - nk] == 0)
+
+
+@pytest.mark.parametrize("scale", [0.05, -0.2])
+def test_backward_scales(cuda_device, scale):
+    _bwd_check(1, 2, 384, 384, True, cuda_device, seed=2660, scale=scale)
+
+
+def test_backward_blocksparse(cuda_device):
+    mask = make_tile_mask(6, seed=23, density=0.4)
+    mask[2, :] = 0
+    mask[:, 4] = 0
+    mask[4, 4] = 0
+    _, (dq, dk, dv) = _bwd_check(1, 2, 768, 768, False, cuda_device, seed=2670, mask=mask)
+    assert torch.all(dq[:, :, 256:384] == 0)
+    assert torch.all(dk[:, :, 512:640] == 0) and torch.all(dv[:, :, 512:640] == 0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_many_items(cuda_device, causal):
+    """More (key tile, column half, head) items than SMs."""
+    _bwd_check(2, 48, 384, 384, causal, cuda_device, seed=2680)
+
+
+def test_backward_2048_full_heads(cuda_device):
+    _bwd_check(1, 4, 2048, 2048, True, cuda_device, seed=0, heads=[(0, 0), (0, 3)])
+
+
+def test_backward_bnhd_layout(cuda_device):
+    B, H, N = 1, 3, 300
+    t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, N, D, seed=2690).items()}
+    o, lse = fa.forward(t["q"], t["k"], t["v"], causal=True)
+    ref = fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=True)
+    tt = {k: x.transpose(1, 2).contiguous() for k, x in t.items()}
+    g = fa.backward(tt["q"], tt["k"], tt["v"], o.transpose(1, 2).contiguous(), lse, tt["do"], causal=True,
+                    layout="bnhd")
+    torch.cuda.synchronize()
+    for x, y in zip(g, ref):
+        assert float((x.transpose(1, 2).float() - y.float()).abs().max()) <= 2e-2 * float(y.float().abs().max())
+
+
+def test_backward_deterministic_path_is_not_offered(cuda_device):
+    """Head dim 256 has only the fused backward: asking for the deterministic one raises,
+    and the C entry point of the deterministic backward refuses the size."""
+    t = {k: x.to(cuda_device) for k, x in make_qkv(1, 1, 128, D, seed=2700).items()}
     o, lse = fa.forward(t["q"], t["k"], t["v"])
-    with pytest.raises(fa.FAError) as e:
-        fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"])
-    assert e.value.status == 2
+    with pytest.raises(ValueError):
+        fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], deterministic=True)
+    ws = torch.empty(fa.bwd_workspace_bytes(1, 1, 128, D), dtype=torch.uint8, device=cuda_device)
+    g = [torch.empty_like(t["q"]) for _ in range(3)]
+    st = fa.lib().fa_bwd(t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), o.data_ptr(), lse.data_ptr(),
+                         t["do"].data_ptr(), g[0].data_ptr(), g[1].data_ptr(), g[2].data_ptr(), ws.data_ptr(),
+                         ws.numel(), 1, 1, 128, D, 0, 0.0625, fa._stream_ptr(cuda_device))
+    assert st == 2
