@@ -42,15 +42,28 @@ struct FusedCfg {
   static constexpr int kBlockBytes = 128 * 128;  // one 64-column block of a 128-row bf16 tile
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kDoStages = (D == 128) ? 1 : 2;  // dO ring depth (shared memory is short at 128)
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kTileBytes;
-  static constexpr int kOffQ = kOffV + kTileBytes;                  // 2 stages
+  // K_j, V_j per item: at head dim 64 two stages, so that the next item's tiles load while
+  // this item's last query tiles run (the item boundary then costs little more than the
+  // dK/dV epilogue); at 128 one.
+  static constexpr int kKvStages = (D == 128) ? 1 : 2;
+  static constexpr int kOffK = 0;                                   // kKvStages stages
+  static constexpr int kOffV = kOffK + kKvStages * kTileBytes;      // kKvStages stages
+  static constexpr int kOffQ = kOffV + kKvStages * kTileBytes;      // 2 stages
   static constexpr int kOffDO = kOffQ + 2 * kTileBytes;             // kDoStages stages
   static constexpr int kOffDS = kOffDO + kDoStages * kTileBytes;    // dS bf16 128 x 128 / dQ stages
   static constexpr int kOffL = kOffDS + 32768;                      // -lse log2 e rows, 2 stages
   static constexpr int kOffDr = kOffL + 1024;                       // D rows, 2 stages
-  static constexpr int kOffBar = kOffDr + 1024;
-  static constexpr int kSmemBytes = kOffBar + 512 + 1024;           // barriers + alignment slack
+  // Head dim 128: a second dQ staging area (4 KB per compute warp), so that a warp's two
+  // 32-column boxes leave without waiting for the first copy to read its stage.
+  static constexpr int kStage2Bytes = (D == 128) ? 32768 : 0;
+  static constexpr int kOffStage2 = kOffDr + 1024;
+  static constexpr int kOffBar = kOffStage2 + kStage2Bytes;
+  // Barriers (well under 256 bytes), plus 1 KB of alignment slack at head dim 64. At head
+  // dim 128 there is no room for the slack: the kernel then requires the dynamic
+  // shared-memory base to be 1024-byte aligned (it is when, as here, the kernel declares
+  // no static shared memory) and returns with an error status if it is not.
+  static constexpr bool kAlignedBase = (D == 128);
+  static constexpr int kSmemBytes = kOffBar + 256 + (kAlignedBase ? 0 : 1024);
   static_assert(kSmemBytes <= 227 * 1024, "fused backward shared memory above the per-block limit");
   static constexpr uint32_t kTmDK = 0;
   static constexpr uint32_t kTmDV = D;
@@ -63,8 +76,8 @@ struct FusedCfg {
 };
 
 struct FusedBars {
-  uint64_t kv_full;
-  uint64_t kv_empty;     // every product of the item that reads K_j or V_j is done
+  uint64_t kv_full[2];
+  uint64_t kv_empty[2];  // every product of the item that reads K_j or V_j is done
   uint64_t q_full[2];    // Q_i and the row arrays of tile i
   uint64_t q_empty[2];
   uint64_t do_full[2];
@@ -86,8 +99,10 @@ struct FusedBars {
 enum FusedSite : int {
   kSiteFuKV = 301, kSiteFuQEmpty, kSiteFuDoEmpty, kSiteFuKvEmpty, kSiteFuQFull, kSiteFuDoFull, kSiteFuPReady,
   kSiteFuDsReady, kSiteFuDqTaken, kSiteFuAcc, kSiteFuSFull, kSiteFuDpFull, kSiteFuDqFull, kSiteFuRead,
-  kSiteFuDrain
+  kSiteFuDrain,
+  kSiteFuSmemAlign = 399  // reported with kStatusUnsupported: dynamic shared memory not 1024-aligned
 };
+constexpr int kStatusUnsupported = 2;  // == FA_ERR_UNSUPPORTED
 
 // dK += dS^T Q_i: A = dS^T from shared memory (K-major: key rows, query columns in
 // 64-wide blocks), B = Q_i (N-major), 8 steps of 16 queries.
@@ -129,8 +144,14 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
   using Cfg = FusedCfg<D>;
   constexpr int SD = Cfg::kDoStages;
+  constexpr int SKV = Cfg::kKvStages;
   const int off_ = XQK ? p.off : 0;
   extern __shared__ uint8_t smem_raw[];
+  if (Cfg::kAlignedBase && (smem_u32(smem_raw) & 1023u) != 0) {
+    // Every thread leaves before any barrier, copy or tensor-memory allocation.
+    if (threadIdx.x == 0 && atomicCAS(p.status, 0, kStatusUnsupported) == 0) atomicExch(p.status + 1, kSiteFuSmemAlign);
+    return;
+  }
   uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
   FusedBars* bars = reinterpret_cast<FusedBars*>(smem + Cfg::kOffBar);
   uint8_t* sK = smem + Cfg::kOffK;
@@ -146,9 +167,9 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   WaitCtl wc{&bars->abort, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->kv_full, 1);
-    mbar_init(&bars->kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
       mbar_init(&bars->do_full[s], 1);
@@ -194,11 +215,14 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int j = item.tile, bh = item.bh;
         const int ib = bh / p.H, ih = bh - ib * p.H;
         KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
-        if (kk > 0 && !mbar_wait(&bars->kv_empty, (kk - 1) & 1, wc, kSiteFuKvEmpty)) break;
-        mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kTileBytes);
+        const int kvs = kk % SKV;
+        if (kk >= SKV && !mbar_wait(&bars->kv_empty[kvs], ((kk / SKV) - 1) & 1, wc, kSiteFuKvEmpty)) break;
+        mbar_arrive_expect_tx(&bars->kv_full[kvs], 2 * Cfg::kTileBytes);
         for (int cb = 0; cb < D / 64; ++cb) {
-          tma_load_4d(sK + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full, cb * 64, j * 128, ih, ib);
-          tma_load_4d(sV + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full, cb * 64, j * 128, ih, ib);
+          tma_load_4d(sK + kvs * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_k, &bars->kv_full[kvs], cb * 64,
+                      j * 128, ih, ib);
+          tma_load_4d(sV + kvs * Cfg::kTileBytes + cb * Cfg::kBlockBytes, &tm_v, &bars->kv_full[kvs], cb * 64,
+                      j * 128, ih, ib);
         }
         ++nkv;
         for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
@@ -229,7 +253,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       // On abort, wait (bounded) for this thread's own copies still in flight.
       if (bars->abort) {
-        if (nkv > 0) mbar_wait_drain(&bars->kv_full, (nkv - 1) & 1, wc, kSiteFuDrain);
+        for (int x = (nkv > SKV ? nkv - SKV : 0); x < nkv; ++x)
+          mbar_wait_drain(&bars->kv_full[x % SKV], (x / SKV) & 1, wc, kSiteFuDrain);
         for (int x = (nq > 2 ? nq - 2 : 0); x < nq; ++x)
           mbar_wait_drain(&bars->q_full[x & 1], (x >> 1) & 1, wc, kSiteFuDrain);
         for (int x = (ndo > SD ? ndo - SD : 0); x < ndo; ++x)
@@ -243,17 +268,19 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ------------------------------------------------------------ MMA issuer
     regs_dec<kFusedRegsCtl>();
     if (lane == 0) {
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
+      const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO);
       const uint32_t aDS = smem_u32(sDS);
       bool ok = true;
       int it = 0;  // query tiles processed so far (continues across items)
       BwdItem item;
       for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
         KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
-        if (!mbar_wait(&bars->kv_full, kk & 1, wc, kSiteFuKV)) { ok = false; break; }
+        const int kvs = kk % SKV;
+        const uint32_t aK = smem_u32(sK) + kvs * Cfg::kTileBytes, aV = smem_u32(sV) + kvs * Cfg::kTileBytes;
+        if (!mbar_wait(&bars->kv_full[kvs], (kk / SKV) & 1, wc, kSiteFuKV)) { ok = false; break; }
         tc_fence_after();
         int i = sch.first();
-        if (i < 0) mma_commit(&bars->kv_empty);
+        if (i < 0) mma_commit(&bars->kv_empty[kvs]);
         if (i >= 0) {
           // The item's first S^T and dP^T.
           if (!mbar_wait(&bars->q_full[it & 1], (it >> 1) & 1, wc, kSiteFuQFull)) { ok = false; break; }
@@ -300,7 +327,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           mma_dq_ss<D>(tmem + Cfg::kTmDQ, aDS, aK);
           mma_commit(&bars->dq_full);
           mma_commit(&bars->q_empty[st]);
-          if (in < 0) mma_commit(&bars->kv_empty);  // every product reading K_j, V_j is issued
+          if (in < 0) mma_commit(&bars->kv_empty[kvs]);  // every product reading K_j, V_j is issued
           if (in >= 0) {
             if (Cfg::kDqInY && !mbar_wait(&bars->dq_taken, it & 1, wc, kSiteFuDqTaken)) { ok = false; break; }
             const int dn = (it + 1) % SD;
@@ -341,12 +368,13 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // h), and after dQ's product the staging area of its dQ boxes.
     uint8_t* my_ds = sDS + h * 16384 + r * 128;
     uint8_t* my_stage = sDS + h * 16384 + quarter * 4096;
+    uint8_t* my_stage2 = smem + Cfg::kOffStage2 + (h * 4 + quarter) * 4096;  // head dim 128 only
     bool ok = true;
     int it = 0;
     // dQ_t out of tensor memory into global dQacc rows [128 ti + 32 quarter, +32), columns
     // [h D/2, (h+1) D/2), in 32 x 32 fp32 boxes through the stage.
-    auto stage_box = [&](const uint32_t (&v)[32]) {
-      uint4* s4 = reinterpret_cast<uint4*>(my_stage);
+    auto stage_box = [&](const uint32_t (&v)[32], uint8_t* stage) {
+      uint4* s4 = reinterpret_cast<uint4*>(stage);
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         s4[lane * 8 + (c ^ (lane & 7))] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
@@ -363,16 +391,17 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if constexpr (D == 64) {
         tc_fence_before();
         mbar_arrive(&bars->dq_taken);
-        stage_box(v);
+        stage_box(v, my_stage);
         if (lane == 0) {
           tma_reduce_add_3d(&tm_dqacc, my_stage, x0, y0, bh);
           bulk_commit();
         }
       } else {
-        // Two 32-column boxes through the one 4 KB stage: the first is staged before
-        // the second leaves tensor memory, so that Y is released early (only 32 values
-        // are held in registers at a time).
-        stage_box(v);
+        // Two 32-column boxes through two 4 KB stages: the first is staged before the
+        // second leaves tensor memory, so that Y is released early (only 32 values are
+        // held in registers at a time), and neither copy is waited for here (the wait
+        // comes before this warp next writes dS, a phase later).
+        stage_box(v, my_stage);
         tmem_ld32(trow + Cfg::kTmDQ + h * (D / 2) + 32, v);
         tmem_wait_ld();
         tc_fence_before();
@@ -380,12 +409,10 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (lane == 0) {
           tma_reduce_add_3d(&tm_dqacc, my_stage, x0, y0, bh);
           bulk_commit();
-          bulk_wait_read0();  // the first box has left the stage
         }
-        __syncwarp();
-        stage_box(v);
+        stage_box(v, my_stage2);
         if (lane == 0) {
-          tma_reduce_add_3d(&tm_dqacc, my_stage, x0 + 32, y0, bh);
+          tma_reduce_add_3d(&tm_dqacc, my_stage2, x0 + 32, y0, bh);
           bulk_commit();
         }
       }
@@ -470,7 +497,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ds[t] = pack_bf16(v.x, v.y);
           }
         }
-        // The stage may still be read by this warp's last reduce-add copy.
+        // The stages may still be read by this warp's last reduce-add copies.
         if (lane == 0) bulk_wait_read0();
         __syncwarp();
         {

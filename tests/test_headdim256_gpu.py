@@ -10,7 +10,7 @@ import torch
 import exact_tiled_attention_34_b200 as fa
 import oracle
 from exact_tiled_attention_34_b200.inputs import make_qkv, make_tile_mask
-from tests.parity import assert_fwd_close, sample_rows, sampled_fwd_check, tol_o_sharp
+from tests.parity import assert_fwd_close, assert_grad_close, sample_rows, sampled_fwd_check, tol_o_sharp
 from tests.test_ragged_gpu import _padded, _tail_untouched
 
 pytestmark = pytest.mark.gpu
