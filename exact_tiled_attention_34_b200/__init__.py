@@ -28,7 +28,7 @@ __all__ = [
     "FAError", "lib", "lib_path", "exported_names", "forward", "forward_blocksparse", "backward",
     "backward_blocksparse", "bwd_workspace_bytes", "device_status", "STATUS", "bwd_preprocess", "bwd_dkdv",
     "bwd_dq", "bwd_fused_preprocess", "bwd_fused_main", "bwd_fused_dq", "attention", "attention_blocksparse", "forward_dropout", "backward_dropout", "merge_partial",
-    "accumulate_bf16", "to_bf16",
+    "accumulate_bf16", "to_bf16", "forward_merge", "bwd_fused_main_f32", "accumulate_f32",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +80,9 @@ _SIGS = {
     "fa_bwd_fused_preprocess": ([_vp] * 4 + [_sz] + [_i] * 4 + [_vp], _i),
     "fa_bwd_fused_main": ([_vp] * 7 + [_sz, _vp, _i] + [_i] * 5 + [_f, _vp], _i),
     "fa_bwd_fused_dq": ([_vp, _vp, _sz] + [_i] * 4 + [_f, _vp], _i),
+    "fa_fwd_merge": ([_vp] * 5 + [_i] * 5 + [_f, _vp], _i),
+    "fa_bwd_fused_main_f32": ([_vp] * 7 + [_sz] + [_i] * 5 + [_f, _vp], _i),
+    "fa_accumulate_f32": ([_vp, _vp, ctypes.c_longlong, _vp], _i),
     "fa_debug_exp2": ([_vp, _vp, _i, _i, _vp], _i),
     "fa_debug_wait_timeout": ([_i, _vp, _vp], _i),
     "fa_debug_stall_producer": ([_i, _i], _i),
@@ -490,6 +493,51 @@ def accumulate_bf16(acc, x, overwrite: bool = False):
         st = lib().fa_accumulate_bf16(acc.data_ptr(), x.data_ptr(), acc.numel(), int(bool(overwrite)),
                                       _stream_ptr(acc.device))
     _check(st, "fa_accumulate_bf16")
+
+
+def forward_merge(q, k, v, o_acc, lse_acc, causal: bool = False, scale=None):
+    """In place: (o_acc fp32 [B, H, N, d], lse_acc fp32 [B, H, N]) <- the running result
+    merged with the attention of q against this key block (k, v), in the kernel."""
+    import torch
+    _check_qkv(q, k, v)
+    if k.shape != q.shape:
+        raise ValueError("query and key blocks must have the same shape")
+    if o_acc.dtype != torch.float32 or tuple(o_acc.shape) != tuple(q.shape) or not o_acc.is_contiguous():
+        raise ValueError("o_acc must be a contiguous fp32 tensor of q's shape")
+    if lse_acc.dtype != torch.float32 or tuple(lse_acc.shape) != tuple(q.shape[:3]) or not lse_acc.is_contiguous():
+        raise ValueError("lse_acc must be a contiguous fp32 [B, H, N] tensor")
+    B, H, N, d = q.shape
+    with torch.cuda.device(q.device):
+        st = lib().fa_fwd_merge(q.data_ptr(), k.data_ptr(), v.data_ptr(), o_acc.data_ptr(), lse_acc.data_ptr(), B, H, N,
+                                d, int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_fwd_merge")
+
+
+def bwd_fused_main_f32(q, k, v, do, dk32, dv32, workspace, causal=False, scale=None):
+    """The fused backward's main kernel with fp32 dK, dV outputs (dQ's share added into the
+    workspace's accumulator, as bwd_fused_main)."""
+    import torch
+    B, H, N, d = q.shape
+    for t in (dk32, dv32):
+        if t.dtype != torch.float32 or tuple(t.shape) != tuple(k.shape) or not t.is_contiguous():
+            raise ValueError("dk32 and dv32 must be contiguous fp32 tensors of k's shape")
+    with torch.cuda.device(q.device):
+        st = lib().fa_bwd_fused_main_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk32.data_ptr(),
+                                         dv32.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, N, d,
+                                         int(bool(causal)), _scale(scale, d), _stream_ptr(q.device))
+    _check(st, "fa_bwd_fused_main_f32")
+
+
+def accumulate_f32(acc, x):
+    """In place: acc (fp32) += x (fp32), same shape."""
+    import torch
+    if acc.dtype != torch.float32 or x.dtype != torch.float32 or acc.shape != x.shape:
+        raise ValueError("acc and x must be fp32 of one shape")
+    if not (acc.is_cuda and x.is_cuda and acc.is_contiguous() and x.is_contiguous()):
+        raise ValueError("contiguous CUDA tensors expected")
+    with torch.cuda.device(acc.device):
+        st = lib().fa_accumulate_f32(acc.data_ptr(), x.data_ptr(), acc.numel(), _stream_ptr(acc.device))
+    _check(st, "fa_accumulate_f32")
 
 
 def to_bf16(x, out=None):

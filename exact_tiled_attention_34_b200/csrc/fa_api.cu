@@ -156,13 +156,13 @@ fa_status set_smem(K kernel, int bytes, std::once_flag (&flags)[kMaxDevices], cu
 }
 
 
-template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, int DS = D, bool DROP = false>
+template <int D, bool CAUSAL, bool SPARSE, bool XQK = false, int DS = D, bool DROP = false, bool MERGE = false>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const fa::FwdParamsT<DROP>& p, cudaStream_t stream) {
   static std::once_flag flags[kMaxDevices];
   static cudaError_t errs[kMaxDevices];
   static int regs[kMaxDevices];
-  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK, DS, DROP>;
+  auto kernel = fa::fa_fwd_kernel<D, CAUSAL, SPARSE, XQK, DS, DROP, MERGE>;
   constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
   if (set_smem(kernel, smem, flags, errs) != FA_OK) return FA_ERR_CUDA;
   // The kernel re-divides its register pool between warpgroups: refuse to launch a
@@ -201,16 +201,23 @@ fa_status launch_fwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
 }
 
 // drop: dropout settings, or nullptr (dropout needs d 64 or 128, N_q = N_k and no tile mask).
+// o_acc, lse_acc: the merging forward (fp32 running result updated in place; then o and
+// lse are not used): N_q = N_k, [B, H, N, d] layout, d 64 or 128, no mask or dropout.
 fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
                      int B, int H, int N, int Nk, int d, int layout, int causal, float scale, void* stream,
-                     const fa::DropParams* drop = nullptr) {
+                     const fa::DropParams* drop = nullptr, float* o_acc = nullptr, float* lse_acc = nullptr) {
   fa_status s;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
   const bool bnhd = layout == FA_LAYOUT_BNHD;
-  if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
+  const bool merge = o_acc != nullptr;
+  if ((s = check_ptrs({q, k, v, merge ? static_cast<const void*>(o_acc) : o,
+                       merge ? static_cast<const void*>(lse_acc) : lse})) != FA_OK)
+    return s;
   if ((s = check_sizes(B, H, N, d)) != FA_OK) return s;
   if ((s = check_sizes(B, H, Nk, d)) != FA_OK) return s;
   if (mask != nullptr && Nk != N) return FA_ERR_UNSUPPORTED;
+  if (merge && (mask != nullptr || drop != nullptr || Nk != N || bnhd || (d != 64 && d != 128)))
+    return FA_ERR_UNSUPPORTED;
   if (drop != nullptr && (mask != nullptr || Nk != N || d == 96 || d == 256)) return FA_ERR_UNSUPPORTED;
   if ((s = check_scale(scale)) != FA_OK) return s;
   if ((s = encoder()) != FA_OK) return s;
@@ -239,7 +246,16 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.n_qblocks = (p.n_tiles + 1) / 2;
   p.n_items = p.n_qblocks * BH;
   p.c_log2 = scale * 1.4426950408889634f;
+  p.o_acc = o_acc;
+  p.lse_acc = lse_acc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (merge) {
+    if (causal)
+      return d == 64 ? launch_fwd<64, true, false, false, 64, false, true>(mq, mk, mv, p, st)
+                     : launch_fwd<128, true, false, false, 128, false, true>(mq, mk, mv, p, st);
+    return d == 64 ? launch_fwd<64, false, false, false, 64, false, true>(mq, mk, mv, p, st)
+                   : launch_fwd<128, false, false, false, 128, false, true>(mq, mk, mv, p, st);
+  }
   if (d == 256) {  // one Q tile per work item
     p.n_qblocks = p.n_tiles;
     p.n_items = p.n_tiles * BH;
@@ -417,6 +433,8 @@ fa_status bwd_stage(BwdStage stage, const void* q, const void* k, const void* v,
   p.dq = stage == BwdStage::kDq ? static_cast<__nv_bfloat16*>(out0) : nullptr;
   p.dk = stage == BwdStage::kDkdv ? static_cast<__nv_bfloat16*>(out0) : nullptr;
   p.dv = stage == BwdStage::kDkdv ? static_cast<__nv_bfloat16*>(out1) : nullptr;
+  p.dk32 = nullptr;
+  p.dv32 = nullptr;
   p.tile_mask = mask;
   p.status = status;
   set_wait_limit(&p.timeout_ns, &p.stall);
@@ -605,6 +623,14 @@ fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, f
   return fwd_common(q, k, v, o, lse, nullptr, B, H, N, N, d, FA_LAYOUT_BHND, causal != 0, scale, stream, &dp);
 }
 
+fa_status fa_fwd_merge(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, int B, int H,
+                       int N, int d, int causal, float scale, void* stream) {
+  if (o_acc == nullptr || lse_acc == nullptr) return FA_ERR_INVALID_ARG;
+  // o and lse are not written by the merging kernels; the running result stands in for them.
+  return fwd_common(q, k, v, o_acc, lse_acc, nullptr, B, H, N, N, d, FA_LAYOUT_BHND, causal != 0, scale, stream,
+                    nullptr, o_acc, lse_acc);
+}
+
 fa_status fa_device_status(void* stream, int* detail) {
   int* status;
   if (detail) *detail = 0;
@@ -790,9 +816,10 @@ fa_status fused_pre(const void* o, const void* dO, const float* lse, void* ws, s
 
 // The fused kernel: dk, dv written, dQ added into the accumulator (which the
 // pre-pass must have zeroed).
+// f32: dk and dv are fp32 outputs (float*), else bf16.
 fa_status fused_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const void* ws,
                      size_t ws_bytes, const uint8_t* mask, int mask_block, int B, int H, int N, int Nk, int d,
-                     int layout, int causal, float scale, void* stream) {
+                     int layout, int causal, float scale, void* stream, bool f32 = false) {
   fa_status s;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID_ARG;
   const bool bnhd = layout == FA_LAYOUT_BNHD;
@@ -820,8 +847,10 @@ fa_status fused_main(const void* q, const void* k, const void* v, const void* dO
   p.lse2 = a.lse2;
   p.Drow = a.Drow;
   p.dq = nullptr;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk = f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
+  p.dv = f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
+  p.dk32 = f32 ? static_cast<float*>(dk) : nullptr;
+  p.dv32 = f32 ? static_cast<float*>(dv) : nullptr;
   p.tile_mask = mask;
   p.status = status;
   set_wait_limit(&p.timeout_ns, &p.stall);
@@ -934,6 +963,14 @@ fa_status fa_bwd_fused_main(const void* q, const void* k, const void* v, const v
                             int H, int N, int d, int causal, float scale, void* stream) {
   return fused_main(q, k, v, dO, dk, dv, workspace, workspace_bytes, tile_mask, mask_block, B, H, N, N, d,
                     FA_LAYOUT_BHND, causal != 0, scale, stream);
+}
+
+fa_status fa_bwd_fused_main_f32(const void* q, const void* k, const void* v, const void* dO, float* dk, float* dv,
+                                void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
+                                float scale, void* stream) {
+  if (d == 256) return FA_ERR_UNSUPPORTED;  // the head-dim-256 kernel writes bf16 only
+  return fused_main(q, k, v, dO, dk, dv, workspace, workspace_bytes, nullptr, 128, B, H, N, N, d, FA_LAYOUT_BHND,
+                    causal != 0, scale, stream, true);
 }
 
 fa_status fa_bwd_fused_dq(void* dq, const void* workspace, size_t workspace_bytes, int B, int H, int N, int d,

@@ -112,6 +112,8 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dk32;          // fused backward with fp32 outputs: dK, dV written as fp32 (dk, dv unused)
+  float* dv32;
   const uint8_t* tile_mask;  // [nT, nT] or nullptr
   int* status;
   unsigned long long timeout_ns;
@@ -280,6 +282,19 @@ __device__ __forceinline__ void store_regs_bf16(__nv_bfloat16* dst, const uint32
     for (int t = 0; t < 16; ++t)
       w[t] = pack_bf16(__uint_as_float(v[cc * 32 + 2 * t]) * mul, __uint_as_float(v[cc * 32 + 2 * t + 1]) * mul);
     store_row64(dst + cc * 32, w, v8);
+  }
+}
+
+// The first ncols (a multiple of 32) of NCOL fp32 values of the thread's row, times mul,
+// as fp32 to dst (16-byte aligned).
+template <int NCOL>
+__device__ __forceinline__ void store_regs_f32(float* dst, const uint32_t (&v)[NCOL], float mul, int ncols) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int c = 0; c < NCOL / 4; ++c) {
+    if (c * 4 >= ncols) break;
+    d4[c] = make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
+                        __uint_as_float(v[4 * c + 2]) * mul, __uint_as_float(v[4 * c + 3]) * mul);
   }
 }
 

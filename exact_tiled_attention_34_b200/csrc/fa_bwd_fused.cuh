@@ -537,7 +537,12 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty);
-      if (kvalid) store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row, acc, h == 0 ? p.scale : 1.f, p.ds, p.v8 != 0);
+      if (kvalid) {
+        if (p.dk32 != nullptr)  // fp32 outputs (a key block's share of a longer sequence's gradients)
+          store_regs_f32<D>((h == 0 ? p.dk32 : p.dv32) + row, acc, h == 0 ? p.scale : 1.f, p.ds);
+        else
+          store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row, acc, h == 0 ? p.scale : 1.f, p.ds, p.v8 != 0);
+      }
     }
     // Every reduce-add copy of this warp must be complete (its source is this CTA's
     // shared memory and its target the caller's workspace) before the kernel ends.

@@ -56,6 +56,10 @@ struct FwdParams {
   int n_qblocks;             // ceil(n_tiles / 2)
   int n_items;               // n_qblocks * BH work items (query block, batch*head)
   float c_log2;              // scale * log2(e)
+  // Merging kernels (MERGE): the running result of earlier key blocks, updated in place
+  // (fp32 [BH, N, D] and [BH, N]); o and lse above are then not written.
+  float* o_acc;
+  float* lse_acc;
 };
 
 // The dropout kernels' parameters (the others keep the plain block unchanged).
@@ -259,7 +263,10 @@ constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 // DS: the head dim as stored (row length of q, k, v, o): D, or 96 on the D = 128 kernels
 // (the loads read zeros for columns 96..127; only DS columns of O are written).
 // DROP: dropout on the probabilities that multiply V (keep masks regenerated per tile).
-template <int D, bool CAUSAL, bool SPARSE, bool XQK, int DS, bool DROP = false>
+// MERGE: this call's keys are one block of a longer key sequence: the epilogue merges the
+// block's result into a running fp32 (O_acc, lse_acc) through their log-sum-exp, with no
+// bf16 rounding of the block's partial O (the online softmax's combination, one level up).
+template <int D, bool CAUSAL, bool SPARSE, bool XQK, int DS, bool DROP = false, bool MERGE = false>
 __global__ void __launch_bounds__(384, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParamsT<DROP> p) {
@@ -594,7 +601,44 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int ib = item.bh / p.H, ih = item.bh - ib * p.H;
       __nv_bfloat16* orow = p.o + seq_row_offset(ib, ih, tile * 128 + r, p.N, p.H, DS, p.bnhd != 0);
       const bool row_ok = tile * 128 + r < p.N;  // rows past N (last tile) do not exist
-      if (active && local > 0) {
+      if (MERGE && active && local > 0) {
+        // lse' = ln(e^lse_acc + e^lse_b), O_acc' = O_acc e^(lse_acc - lse') + (O / l) e^(lse_b - lse'),
+        // 32 columns of O at a time (then O_i is released).
+        float wa = 0.f, wb = 0.f, lnew = 0.f;
+        if (row_ok) {
+          const float lb = (m + __log2f(l)) * 0.69314718055994531f;  // this block's lse (l > 0 here)
+          const float la = p.lse_acc[row];
+          const float mx = fmaxf(la, lb);
+          wa = expf(la - mx);
+          wb = expf(lb - mx);
+          const float ssum = wa + wb;
+          lnew = mx + logf(ssum);
+          wa /= ssum;
+          wb /= ssum * l;  // with the 1 / l of this block's O
+        }
+        float4* oa = reinterpret_cast<float4*>(p.o_acc + row * D);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(trow + Cfg::tm_o(i) + cc * 32, ov);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 a = oa[cc * 8 + c];
+              oa[cc * 8 + c] =
+                  make_float4(a.x * wa + __uint_as_float(ov[4 * c]) * wb, a.y * wa + __uint_as_float(ov[4 * c + 1]) * wb,
+                              a.z * wa + __uint_as_float(ov[4 * c + 2]) * wb,
+                              a.w * wa + __uint_as_float(ov[4 * c + 3]) * wb);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->o_empty[i]);
+        if (row_ok) p.lse_acc[row] = lnew;
+      } else if (MERGE) {
+        mbar_arrive(&bars->o_empty[i]);  // the row saw no key of this block: nothing to merge
+      } else if (active && local > 0) {
         // l = 0: the row saw no key (causal with N_q > N_k): O = 0, lse = -inf.
         const float inv_l = (!XQK || l > 0.f) ? 1.f / l : 0.f;
         uint32_t ov[D];

@@ -78,6 +78,17 @@ __global__ void fa_accumulate_kernel(float* __restrict__ acc, const __nv_bfloat1
   a[1] = make_float4(a1.x + f2.x, a1.y + f2.y, a1.z + f3.x, a1.w + f3.y);
 }
 
+// acc[i] += x[i] (fp32), 8 elements per thread.
+__global__ void fa_accumulate_f32_kernel(float* __restrict__ acc, const float* __restrict__ x, long long n8) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= n8) return;
+  float4* a = reinterpret_cast<float4*>(acc) + 2 * t;
+  const float4* b = reinterpret_cast<const float4*>(x) + 2 * t;
+  const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
+  a[0] = make_float4(a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w);
+  a[1] = make_float4(a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w);
+}
+
 // out[i] = bf16(in[i]) (round to nearest even), 8 elements per thread.
 __global__ void fa_to_bf16_kernel(__nv_bfloat16* __restrict__ out, const float* __restrict__ in, long long n8) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -122,6 +133,16 @@ fa_status fa_accumulate_bf16(float* acc, const void* x, long long n, int overwri
   if (!grid_fits(n / 8)) return FA_ERR_UNSUPPORTED;
   fa_accumulate_kernel<<<blocks_for(n / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       acc, static_cast<const __nv_bfloat16*>(x), n / 8, overwrite != 0);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_accumulate_f32(float* acc, const float* x, long long n, void* stream) {
+  if (n < 0 || n % 8 != 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!acc || !x) return FA_ERR_INVALID_ARG;
+  if (!aligned(acc, 16) || !aligned(x, 16)) return FA_ERR_ALIGNMENT;
+  if (!grid_fits(n / 8)) return FA_ERR_UNSUPPORTED;
+  fa_accumulate_f32_kernel<<<blocks_for(n / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(acc, x, n / 8);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -342,6 +342,32 @@ fa_status fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, con
                            int d, void* stream);
 
 /*
+ * fa_fwd_merge: the attention of q against one key block (k, v), merged straight into the
+ * running result (o_acc fp32 [B,H,N,d], lse_acc fp32 [B,H,N], updated in place) by the
+ * kernel's epilogue with the rule of fa_merge_partial, without rounding the block's
+ * partial O to bf16 first. Query and key blocks have N rows each; causal = 1 applies the
+ * causal mask within the pair (the diagonal block of a longer sequence), else every key
+ * is visible. d 64 or 128 (else FA_ERR_UNSUPPORTED); a row that sees no key of the block
+ * is left unchanged. Other arguments and rules as for fa_fwd.
+ */
+fa_status fa_fwd_merge(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, int B, int H,
+                       int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_bwd_fused_main with fp32 outputs: dk and dv are fp32 [B,H,N,d] (a key block's share
+ * of the gradients of a longer sequence, to be accumulated in fp32 without a bf16
+ * rounding). The workspace's dQ accumulator receives dq's share as in fa_bwd_fused_main,
+ * so successive calls on one workspace (after one fa_bwd_fused_preprocess) add up the
+ * shares of several key blocks. d 64, 96 or 128 (256: FA_ERR_UNSUPPORTED); no mask.
+ */
+fa_status fa_bwd_fused_main_f32(const void* q, const void* k, const void* v, const void* dO, float* dk, float* dv,
+                                void* workspace, size_t workspace_bytes, int B, int H, int N, int d, int causal,
+                                float scale, void* stream);
+
+/* acc[i] += x[i] for i < n (fp32; device pointers, 16-byte aligned; n a multiple of 8). */
+fa_status fa_accumulate_f32(float* acc, const float* x, long long n, void* stream);
+
+/*
  * acc[i] = (overwrite ? 0 : acc[i]) + x[i] for i < n: fp32 accumulation of a bf16
  * partial gradient (device pointers, both 16-byte aligned; n a multiple of 8).
  */

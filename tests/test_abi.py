@@ -26,7 +26,8 @@ def test_exports_every_declared_symbol(L):
             "fa_bwd_dq", "fa_bwd_noalloc", "fa_debug_wait_timeout",
             "fa_debug_stall_producer", "fa_fwd_dropout", "fa_bwd_dropout", "fa_merge_partial",
             "fa_accumulate_bf16", "fa_to_bf16", "fa_bwd_fused_workspace_bytes", "fa_bwd_fused", "fa_bwd_fused_ex",
-            "fa_bwd_fused_preprocess", "fa_bwd_fused_main", "fa_bwd_fused_dq"} <= set(names)
+            "fa_bwd_fused_preprocess", "fa_bwd_fused_main", "fa_bwd_fused_dq", "fa_fwd_merge", "fa_bwd_fused_main_f32",
+            "fa_accumulate_f32"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True,
                          check=True).stdout
     defined = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -161,6 +162,23 @@ def test_fused_argument_checks(L):
     assert conv(A, A, need, 1, 1, 128, 64, float("inf"), None) == INVALID
     if NO_GPU:  # valid arguments get as far as the first CUDA call, as a forward does
         assert f() == _fwd(L)
+
+
+def test_merge_forward_and_f32_argument_checks(L):
+    m = lambda q=A, oa=A, la=A, d=64, N=128: L.fa_fwd_merge(q, A, A, oa, la, 1, 1, N, d, 0, 0.1, None)
+    assert m(oa=None) == INVALID and m(la=None) == INVALID and m(q=None) == INVALID
+    assert m(oa=A + 8) == ALIGN
+    assert m(d=96) == UNSUPPORTED and m(d=256) == UNSUPPORTED  # merging kernels: head dims 64 and 128
+    assert m(N=0) == INVALID
+    need = L.fa_bwd_fused_workspace_bytes(1, 1, 128, 64)
+    f = lambda dk=A, d=64, wsb=need: L.fa_bwd_fused_main_f32(A, A, A, A, dk, A, A, wsb, 1, 1, 128, d, 0, 0.1, None)
+    assert f(dk=None) == INVALID and f(dk=A + 4) == ALIGN
+    assert f(wsb=L.fa_bwd_workspace_bytes(1, 1, 128, 64)) == WORKSPACE
+    assert f(d=256) == UNSUPPORTED
+    acc = L.fa_accumulate_f32
+    assert acc(A, A, 12, None) == INVALID and acc(A, A, -8, None) == INVALID
+    assert acc(None, A, 8, None) == INVALID and acc(A + 8, A, 8, None) == ALIGN
+    assert acc(A, A, 0, None) == OK
 
 
 def test_dropout_argument_checks(L):

@@ -59,9 +59,13 @@ def test_merge_and_accumulate_check_dtypes_and_devices():
 
 
 def test_ring_visibility_rule():
-    # causal: key block src is visible to query block r iff src <= r; all without the mask
-    assert [ring._visible(True, s, 2) for s in range(4)] == [True, True, True, False]
-    assert all(ring._visible(False, s, 0) for s in range(4))
+    # chunks of one length at multiples of it: causal key chunk before the query chunk is
+    # fully visible, the same chunk is the causal diagonal, a later one is invisible
+    n = 64
+    assert [ring._pair_kind(True, 2 * n, s * n) for s in range(4)] == ["full", "full", "diag", None]
+    assert all(ring._pair_kind(False, 0, s * n) == "full" for s in range(4))
+    assert ring.chunk_offsets(1, 4, 128, False) == [128]
+    assert ring.chunk_offsets(1, 4, 128, True) == [64, 6 * 64]  # chunks 1 and 2R - 1 - 1 = 6
 
 
 class _RingThatMustNotExchange:

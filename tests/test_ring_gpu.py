@@ -50,17 +50,21 @@ class ThreadRing:
         return self.finish(self.start(tensors))
 
 
-def _run_ring(q, k, v, do, world, causal, scale):
+def _run_ring(q, k, v, do, world, causal, scale, zigzag=False):
+    """The ring's outputs, put back in global row order."""
     n = q.shape[2] // world
-    blk = lambda x, r: x[:, :, r * n:(r + 1) * n].contiguous()
+    rows = {r: (np.concatenate([np.arange(o, o + n // 2) for o in ring.chunk_offsets(r, world, n, True)])
+                if zigzag else np.arange(r * n, (r + 1) * n)) for r in range(world)}
+    blk = lambda x, r: x[:, :, torch.as_tensor(rows[r], device=x.device)].contiguous()
     inboxes = [queue.Queue() for _ in range(world)]
     res, errs = {}, []
 
     def rank_main(r):
         try:
             rg = ThreadRing(r, world, inboxes)
-            o, lse = ring.ring_forward(blk(q, r), blk(k, r), blk(v, r), causal, scale, rg)
-            g = ring.ring_backward(blk(q, r), blk(k, r), blk(v, r), o, lse, blk(do, r), causal, scale, rg)
+            o, lse = ring.ring_forward(blk(q, r), blk(k, r), blk(v, r), causal, scale, rg, zigzag=zigzag)
+            g = ring.ring_backward(blk(q, r), blk(k, r), blk(v, r), o, lse, blk(do, r), causal, scale, rg,
+                                   zigzag=zigzag)
             res[r] = (o, lse) + tuple(g)
         except Exception as e:  # reported below
             errs.append(e)
@@ -72,25 +76,118 @@ def _run_ring(q, k, v, do, world, causal, scale):
         t.join(timeout=300)
     assert not errs, errs
     torch.cuda.synchronize()
-    cat = lambda i: torch.cat([res[r][i] for r in range(world)], dim=2)
+    order = torch.as_tensor(np.argsort(np.concatenate([rows[r] for r in range(world)])), device=q.device)
+    cat = lambda i: torch.cat([res[r][i] for r in range(world)], dim=2)[:, :, order]
     return [cat(i) for i in range(5)]
 
 
 @pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("causal", [False, True])
-def test_ring_parity(cuda_device, world, d, causal):
+@pytest.mark.parametrize("causal,zigzag", [(False, False), (True, False), (True, True)])
+def test_ring_parity(cuda_device, world, d, causal, zigzag):
     B, H, n = 1, 2, 256
     N = world * n
     t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, N, d, seed=40 + world + d).items()}
     sc = 1.0 / math.sqrt(d)
-    o, lse, dq, dk, dv = _run_ring(t["q"], t["k"], t["v"], t["do"], world, causal, sc)
+    o, lse, dq, dk, dv = _run_ring(t["q"], t["k"], t["v"], t["do"], world, causal, sc, zigzag)
     assert fa.device_status() == (0, 0)
     ref = oracle.attn_bwd_ref(t["q"].cpu(), t["k"].cpu(), t["v"].cpu(), t["do"].cpu(), causal, sc)
     what = f"ring R={world} d={d} causal={causal}"
     assert_fwd_close(o.cpu(), lse.cpu(), ref["o"], ref["lse"], what)
     for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
         assert_grad_close(g.cpu(), ref[name], name, what)
+
+
+@pytest.mark.parametrize("causal,zigzag", [(True, False), (True, True), (False, False)])
+def test_ring_eight_ranks_long_blocks(cuda_device, causal, zigzag):
+    """R = 8 ranks of 1024 positions each (N = 8192), d = 128: the whole sequence against
+    the oracle; the fp32 accumulation of partial results keeps the error within the
+    single-GPU tolerances."""
+    world, B, H, n, d = 8, 1, 2, 1024, 128
+    N = world * n
+    t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, N, d, seed=48).items()}
+    sc = 1.0 / math.sqrt(d)
+    o, lse, dq, dk, dv = _run_ring(t["q"], t["k"], t["v"], t["do"], world, causal, sc, zigzag)
+    assert fa.device_status() == (0, 0)
+    c = {k: x.cpu() for k, x in t.items()}
+    for h in range(H):
+        ref = oracle.attn_bwd_ref(c["q"][:, h:h + 1], c["k"][:, h:h + 1], c["v"][:, h:h + 1], c["do"][:, h:h + 1],
+                                  causal, sc)
+        what = f"ring R=8 n=1024 causal={causal} zigzag={zigzag} h={h}"
+        assert_fwd_close(o[:, h:h + 1].cpu(), lse[:, h:h + 1].cpu(), ref["o"], ref["lse"], what)
+        for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+            assert_grad_close(g[:, h:h + 1].cpu(), ref[name], name, what)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_forward_merge_of_key_blocks(cuda_device, d):
+    """The merging forward over four key blocks (one on the causal diagonal) equals causal
+    attention of the last query block over all keys; rows are merged in fp32."""
+    B, H, c = 2, 3, 256
+    t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, 4 * c, d, seed=8, with_do=False).items()}
+    sc = 1.0 / math.sqrt(d)
+    q = t["q"][:, :, 3 * c:].contiguous()
+    acc = torch.zeros(q.shape, dtype=torch.float32, device=cuda_device)
+    lse = torch.full(q.shape[:3], -math.inf, dtype=torch.float32, device=cuda_device)
+    for b in range(4):
+        sl = slice(b * c, (b + 1) * c)
+        fa.forward_merge(q, t["k"][:, :, sl].contiguous(), t["v"][:, :, sl].contiguous(), acc, lse, causal=b == 3,
+                         scale=sc)
+    torch.cuda.synchronize()
+    assert fa.device_status() == (0, 0)
+    rows = np.arange(3 * c, 4 * c)
+    for bb in range(B):
+        for h in range(H):
+            o_ref, l_ref = oracle.attn_fwd_rows_ref(t["q"][bb, h].cpu()[3 * c:], rows, t["k"][bb, h].cpu(),
+                                                    t["v"][bb, h].cpu(), True, sc)
+            assert_fwd_close(acc[bb, h].cpu().numpy(), lse[bb, h].cpu().numpy(), o_ref, l_ref, f"merge d={d}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fused_f32_shares_sum_to_full(cuda_device, d):
+    """The sequence split into two halves: for every (query half, key half) pair the fused
+    kernel's fp32 dK, dV shares (with the whole sequence's row statistics), summed in fp32
+    over the query halves, and the dQ shares added in each query half's accumulator, give
+    the full gradients."""
+    B, H, N = 1, 2, 512
+    t = {k: x.to(cuda_device) for k, x in make_qkv(B, H, N, d, seed=9).items()}
+    sc = 1.0 / math.sqrt(d)
+    o, lse = fa.forward(t["q"], t["k"], t["v"], scale=sc)
+    half = lambda x, a: x[:, :, a * (N // 2):(a + 1) * (N // 2)].contiguous()
+    wss = []
+    for a in range(2):
+        ws = torch.empty(fa.bwd_workspace_bytes(B, H, N // 2, d, deterministic=False), dtype=torch.uint8,
+                         device=cuda_device)
+        fa.bwd_fused_preprocess(half(o, a), half(t["do"], a), half(lse, a), ws)
+        wss.append(ws)
+    acc = {n: [torch.zeros((B, H, N // 2, d), dtype=torch.float32, device=cuda_device) for _ in range(2)]
+           for n in ("dk", "dv")}
+    for a in range(2):
+        for b in range(2):
+            dk, dv = (torch.empty((B, H, N // 2, d), dtype=torch.float32, device=cuda_device) for _ in range(2))
+            fa.bwd_fused_main_f32(half(t["q"], a), half(t["k"], b), half(t["v"], b), half(t["do"], a), dk, dv, wss[a],
+                                  scale=sc)
+            fa.accumulate_f32(acc["dk"][b], dk)
+            fa.accumulate_f32(acc["dv"][b], dv)
+    dqs = []
+    for a in range(2):
+        dq = torch.empty((B, H, N // 2, d), dtype=torch.bfloat16, device=cuda_device)
+        fa.bwd_fused_dq(dq, wss[a], scale=sc)
+        dqs.append(dq)
+    torch.cuda.synchronize()
+    assert fa.device_status() == (0, 0)
+    ref = oracle.attn_bwd_ref(t["q"].cpu(), t["k"].cpu(), t["v"].cpu(), t["do"].cpu(), False, sc)
+    assert_grad_close(torch.cat(dqs, dim=2).cpu(), ref["dq"], "dq", f"fp32 shares d={d}")
+    assert_grad_close(torch.cat(acc["dk"], dim=2).cpu().numpy(), ref["dk"], "dk", f"fp32 shares d={d}")
+    assert_grad_close(torch.cat(acc["dv"], dim=2).cpu().numpy(), ref["dv"], "dv", f"fp32 shares d={d}")
+
+
+def test_accumulate_f32(cuda_device):
+    a = torch.randn(4096, device=cuda_device)
+    x = torch.randn(4096, device=cuda_device)
+    ref = a + x
+    fa.accumulate_f32(a, x)
+    assert torch.equal(a, ref)
 
 
 @pytest.mark.parametrize("d", [64, 128])

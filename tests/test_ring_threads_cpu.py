@@ -10,18 +10,19 @@ import torch
 
 import oracle
 from exact_tiled_attention_34_b200 import ring
-from tests.test_ring_cpu import OracleBlockOps
+from tests.test_ring_cpu import OracleBlockOps, zigzag_rows
 from tests.test_ring_gpu import ThreadRing
 
 
-@pytest.mark.parametrize("world", [1, 2, 4])
-@pytest.mark.parametrize("causal", [False, True])
-def test_thread_ring_matches_full_attention(world, causal):
+@pytest.mark.parametrize("world", [1, 2, 4, 8])
+@pytest.mark.parametrize("causal,zigzag", [(False, False), (True, False), (True, True)])
+def test_thread_ring_matches_full_attention(world, causal, zigzag):
     B, H, n, d, scale = 1, 2, 4, 3, 0.9
     N = world * n
     g = torch.Generator().manual_seed(3 + world)
     q, k, v, do = (torch.randn((B, H, N, d), generator=g, dtype=torch.float64) for _ in range(4))
-    blk = lambda x, r: x[:, :, r * n:(r + 1) * n].contiguous()
+    rows = {r: (zigzag_rows(r, world, n) if zigzag else np.arange(r * n, (r + 1) * n)) for r in range(world)}
+    blk = lambda x, r: x[:, :, torch.as_tensor(rows[r])].contiguous()
     inboxes = [queue.Queue() for _ in range(world)]
     res, errs = {}, []
 
@@ -29,9 +30,9 @@ def test_thread_ring_matches_full_attention(world, causal):
         try:
             rg = ThreadRing(r, world, inboxes)
             ops = OracleBlockOps(scale)
-            o, lse = ring.ring_forward(blk(q, r), blk(k, r), blk(v, r), causal, scale, rg, ops)
+            o, lse = ring.ring_forward(blk(q, r), blk(k, r), blk(v, r), causal, scale, rg, ops, zigzag)
             res[r] = (o, lse) + tuple(ring.ring_backward(blk(q, r), blk(k, r), blk(v, r), o, lse, blk(do, r),
-                                                          causal, scale, rg, ops))
+                                                          causal, scale, rg, ops, zigzag))
         except Exception as e:  # reported below
             errs.append(e)
 
@@ -43,5 +44,5 @@ def test_thread_ring_matches_full_attention(world, causal):
     assert not errs, errs
     full = oracle.attn_bwd_ref(q, k, v, do, causal, scale)
     for i, name in enumerate(("o", "lse", "dq", "dk", "dv")):
-        got = torch.cat([res[r][i] for r in range(world)], dim=2).numpy()
-        assert np.max(np.abs(got - full[name])) < 1e-12, name
+        for r in range(world):
+            assert np.max(np.abs(res[r][i].numpy() - full[name][:, :, rows[r]])) < 1e-12, (name, r)
