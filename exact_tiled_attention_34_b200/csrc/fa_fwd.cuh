@@ -253,11 +253,11 @@ __device__ __forceinline__ void softmax_row(float (&s)[128], int lim, float c, f
 }
 
 // Register split of the 384-thread forward block (launched with 168 per thread,
-// 64,512 in all): the producer/MMA warpgroup drops to 104, the two softmax
-// warpgroups rise to 184 -> 128 * (104 + 2 * 184) = 60,416. Only the softmax
-// warpgroups increase, once, by less than the first warpgroup releases.
-constexpr int kFwdRegsCtl = 104;
-constexpr int kFwdRegsSoftmax = 184;
+// 64,512 in all): the producer/MMA warpgroup drops to 88, the two softmax
+// warpgroups rise to 208 -> 128 * (88 + 2 * 208) = 64,512. Only the softmax
+// warpgroups increase, once, by what the first warpgroup releases.
+constexpr int kFwdRegsCtl = 88;
+constexpr int kFwdRegsSoftmax = 208;
 constexpr int kFwdRegsNeeded = 128 * (kFwdRegsCtl + 2 * kFwdRegsSoftmax);
 
 // DS: the head dim as stored (row length of q, k, v, o): D, or 96 on the D = 128 kernels
