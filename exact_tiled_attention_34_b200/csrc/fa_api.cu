@@ -768,13 +768,13 @@ fa_status launch_fused(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     regs[dev] = attr.numRegs;
   }
   // The kernel re-divides its register pool between warpgroups.
-  if (regs[dev] * fa::kBwdThreads < fa::kFusedRegsNeeded) return FA_ERR_UNSUPPORTED;
+  if (regs[dev] * fa::kFusedThreads < fa::kFusedRegsNeeded) return FA_ERR_UNSUPPORTED;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return FA_ERR_CUDA;
   unsigned grid = unsigned(p.n_ktiles) * unsigned(p.BH);
   if (grid > unsigned(sms)) grid = unsigned(sms);  // persistent: at most one CTA per SM
-  kernel<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, macc, p);
+  kernel<<<grid, fa::kFusedThreads, smem, stream>>>(mq, mk, mv, mdo, macc, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -794,7 +794,7 @@ fa_status launch_bwd256(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
     regs[dev] = attr.numRegs;
   }
-  if (regs[dev] * fa::kBwdThreads < fa::kFusedRegsNeeded) return FA_ERR_UNSUPPORTED;
+  if (regs[dev] * fa::kBwdThreads < fa::kBwd256RegsNeeded) return FA_ERR_UNSUPPORTED;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return FA_ERR_CUDA;

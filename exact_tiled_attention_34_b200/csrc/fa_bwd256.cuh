@@ -85,6 +85,14 @@ struct SubSched256 {
   __device__ __forceinline__ int first() const { return next(-1); }
 };
 
+// Register split of the 384-thread block (launched with 168 per thread, 64,512 in all):
+// the producer/MMA warpgroup drops to 120, the compute warpgroups rise to 192:
+// 128 * (120 + 2 * 192) = 64,512. Only the compute warpgroups increase, once, by what
+// the first releases.
+constexpr int kBwd256RegsCtl = 120;
+constexpr int kBwd256RegsCompute = 192;
+constexpr int kBwd256RegsNeeded = 128 * (kBwd256RegsCtl + 2 * kBwd256RegsCompute);
+
 template <bool CAUSAL, bool SPARSE, bool XQK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -149,7 +157,7 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    regs_dec<kFusedRegsCtl>();
+    regs_dec<kBwd256RegsCtl>();
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -197,7 +205,7 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    regs_dec<kFusedRegsCtl>();
+    regs_dec<kBwd256RegsCtl>();
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
       const uint32_t aDS = smem_u32(sDS);
@@ -288,11 +296,11 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmCols);
   } else if (warp < 4) {
-    regs_dec<kFusedRegsCtl>();
+    regs_dec<kBwd256RegsCtl>();
     __syncthreads();
   } else {
     // ------------------------------------------------------------ compute warpgroups
-    regs_inc<kFusedRegsCompute>();
+    regs_inc<kBwd256RegsCompute>();
     const int h = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row (S^T, dP^T, dK, dV) / head-dim row (dQ^T)

@@ -15,22 +15,28 @@
 // (whole 128-byte lines reduced in L2). The order in which key tiles add into a dQ
 // row varies from run to run, so dQ is not bit-reproducible (dK and dV are).
 //
-// Work item = (128-key tile j, batch*head) as in the dK/dV kernel; 384 threads:
-//   warp 0      TMA producer: K_j, V_j per item; Q_i (+ row arrays) and dO_i per tile
-//   warp 1      MMA issuer + TMEM owner
-//   warps 4-11  two compute warpgroups (thread = key row = TMEM lane; warpgroup h
-//               takes query columns [64h, 64h + 64) of S^T and dP^T)
+// Work item = (128-key tile j, batch*head) as in the dK/dV kernel; 512 threads:
+//   warp 0       TMA producer: K_j, V_j per item; Q_i (+ row arrays) and dO_i per tile
+//   warp 1       MMA issuer + TMEM owner
+//   warps 4-11   two compute warpgroups (thread = key row = TMEM lane; warpgroup h
+//                takes query columns [64h, 64h + 64) of S^T and dP^T)
+//   warps 12-15  dQ warpgroup (thread = query row = TMEM lane): dQ_i out of tensor
+//                memory, through shared memory, into dQacc by reduce-add copies
 // dS leaves the compute warps through shared memory (bf16, 128 x 128, 128-byte
 // swizzle, [query block of 64][key row][128 B]); that one buffer is the K-major A
-// operand of dK += dS^T Q and the MN-major A operand of dQ = dS K. After dQ's
-// product completes, each compute warp reuses its own 4 KB of that buffer as the
-// staging area of its dQ rows (fp32, 32 x 32 boxes) for the reduce-add.
+// operand of dK += dS^T Q and the MN-major A operand of dQ = dS K. Each dQ warp stages
+// its 32 dQ rows (fp32, 32 x 32 boxes, 4 KB each) for the reduce-add in a stage area
+// of its own (8 KB per warp); at head dim 128, where a warp has four boxes and shared
+// memory has no room for 16 KB per warp, its first two boxes go to 8 KB of the dS buffer
+// (free once dQ's product is done) and the compute warps write the next dS only once
+// those two copies have read their stages. With the drain in warps of its own, the
+// compute warps go from one tile's dS straight to the next tile's exponentials.
 //
 // Tensor memory (512 columns): dK | dV | X (S^T, then P^T as packed bf16) |
 // Y (dP^T; at head dim 128 also dQ) | Z (dQ at head dim 64). At head dim 128 the five
 // buffers do not fit, so dQ_i shares Y with dP^T: dP^T of the next tile is issued once
-// the compute warps have read dQ_i out (they do that after the next tile's
-// exponentials, in the shadow of the other products).
+// the dQ warps have read dQ_i out (while the compute warps run the next tile's
+// exponentials). At head dim 64 the next dQ product waits for the same read.
 #pragma once
 
 #include "fa_bwd.cuh"
@@ -53,11 +59,11 @@ struct FusedCfg {
   static constexpr int kOffDS = kOffDO + kDoStages * kTileBytes;    // dS bf16 128 x 128 / dQ stages
   static constexpr int kOffL = kOffDS + 32768;                      // -lse log2 e rows, 2 stages
   static constexpr int kOffDr = kOffL + 1024;                       // D rows, 2 stages
-  // Head dim 128: a second dQ staging area (4 KB per compute warp), so that a warp's two
-  // 32-column boxes leave without waiting for the first copy to read its stage.
-  static constexpr int kStage2Bytes = (D == 128) ? 32768 : 0;
-  static constexpr int kOffStage2 = kOffDr + 1024;
-  static constexpr int kOffBar = kOffStage2 + kStage2Bytes;
+  // dQ stage area, 8 KB per dQ warp: all of a warp's boxes at head dim 64, the last two
+  // of its four at head dim 128 (the first two are staged in the dS buffer).
+  static constexpr bool kStageInDs = (D == 128);
+  static constexpr int kOffStage = kOffDr + 1024;
+  static constexpr int kOffBar = kOffStage + 32768;
   // Barriers (well under 256 bytes), plus 1 KB of alignment slack at head dim 64. At head
   // dim 128 there is no room for the slack: the kernel then requires the dynamic
   // shared-memory base to be 1024-byte aligned (it is when, as here, the kernel declares
@@ -87,7 +93,8 @@ struct FusedBars {
   uint64_t dq_full;      // dQ_i's product is done (and with it every read of dS_i)
   uint64_t p_ready;      // 256 arrivals: P^T is in tensor memory
   uint64_t ds_ready;     // 256: dS is in shared memory and dP^T has been read
-  uint64_t dq_taken;     // 256: dQ_i has been read out of tensor memory
+  uint64_t dq_taken;     // 128: dQ_i has been read out of tensor memory
+  uint64_t ds_free;      // 4 (one per dQ warp): the copies staged in the dS buffer have read it (head dim 128)
   uint64_t rd_s;         // 256: both warpgroups have read S^T
   uint64_t acc_done;
   uint64_t acc_empty;    // 256: the epilogue has read dK and dV
@@ -99,7 +106,7 @@ struct FusedBars {
 enum FusedSite : int {
   kSiteFuKV = 301, kSiteFuQEmpty, kSiteFuDoEmpty, kSiteFuKvEmpty, kSiteFuQFull, kSiteFuDoFull, kSiteFuPReady,
   kSiteFuDsReady, kSiteFuDqTaken, kSiteFuAcc, kSiteFuSFull, kSiteFuDpFull, kSiteFuDqFull, kSiteFuRead,
-  kSiteFuDrain,
+  kSiteFuDrain, kSiteFuDsFree,
   kSiteFuSmemAlign = 399  // reported with kStatusUnsupported: dynamic shared memory not 1024-aligned
 };
 constexpr int kStatusUnsupported = 2;  // == FA_ERR_UNSUPPORTED
@@ -129,16 +136,20 @@ __device__ __forceinline__ void mma_dq_ss(uint32_t tm, uint32_t a_ds, uint32_t b
            k > 0 ? 1u : 0u);
 }
 
-// Register split of the 384-thread block (launched with 168 per thread, 64,512 in all):
-// the producer/MMA warpgroup drops to 120 (the issuer keeps the descriptors of five
-// products in registers), the compute warpgroups rise to 192: 128 * (120 + 2 * 192) =
-// 64,512. Only the compute warpgroups increase, once, by what the first releases.
-constexpr int kFusedRegsCtl = 120;
-constexpr int kFusedRegsCompute = 192;
-constexpr int kFusedRegsNeeded = 128 * (kFusedRegsCtl + 2 * kFusedRegsCompute);
+// Register split of the 512-thread block (launched with 128 per thread, 65,536 in all):
+// the producer/MMA warpgroup drops to 96 (the issuer keeps the descriptors of five
+// products in registers), the dQ warpgroup keeps 96 (64 hold two boxes of dQ), the
+// compute warpgroups rise to 160: 128 * (96 + 96 + 2 * 160) = 65,536. Only the compute
+// warpgroups increase, once, by what the first releases.
+constexpr int kFusedThreads = 512;
+constexpr int kFusedRegsCtl = 96;
+constexpr int kFusedRegsDrain = 96;
+constexpr int kFusedRegsCompute = 160;
+constexpr int kFusedRegsNeeded = 128 * (kFusedRegsCtl + kFusedRegsDrain + 2 * kFusedRegsCompute);
+static_assert(kFusedRegsNeeded <= 65536, "fused backward register split above the register file");
 
 template <int D, bool CAUSAL, bool SPARSE, bool XQK>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kFusedThreads, 1)
 fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
@@ -180,7 +191,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
-    mbar_init(&bars->dq_taken, 256);
+    mbar_init(&bars->dq_taken, 128);
+    mbar_init(&bars->ds_free, 4);
     mbar_init(&bars->rd_s, 256);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->acc_empty, 256);
@@ -322,6 +334,11 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           // dK += dS^T Q_i and dQ_i = dS K_j, both reading dS from shared memory.
           if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteFuDsReady)) { ok = false; break; }
+          // Head dim 64: Z may still hold the previous tile's dQ.
+          if (!Cfg::kDqInY && it > 0 && !mbar_wait(&bars->dq_taken, (it - 1) & 1, wc, kSiteFuDqTaken)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           mma_dk_ss<D>(tmem + Cfg::kTmDK, aDS, aQ + st * Cfg::kTileBytes, !first);
           mma_dq_ss<D>(tmem + Cfg::kTmDQ, aDS, aK);
@@ -356,6 +373,88 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // idle warps of the first warpgroup: they take part in its register hand-over
     regs_dec<kFusedRegsCtl>();
     __syncthreads();
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ dQ warpgroup
+    // dQ_t out of tensor memory (thread = query row 32 quarter + lane of tile t) into
+    // global dQacc rows [128 t + 32 quarter, +32), in 32 x 32 fp32 boxes through this
+    // warp's stages, each box added by one reduce-add copy as soon as it is staged.
+    regs_dec<kFusedRegsDrain>();
+    const int quarter = warp & 3;
+    const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
+    bool ok = true;
+    int it = 0;
+    BwdItem item;
+    for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
+      KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
+      for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, it & 1, wc, kSiteFuDqFull))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int y0 = i * 128 + quarter * 32;
+        // Two 32-column boxes leave tensor memory in one load (64 registers); each is
+        // staged and reduce-added by lane 0 as one copy.
+        uint32_t v[64];
+        auto stage_box = [&](int b, int half, uint8_t* stage) {
+          uint4* s4 = reinterpret_cast<uint4*>(stage);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int o = half * 32 + 4 * c;
+            s4[lane * 8 + (c ^ (lane & 7))] = make_uint4(v[o], v[o + 1], v[o + 2], v[o + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tma_reduce_add_3d(&tm_dqacc, stage, b * 32, y0, item.bh);
+        };
+        uint8_t* area = smem + Cfg::kOffStage + quarter * 8192;
+        if constexpr (Cfg::kStageInDs) {
+          // Boxes 0 and 1 into this warp's 8 KB of the dS buffer (free: dQ's product, the
+          // last reader of dS, is done), committed as a group of their own so that the
+          // buffer is released as soon as they are read; boxes 2 and 3 into the stage area.
+          uint8_t* in_ds = sDS + quarter * 8192;
+          tmem_ld64(trow + Cfg::kTmDQ, v);
+          tmem_wait_ld();
+          stage_box(0, 0, in_ds);
+          stage_box(1, 1, in_ds + 4096);
+          if (lane == 0) bulk_commit();
+          tmem_ld64(trow + Cfg::kTmDQ + 64, v);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&bars->dq_taken);  // every column of dQ_t is in registers: its columns are free
+          stage_box(2, 0, area);
+          stage_box(3, 1, area + 4096);
+          if (lane == 0) {
+            bulk_commit();
+            bulk_wait_read1();  // boxes 0 and 1 are read: the next dS may be written
+            mbar_arrive(&bars->ds_free);
+            bulk_wait_read0();  // this warp's stage area may be overwritten by the next tile
+          }
+        } else {
+          tmem_ld64(trow + Cfg::kTmDQ, v);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&bars->dq_taken);
+          stage_box(0, 0, area);
+          stage_box(1, 1, area + 4096);
+          if (lane == 0) {
+            bulk_commit();
+            bulk_wait_read0();
+          }
+        }
+        __syncwarp();
+      }
+    }
+    // Every reduce-add copy of this warp must be complete (its source is this CTA's
+    // shared memory and its target the caller's workspace) before the kernel ends; a
+    // copy issued before an abort may not be committed yet, hence the commit.
+    if (lane == 0) {
+      bulk_commit();
+      bulk_wait0();
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
   } else {
     // ------------------------------------------------------------ compute warpgroups
     regs_inc<kFusedRegsCompute>();
@@ -364,66 +463,15 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int r = quarter * 32 + lane;  // key row within tile j (TMEM lane of S^T, dP^T, dK, dV)
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;
-    // This warp's 4 KB of the dS buffer: its dS rows (key rows of the warp, query block
-    // h), and after dQ's product the staging area of its dQ boxes.
-    uint8_t* my_ds = sDS + h * 16384 + r * 128;
-    uint8_t* my_stage = sDS + h * 16384 + quarter * 4096;
-    uint8_t* my_stage2 = smem + Cfg::kOffStage2 + (h * 4 + quarter) * 4096;  // head dim 128 only
+    uint8_t* my_ds = sDS + h * 16384 + r * 128;  // this thread's dS row (key row r, query block h)
     bool ok = true;
     int it = 0;
-    // dQ_t out of tensor memory into global dQacc rows [128 ti + 32 quarter, +32), columns
-    // [h D/2, (h+1) D/2), in 32 x 32 fp32 boxes through the stage.
-    auto stage_box = [&](const uint32_t (&v)[32], uint8_t* stage) {
-      uint4* s4 = reinterpret_cast<uint4*>(stage);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        s4[lane * 8 + (c ^ (lane & 7))] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-    };
-    auto drain = [&](int t, int ti, int bh) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, t & 1, wc, kSiteFuDqFull))) return false;
-      tc_fence_after();
-      const int x0 = h * (D / 2), y0 = ti * 128 + quarter * 32;
-      uint32_t v[32];
-      tmem_ld32(trow + Cfg::kTmDQ + h * (D / 2), v);
-      tmem_wait_ld();
-      if constexpr (D == 64) {
-        tc_fence_before();
-        mbar_arrive(&bars->dq_taken);
-        stage_box(v, my_stage);
-        if (lane == 0) {
-          tma_reduce_add_3d(&tm_dqacc, my_stage, x0, y0, bh);
-          bulk_commit();
-        }
-      } else {
-        // Two 32-column boxes through two 4 KB stages: the first is staged before the
-        // second leaves tensor memory, so that Y is released early (only 32 values are
-        // held in registers at a time), and neither copy is waited for here (the wait
-        // comes before this warp next writes dS, a phase later).
-        stage_box(v, my_stage);
-        tmem_ld32(trow + Cfg::kTmDQ + h * (D / 2) + 32, v);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars->dq_taken);
-        if (lane == 0) {
-          tma_reduce_add_3d(&tm_dqacc, my_stage, x0, y0, bh);
-          bulk_commit();
-        }
-        stage_box(v, my_stage2);
-        if (lane == 0) {
-          tma_reduce_add_3d(&tm_dqacc, my_stage2, x0 + 32, y0, bh);
-          bulk_commit();
-        }
-      }
-      return true;
-    };
     BwdItem item;
     for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
       const int j = item.tile;
       KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
       const bool kvalid = j * 128 + r < p.Nk;  // key rows past N_k (last tile) contribute nothing
-      int local = 0, prev_i = -1;
+      int local = 0;
       for (int i = sch.first(); i >= 0; i = sch.next(i), ++it, ++local) {
         const int st = it & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->q_full[st], (it >> 1) & 1, wc, kSiteFuQFull)) ||
@@ -471,11 +519,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
-        // ---- the previous tile's dQ leaves tensor memory (in the shadow of this tile's products)
-        if (local > 0 && !drain(it - 1, prev_i, item.bh)) {
-          ok = false;
-          break;
-        }
         // ---- dS = P (dP - D) into shared memory
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full, it & 1, wc, kSiteFuDpFull))) {
           ok = false;
@@ -497,9 +540,12 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ds[t] = pack_bf16(v.x, v.y);
           }
         }
-        // The stages may still be read by this warp's last reduce-add copies.
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
+        // Head dim 128: the dS buffer may still be read by the previous tile's copies.
+        if (Cfg::kStageInDs && it > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&bars->ds_free, (it - 1) & 1, wc, kSiteFuDsFree))) {
+          ok = false;
+          break;
+        }
         {
           uint4* d4 = reinterpret_cast<uint4*>(my_ds);
 #pragma unroll
@@ -509,13 +555,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars->ds_ready);
-        prev_i = i;
       }
       if (!ok) break;
-      if (local > 0 && !drain(it - 1, prev_i, item.bh)) {
-        ok = false;
-        break;
-      }
       // -------------------------------------------------------- epilogue: dK (h = 0), dV (h = 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_done, kk & 1, wc, kSiteFuAcc))) {
         ok = false;
@@ -544,10 +585,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           store_regs_bf16<D>((h == 0 ? p.dk : p.dv) + row, acc, h == 0 ? p.scale : 1.f, p.ds, p.v8 != 0);
       }
     }
-    // Every reduce-add copy of this warp must be complete (its source is this CTA's
-    // shared memory and its target the caller's workspace) before the kernel ends.
-    if (lane == 0) bulk_wait0();
-    __syncwarp();
     tc_fence_before();
     __syncthreads();
   }

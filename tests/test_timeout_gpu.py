@@ -103,3 +103,42 @@ def test_stall_hook_arguments():
     with pytest.raises(fa.FAError):
         fa.debug_stall_producer(True, 100001)
     fa.debug_stall_producer(False)
+
+
+# The fused backward (head dims 64, 128) and the head-dim-256 kernels: which of their
+# waits gives up first depends on timing, so any site of the kernel is accepted.
+FUSED_SITES = set(range(301, 317))
+FWD256_SITES = set(range(401, 413))
+BWD256_SITES = set(range(501, 515))
+
+
+@pytest.mark.parametrize("d,causal", [(64, True), (128, False), (256, True)])
+def test_fused_kernels_end_through_timeout(cuda_device, d, causal):
+    B, H, N = 2, 2, 640
+    t = _inputs(B, H, N, d, cuda_device, seed=6)
+    sc = 1.0 / math.sqrt(d)
+    assert fa.device_status() == (0, 0)
+    o, lse = fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc)
+    ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d, deterministic=False), dtype=torch.uint8, device=cuda_device)
+    dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["q"])
+    with _stalled(2000):
+        if d == 256:
+            fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc, out=torch.empty_like(o),
+                       lse=torch.empty_like(lse))
+            st_fwd = fa.device_status()
+        fa.bwd_fused_preprocess(o, t["do"], lse, ws)
+        fa.bwd_fused_main(t["q"], t["k"], t["v"], t["do"], dk, dv, ws, causal=causal, scale=sc)
+        st_bwd = fa.device_status()
+    if d == 256:
+        assert st_fwd[0] == TIMEOUT and st_fwd[1] in FWD256_SITES, st_fwd
+    assert st_bwd[0] == TIMEOUT and st_bwd[1] in (BWD256_SITES if d == 256 else FUSED_SITES), st_bwd
+    # Normal launches again, in the same context: parity with the oracle.
+    o, lse = fa.forward(t["q"], t["k"], t["v"], causal=causal, scale=sc)
+    dq, dk, dv = fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], causal=causal, scale=sc, deterministic=False)
+    assert fa.device_status() == (0, 0)
+    for b, h in ((0, 0), (B - 1, H - 1)):
+        sl = lambda x: x[b:b + 1, h:h + 1].cpu()
+        ref = oracle.attn_bwd_ref(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["do"]), causal, sc, None, 128)
+        assert_fwd_close(sl(o), sl(lse), ref["o"], ref["lse"], f"after timeout d={d} causal={causal}")
+        for name, g in (("q", dq), ("k", dk), ("v", dv)):
+            assert_grad_close(sl(g), ref["d" + name], name, f"after timeout d={d} causal={causal}")
