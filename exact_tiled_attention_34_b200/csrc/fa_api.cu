@@ -772,7 +772,8 @@ fa_status launch_fused(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return FA_ERR_CUDA;
-  unsigned grid = unsigned(p.n_ktiles) * unsigned(p.BH);
+  // Causal items come in pairs of key tiles (j, n - 1 - j), one position per pair.
+  unsigned grid = unsigned(CAUSAL ? (p.n_ktiles + 1) / 2 : p.n_ktiles) * unsigned(p.BH);
   if (grid > unsigned(sms)) grid = unsigned(sms);  // persistent: at most one CTA per SM
   kernel<<<grid, fa::kFusedThreads, smem, stream>>>(mq, mk, mv, mdo, macc, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;

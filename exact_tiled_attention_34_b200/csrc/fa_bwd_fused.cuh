@@ -136,6 +136,38 @@ __device__ __forceinline__ void mma_dq_ss(uint32_t tm, uint32_t a_ds, uint32_t b
            k > 0 ? 1u : 0u);
 }
 
+// The items one CTA visits, in order. Causal: key tiles j and n - 1 - j of one head form
+// a pair that costs n + 1 query tiles in all, so pairs are uniform and need no
+// costliest-first order; pairs are dealt head-major by item_position's alternating deal,
+// so the CTAs at work at any time hold the pairs of a few heads, and those heads' Q, dO
+// and dQ accumulator rows stay in L2 while all their key tiles add into them (dealing
+// single items costliest first spreads every head over the whole run). A middle tile
+// (n odd) is a pair of one item. Not causal: bwd_item's head-major order.
+template <bool CAUSAL>
+struct FusedWalk {
+  int n, BH;
+  int k = 0;         // pair (or item) position of this CTA
+  bool second = false;
+  __device__ __forceinline__ bool next(BwdItem& it) {
+    if (!CAUSAL) return bwd_item<false, true>(n, BH, k++, it);
+    const int n_pairs = (n + 1) >> 1;
+    const long long pos = item_position(static_cast<long long>(n_pairs) * BH, k);
+    if (pos < 0) return false;
+    const int pr = static_cast<int>(pos % n_pairs);
+    it.bh = static_cast<int>(pos / n_pairs);
+    if (second) {
+      it.tile = n - 1 - pr;
+      second = false;
+      ++k;
+    } else {
+      it.tile = pr;
+      second = n - 1 - pr != pr;
+      if (!second) ++k;
+    }
+    return true;
+  }
+};
+
 // Register split of the 512-thread block (launched with 128 per thread, 65,536 in all):
 // the producer/MMA warpgroup drops to 96 (the issuer keeps the descriptors of five
 // products in registers), the dQ warpgroup keeps 96 (64 hold two boxes of dQ), the
@@ -223,7 +255,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       int nq = 0, ndo = 0;  // Q and dO loads issued (for the drain on abort)
       bool ok = p.stall == 0;
       BwdItem item;
-      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
+      FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+      for (int kk = 0; ok && walk.next(item); ++kk) {
         const int j = item.tile, bh = item.bh;
         const int ib = bh / p.H, ih = bh - ib * p.H;
         KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
@@ -285,7 +318,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       bool ok = true;
       int it = 0;  // query tiles processed so far (continues across items)
       BwdItem item;
-      for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
+      FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+      for (int kk = 0; ok && walk.next(item); ++kk) {
         KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
         const int kvs = kk % SKV;
         const uint32_t aK = smem_u32(sK) + kvs * Cfg::kTileBytes, aV = smem_u32(sV) + kvs * Cfg::kTileBytes;
@@ -384,7 +418,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bool ok = true;
     int it = 0;
     BwdItem item;
-    for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
+    FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+    for (int kk = 0; ok && walk.next(item); ++kk) {
       KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
       for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, it & 1, wc, kSiteFuDqFull))) {
@@ -467,7 +502,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bool ok = true;
     int it = 0;
     BwdItem item;
-    for (int kk = 0; ok && bwd_item<CAUSAL, true>(p.n_ktiles, p.BH, kk, item); ++kk) {
+    FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+    for (int kk = 0; ok && walk.next(item); ++kk) {
       const int j = item.tile;
       KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
       const bool kvalid = j * 128 + r < p.Nk;  // key rows past N_k (last tile) contribute nothing
