@@ -772,10 +772,21 @@ fa_status launch_fused(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return FA_ERR_CUDA;
-  // Causal items come in pairs of key tiles (j, n - 1 - j), one position per pair.
-  unsigned grid = unsigned(CAUSAL ? (p.n_ktiles + 1) / 2 : p.n_ktiles) * unsigned(p.BH);
-  if (grid > unsigned(sms)) grid = unsigned(sms);  // persistent: at most one CTA per SM
-  kernel<<<grid, fa::kFusedThreads, smem, stream>>>(mq, mk, mv, mdo, macc, p);
+  // Causal: deal key tiles in pairs (j, n - 1 - j), one position per pair, when the
+  // pairs leave at most 5% of the CTA rounds idle (they are of equal cost, so the last
+  // round's empty slots are the whole imbalance); else single items, costliest first.
+  fa::BwdParams q = p;
+  long long npos = static_cast<long long>(p.n_ktiles) * p.BH;
+  if (CAUSAL) {
+    const long long pairs = static_cast<long long>((p.n_ktiles + 1) / 2) * p.BH;
+    const long long slots = (pairs + sms - 1) / sms * sms;
+    if (20 * (slots - pairs) <= slots) {
+      q.paired = 1;
+      npos = pairs;
+    }
+  }
+  const unsigned grid = unsigned(npos < sms ? npos : sms);  // persistent: at most one CTA per SM
+  kernel<<<grid, fa::kFusedThreads, smem, stream>>>(mq, mk, mv, mdo, macc, q);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

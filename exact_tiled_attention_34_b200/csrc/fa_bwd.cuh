@@ -128,6 +128,7 @@ struct BwdParams {
   int off;              // N_k - N_q: with the causal mask key j is visible to query i iff j <= i + off
   int ds;               // head dim as stored (row length of q, k, v, dO, dq, dk, dv): D, or 96 with D = 128
   int v8;               // 1: the gradient outputs are 32-byte aligned (32-byte row stores)
+  int paired = 0;       // fused backward, causal: key tiles dealt in pairs (set by the launcher)
   float scale;          // softmax scale
 };
 

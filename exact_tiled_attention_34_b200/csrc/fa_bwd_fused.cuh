@@ -136,20 +136,22 @@ __device__ __forceinline__ void mma_dq_ss(uint32_t tm, uint32_t a_ds, uint32_t b
            k > 0 ? 1u : 0u);
 }
 
-// The items one CTA visits, in order. Causal: key tiles j and n - 1 - j of one head form
-// a pair that costs n + 1 query tiles in all, so pairs are uniform and need no
-// costliest-first order; pairs are dealt head-major by item_position's alternating deal,
-// so the CTAs at work at any time hold the pairs of a few heads, and those heads' Q, dO
-// and dQ accumulator rows stay in L2 while all their key tiles add into them (dealing
-// single items costliest first spreads every head over the whole run). A middle tile
-// (n odd) is a pair of one item. Not causal: bwd_item's head-major order.
+// The items one CTA visits, in order. Causal and `paired`: key tiles j and n - 1 - j of
+// one head form a pair that costs n + 1 query tiles in all, so pairs are uniform and
+// need no costliest-first order; pairs are dealt head-major by item_position's
+// alternating deal, so the CTAs at work at any time hold the pairs of a few heads, and
+// those heads' Q, dO and dQ accumulator rows stay in L2 while all their key tiles add
+// into them (dealing single items costliest first spreads every head over the whole
+// run). A middle tile (n odd) is a pair of one item. The launcher pairs only when the
+// pairs fill the last round of CTAs well; otherwise (and when not causal) bwd_item's
+// order.
 template <bool CAUSAL>
 struct FusedWalk {
-  int n, BH;
+  int n, BH, paired;
   int k = 0;         // pair (or item) position of this CTA
   bool second = false;
   __device__ __forceinline__ bool next(BwdItem& it) {
-    if (!CAUSAL) return bwd_item<false, true>(n, BH, k++, it);
+    if (!CAUSAL || !paired) return bwd_item<CAUSAL, true>(n, BH, k++, it);
     const int n_pairs = (n + 1) >> 1;
     const long long pos = item_position(static_cast<long long>(n_pairs) * BH, k);
     if (pos < 0) return false;
@@ -255,7 +257,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       int nq = 0, ndo = 0;  // Q and dO loads issued (for the drain on abort)
       bool ok = p.stall == 0;
       BwdItem item;
-      FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+      FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH, p.paired};
       for (int kk = 0; ok && walk.next(item); ++kk) {
         const int j = item.tile, bh = item.bh;
         const int ib = bh / p.H, ih = bh - ib * p.H;
@@ -318,7 +320,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       bool ok = true;
       int it = 0;  // query tiles processed so far (continues across items)
       BwdItem item;
-      FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+      FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH, p.paired};
       for (int kk = 0; ok && walk.next(item); ++kk) {
         KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
         const int kvs = kk % SKV;
@@ -418,7 +420,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bool ok = true;
     int it = 0;
     BwdItem item;
-    FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+    FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH, p.paired};
     for (int kk = 0; ok && walk.next(item); ++kk) {
       KeySched<CAUSAL, SPARSE, XQK> sch{item.tile, p.n_tiles, p.n_ktiles, off_, p.tile_mask};
       for (int i = sch.first(); i >= 0; i = sch.next(i), ++it) {
@@ -502,7 +504,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bool ok = true;
     int it = 0;
     BwdItem item;
-    FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH};
+    FusedWalk<CAUSAL> walk{p.n_ktiles, p.BH, p.paired};
     for (int kk = 0; ok && walk.next(item); ++kk) {
       const int j = item.tile;
       KeySched<CAUSAL, SPARSE, XQK> sch{j, p.n_tiles, p.n_ktiles, off_, p.tile_mask};

@@ -89,6 +89,16 @@ def test_many_items_per_cta(cuda_device, causal, d):
     _full_check(2, 80, 640, d, causal, cuda_device, seed=351 + d)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [300, 1000])
+def test_paired_causal_items(cuda_device, N, d):
+    """Causal items dealt as pairs of key tiles (j, n - 1 - j): with one head per SM the
+    pairs fill every CTA round, so the launcher pairs them; N = 300 has a middle tile
+    (3 key tiles) that forms a pair of its own."""
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    _full_check(1, sms, N, d, True, cuda_device, seed=371 + d, heads=[(0, 0), (0, sms // 2), (0, sms - 1)])
+
+
 def test_head_dim_96(cuda_device):
     _full_check(1, 3, 384, 96, True, cuda_device, seed=361)
     _full_check(1, 2, 256, 96, False, cuda_device, seed=362)
