@@ -55,7 +55,7 @@ def workload(name: str):
         B, H = sweep_shape(N, d)
         causal = len(parts) > 3 and parts[3] == "causal"
         return dict(B=B, H=H, N=N, Nk=N, d=d, variants=[("causal" if causal else "noncausal", causal, None)],
-                    do_scale=0.5)
+                    do_scale=0.5, dropout_p=0.0)
     w = WORKLOADS[name]
     variants = []
     if "sparse_density" in w:

@@ -147,7 +147,9 @@ def attn_dropout_bwd_ref(q, k, v, do, p: float, seed: int, offset: int = 0, caus
                          scale: float | None = None, bh0: int = 0):
     """Gradients of L = sum(O * dO) with dropout (the mask fixed by seed and offset).
     Returns dq, dk, dv, the forward's o and lse, and D = sum_j P_ij dP_ij. bh0: as for
-    ``dropout_keep_mask``."""
+    ``dropout_keep_mask``. Also ``pv_abs`` = sum_j P~_ij |V_jc| (P~ the dropped, rescaled
+    probabilities), the scale of the rounding error a bf16 P~ puts into O_ic, for the
+    tests' element-wise error bounds."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, N, d = q.shape
     n_k = k.shape[2]
@@ -156,7 +158,8 @@ def attn_dropout_bwd_ref(q, k, v, do, p: float, seed: int, offset: int = 0, caus
     t = keep_threshold(p)
     keep = dropout_keep_mask(B, H, N, n_k, p, seed, offset, bh0=bh0)
     out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
-           "o": np.zeros((B, H, N, v.shape[-1])), "lse": np.zeros((B, H, N)), "D": np.zeros((B, H, N))}
+           "o": np.zeros((B, H, N, v.shape[-1])), "lse": np.zeros((B, H, N)), "D": np.zeros((B, H, N)),
+           "pv_abs": np.zeros((B, H, N, v.shape[-1]))}
     for b in range(B):
         for h in range(H):
             s = attn_scores_ref(q[b, h], k[b, h], scale, causal)
@@ -172,6 +175,7 @@ def attn_dropout_bwd_ref(q, k, v, do, p: float, seed: int, offset: int = 0, caus
             out["dk"][b, h] = scale * (ds.T @ q[b, h])
             out["dv"][b, h] = pd.T @ do[b, h]
             out["o"][b, h] = o
+            out["pv_abs"][b, h] = pd @ np.abs(v[b, h])
             out["lse"][b, h] = lse
             out["D"][b, h] = D
     return out

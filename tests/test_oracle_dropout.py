@@ -186,6 +186,19 @@ def pin_threshold_rule(mod):
             mod.keep_threshold(bad)
 
 
+def pin_pv_abs_bounds_o(mod):
+    """sum_j P~_ij |V_jc| bounds |O_ic| (triangle inequality) and equals O_ic when V >= 0;
+    with p = 0 it is plain attention's output on |V|."""
+    q, k, v, do = (_rand((1, 2, 7, 4), s) for s in (71, 72, 73, 74))
+    r = mod.attn_dropout_bwd_ref(q, k, v, do, 0.3, 99, 1, True, 0.6)
+    assert np.all(r["pv_abs"] >= np.abs(r["o"]) - 1e-14)
+    r_pos = mod.attn_dropout_bwd_ref(q, k, np.abs(v), do, 0.3, 99, 1, True, 0.6)
+    assert np.max(np.abs(r_pos["pv_abs"] - r_pos["o"])) < 1e-14
+    r0 = mod.attn_dropout_bwd_ref(q, k, v, do, 0.0, 99, 1, False, 0.6)
+    o_abs, _ = oracle.attn_fwd_ref(q, k, np.abs(v), False, 0.6)
+    assert np.max(np.abs(r0["pv_abs"] - o_abs)) < 1e-12
+
+
 DROPOUT_PINS = [
     pin_philox_known_answers,
     pin_golden_4x4,
@@ -196,6 +209,7 @@ DROPOUT_PINS = [
     pin_expectation_over_seeds,
     pin_threshold_rule,
     pin_head_slices_match_full,
+    pin_pv_abs_bounds_o,
 ]
 
 
