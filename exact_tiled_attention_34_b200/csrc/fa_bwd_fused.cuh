@@ -25,12 +25,12 @@
 // dS leaves the compute warps through shared memory (bf16, 128 x 128, 128-byte
 // swizzle, [query block of 64][key row][128 B]); that one buffer is the K-major A
 // operand of dK += dS^T Q and the MN-major A operand of dQ = dS K. Each dQ warp stages
-// its 32 dQ rows (fp32, 32 x 32 boxes, 4 KB each) for the reduce-add in a stage area
-// of its own (8 KB per warp); at head dim 128, where a warp has four boxes and shared
-// memory has no room for 16 KB per warp, its first two boxes go to 8 KB of the dS buffer
-// (free once dQ's product is done) and the compute warps write the next dS only once
-// those two copies have read their stages. With the drain in warps of its own, the
-// compute warps go from one tile's dS straight to the next tile's exponentials.
+// its 32 dQ rows (fp32, 32 x 32 boxes, 4 KB each) for the reduce-add in a stage area of
+// its own (8 KB per warp, two boxes); at head dim 128 a warp's other two boxes wait in
+// registers until the first two copies have read the area. With the drain in warps of
+// its own, the compute warps go from one tile's dS straight to the next tile's
+// exponentials, and at head dim 128 dQ's product goes before dK's so that dQ's columns
+// (which the next dP^T reuses) are read out while dK's product runs.
 //
 // Tensor memory (512 columns): dK | dV | X (S^T, then P^T as packed bf16) |
 // Y (dP^T; at head dim 128 also dQ) | Z (dQ at head dim 64). At head dim 128 the five
@@ -59,9 +59,7 @@ struct FusedCfg {
   static constexpr int kOffDS = kOffDO + kDoStages * kTileBytes;    // dS bf16 128 x 128 / dQ stages
   static constexpr int kOffL = kOffDS + 32768;                      // -lse log2 e rows, 2 stages
   static constexpr int kOffDr = kOffL + 1024;                       // D rows, 2 stages
-  // dQ stage area, 8 KB per dQ warp: all of a warp's boxes at head dim 64, the last two
-  // of its four at head dim 128 (the first two are staged in the dS buffer).
-  static constexpr bool kStageInDs = (D == 128);
+  // dQ stage area, 8 KB per dQ warp (two 4 KB boxes at a time).
   static constexpr int kOffStage = kOffDr + 1024;
   static constexpr int kOffBar = kOffStage + 32768;
   // Barriers (well under 256 bytes), plus 1 KB of alignment slack at head dim 64. At head
@@ -90,11 +88,10 @@ struct FusedBars {
   uint64_t do_empty[2];
   uint64_t s_full;
   uint64_t dp_full;
-  uint64_t dq_full;      // dQ_i's product is done (and with it every read of dS_i)
+  uint64_t dq_full;      // dQ_i's product is done
   uint64_t p_ready;      // 256 arrivals: P^T is in tensor memory
   uint64_t ds_ready;     // 256: dS is in shared memory and dP^T has been read
   uint64_t dq_taken;     // 128: dQ_i has been read out of tensor memory
-  uint64_t ds_free;      // 4 (one per dQ warp): the copies staged in the dS buffer have read it (head dim 128)
   uint64_t rd_s;         // 256: both warpgroups have read S^T
   uint64_t acc_done;
   uint64_t acc_empty;    // 256: the epilogue has read dK and dV
@@ -106,7 +103,7 @@ struct FusedBars {
 enum FusedSite : int {
   kSiteFuKV = 301, kSiteFuQEmpty, kSiteFuDoEmpty, kSiteFuKvEmpty, kSiteFuQFull, kSiteFuDoFull, kSiteFuPReady,
   kSiteFuDsReady, kSiteFuDqTaken, kSiteFuAcc, kSiteFuSFull, kSiteFuDpFull, kSiteFuDqFull, kSiteFuRead,
-  kSiteFuDrain, kSiteFuDsFree,
+  kSiteFuDrain,
   kSiteFuSmemAlign = 399  // reported with kStatusUnsupported: dynamic shared memory not 1024-aligned
 };
 constexpr int kStatusUnsupported = 2;  // == FA_ERR_UNSUPPORTED
@@ -226,7 +223,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->dq_taken, 128);
-    mbar_init(&bars->ds_free, 4);
     mbar_init(&bars->rd_s, 256);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->acc_empty, 256);
@@ -368,7 +364,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mma_tile_nt<D>(tmem + Cfg::kTmX, aK, aQ + ((it + 1) & 1) * Cfg::kTileBytes);
             mma_commit(&bars->s_full);
           }
-          // dK += dS^T Q_i and dQ_i = dS K_j, both reading dS from shared memory.
+          // dK += dS^T Q_i and dQ_i = dS K_j, both reading dS from shared memory (dQ first
+          // at head dim 128, where the next dP^T waits for dQ's columns to be read out).
           if (!mbar_wait(&bars->ds_ready, it & 1, wc, kSiteFuDsReady)) { ok = false; break; }
           // Head dim 64: Z may still hold the previous tile's dQ.
           if (!Cfg::kDqInY && it > 0 && !mbar_wait(&bars->dq_taken, (it - 1) & 1, wc, kSiteFuDqTaken)) {
@@ -376,9 +373,15 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             break;
           }
           tc_fence_after();
-          mma_dk_ss<D>(tmem + Cfg::kTmDK, aDS, aQ + st * Cfg::kTileBytes, !first);
-          mma_dq_ss<D>(tmem + Cfg::kTmDQ, aDS, aK);
-          mma_commit(&bars->dq_full);
+          if constexpr (Cfg::kDqInY) {
+            mma_dq_ss<D>(tmem + Cfg::kTmDQ, aDS, aK);
+            mma_commit(&bars->dq_full);
+            mma_dk_ss<D>(tmem + Cfg::kTmDK, aDS, aQ + st * Cfg::kTileBytes, !first);
+          } else {
+            mma_dk_ss<D>(tmem + Cfg::kTmDK, aDS, aQ + st * Cfg::kTileBytes, !first);
+            mma_dq_ss<D>(tmem + Cfg::kTmDQ, aDS, aK);
+            mma_commit(&bars->dq_full);
+          }
           mma_commit(&bars->q_empty[st]);
           if (in < 0) mma_commit(&bars->kv_empty[kvs]);  // every product reading K_j, V_j is issued
           if (in >= 0) {
@@ -445,26 +448,25 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (lane == 0) tma_reduce_add_3d(&tm_dqacc, stage, b * 32, y0, item.bh);
         };
         uint8_t* area = smem + Cfg::kOffStage + quarter * 8192;
-        if constexpr (Cfg::kStageInDs) {
-          // Boxes 0 and 1 into this warp's 8 KB of the dS buffer (free: dQ's product, the
-          // last reader of dS, is done), committed as a group of their own so that the
-          // buffer is released as soon as they are read; boxes 2 and 3 into the stage area.
-          uint8_t* in_ds = sDS + quarter * 8192;
+        if constexpr (D == 128) {
+          // Boxes 0 and 1 through the stage area; boxes 2 and 3 stay in registers (dQ's
+          // columns are released as soon as they are loaded) until those copies have read
+          // the area.
           tmem_ld64(trow + Cfg::kTmDQ, v);
           tmem_wait_ld();
-          stage_box(0, 0, in_ds);
-          stage_box(1, 1, in_ds + 4096);
+          stage_box(0, 0, area);
+          stage_box(1, 1, area + 4096);
           if (lane == 0) bulk_commit();
           tmem_ld64(trow + Cfg::kTmDQ + 64, v);
           tmem_wait_ld();
           tc_fence_before();
-          mbar_arrive(&bars->dq_taken);  // every column of dQ_t is in registers: its columns are free
+          mbar_arrive(&bars->dq_taken);
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
           stage_box(2, 0, area);
           stage_box(3, 1, area + 4096);
           if (lane == 0) {
             bulk_commit();
-            bulk_wait_read1();  // boxes 0 and 1 are read: the next dS may be written
-            mbar_arrive(&bars->ds_free);
             bulk_wait_read0();  // this warp's stage area may be overwritten by the next tile
           }
         } else {
@@ -577,12 +579,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
             ds[t] = pack_bf16(v.x, v.y);
           }
-        }
-        // Head dim 128: the dS buffer may still be read by the previous tile's copies.
-        if (Cfg::kStageInDs && it > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(&bars->ds_free, (it - 1) & 1, wc, kSiteFuDsFree))) {
-          ok = false;
-          break;
         }
         {
           uint4* d4 = reinterpret_cast<uint4*>(my_ds);
