@@ -92,7 +92,6 @@ struct FusedBars {
   uint64_t p_ready;      // 256 arrivals: P^T is in tensor memory
   uint64_t ds_ready;     // 256: dS is in shared memory and dP^T has been read
   uint64_t dq_taken;     // 128: dQ_i has been read out of tensor memory
-  uint64_t rd_s;         // 256: both warpgroups have read S^T
   uint64_t acc_done;
   uint64_t acc_empty;    // 256: the epilogue has read dK and dV
   uint64_t mma_done;
@@ -102,7 +101,7 @@ struct FusedBars {
 
 enum FusedSite : int {
   kSiteFuKV = 301, kSiteFuQEmpty, kSiteFuDoEmpty, kSiteFuKvEmpty, kSiteFuQFull, kSiteFuDoFull, kSiteFuPReady,
-  kSiteFuDsReady, kSiteFuDqTaken, kSiteFuAcc, kSiteFuSFull, kSiteFuDpFull, kSiteFuDqFull, kSiteFuRead,
+  kSiteFuDsReady, kSiteFuDqTaken, kSiteFuAcc, kSiteFuSFull, kSiteFuDpFull, kSiteFuDqFull,
   kSiteFuDrain,
   kSiteFuSmemAlign = 399  // reported with kStatusUnsupported: dynamic shared memory not 1024-aligned
 };
@@ -119,6 +118,19 @@ __device__ __forceinline__ void mma_dk_ss(uint32_t tm, uint32_t a_ds, uint32_t b
     mma_ss(tm, sdesc_sw128(a_ds + aoff, 16, 1024), sdesc_sw128(b_q + k * 2048, 16384, 1024), id,
            (acc || k > 0) ? 1u : 0u);
   }
+}
+
+// dV += P^T dO_i: A = P^T packed bf16 in tensor memory, where compute warpgroup h left
+// its 64 queries in the first 32 of its own 64 score columns (X + 64h), so that no
+// warpgroup overwrites scores the other has yet to read; B = dO_i (N-major), 8 steps of
+// 16 queries.
+template <int D>
+__device__ __forceinline__ void mma_dv_ts(uint32_t tm, uint32_t a_tm, uint32_t b, bool acc) {
+  constexpr uint32_t id = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    mma_ts(tm, a_tm + (k >> 2) * 64 + (k & 3) * 8, sdesc_sw128(b + k * 2048, FusedCfg<D>::kBlockBytes, 1024), id,
+           (acc || k > 0) ? 1u : 0u);
 }
 
 // dQ = dS K_j: A = dS from the same buffer read MN-major (query rows contiguous in
@@ -223,7 +235,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->dq_taken, 128);
-    mbar_init(&bars->rd_s, 256);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
@@ -353,7 +364,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             break;
           }
           tc_fence_after();
-          mma_tile_tn<D>(tmem + Cfg::kTmDV, tmem + Cfg::kTmX, aDO + ds_ * Cfg::kTileBytes, !first);
+          mma_dv_ts<D>(tmem + Cfg::kTmDV, tmem + Cfg::kTmX, aDO + ds_ * Cfg::kTileBytes, !first);
           mma_commit(&bars->do_empty[ds_]);
           if (in >= 0) {
             if (!mbar_wait(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1, wc, kSiteFuQFull)) {
@@ -535,16 +546,12 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           uint32_t raw[64];
           tmem_ld64(trow + Cfg::kTmX + h * 64, raw);
           tmem_wait_ld();
-          mbar_arrive(&bars->rd_s);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_s, it & 1, wc, kSiteFuRead))) {
-            ok = false;
-            break;
-          }
           const uint64_t c2v = f2(c2, c2);
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             const int c0 = 2 * t;
-            const float2 nl = *reinterpret_cast<const float2*>(lse2 + c0);
+            const float4 n4 = *reinterpret_cast<const float4*>(lse2 + (c0 & ~3));
+            const float2 nl = (t & 1) ? make_float2(n4.z, n4.w) : make_float2(n4.x, n4.y);
             uint64_t pv = ex2_split_x2<PolyShare<D>::kDkdv>(
                 f2_fma(f2(__uint_as_float(raw[c0]), __uint_as_float(raw[c0 + 1])), c2v, f2(nl.x, nl.y)), t);
             if (diag) {
@@ -555,7 +562,9 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             pk[t] = kvalid ? pack_bf16(v.x, v.y) : 0u;
           }
         }
-        tmem_st32(trow + Cfg::kTmX + h * 32, pk);
+        // P^T over the first half of this warpgroup's own score columns: this thread has read
+        // its row of them, and no other thread reads this row.
+        tmem_st32(trow + Cfg::kTmX + h * 64, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
@@ -573,7 +582,8 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             const float2 pp = unpack_bf16(pk[t]);
-            const float2 dd = *reinterpret_cast<const float2*>(Dr + 2 * t);
+            const float4 d4 = *reinterpret_cast<const float4*>(Dr + ((2 * t) & ~3));
+            const float2 dd = (t & 1) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
             const uint64_t diff =
                 f2_sub(f2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), f2(dd.x, dd.y));
             const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
