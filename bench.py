@@ -456,41 +456,79 @@ def run_ours(args, wl_name, wl):
                 "traffic": profiled_traffic(main_kernel, wl_name)}
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
+    # Three streams, as a user pipelines host data through the library: step s's inputs go
+    # host -> device on a copy stream while step s - 1 computes, and its results go device
+    # -> host on a second copy stream while step s + 1 computes. Every step's copies are
+    # inside the timed region; two sets of device buffers alternate between steps, and
+    # events order each reuse after the copies that read or write the set.
     e2e_steps = max(3, min(K, 10))
     pin = {k: v.pin_memory() for k, v in host.items()}
-    res_host = {label: {n: torch.empty(outs[label][n].shape, dtype=outs[label][n].dtype).pin_memory()
-                        for n in ("o", "lse", "dq", "dk", "dv")} for (label, _, _) in wl["variants"]}
+    labels = [label for (label, _, _) in wl["variants"]]
+    res_host = [{label: {n: torch.empty(outs[label][n].shape, dtype=outs[label][n].dtype).pin_memory()
+                         for n in ("o", "lse", "dq", "dk", "dv")} for label in labels} for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = sum(v.numel() * v.element_size() for r in res_host.values() for v in r.values())
+    d2h = sum(v.numel() * v.element_size() for v in res_host[0][labels[0]].values()) * len(labels)
+    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in pin.items()} for _ in range(2)]
+    dev_out = [{label: {n: torch.empty_like(outs[label][n]) for n in ("o", "lse", "dq", "dk", "dv")}
+                for label in labels} for _ in range(2)]
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready = [ev() for _ in range(2)]    # set's inputs are on the device
+    in_free = [ev() for _ in range(2)]     # compute is done reading the set's inputs
+    out_ready = [ev() for _ in range(2)]   # compute wrote the set's outputs
+    out_free = [ev() for _ in range(2)]    # the set's outputs are on the host
+    for e in in_free + out_free:
+        e.record(stream)
 
-    def e2e_step():
-        x = {k: v.to(dev, non_blocking=True) for k, v in pin.items()}
+    def e2e_step(s):
+        b = s & 1
+        with torch.cuda.stream(s_h2d):
+            s_h2d.wait_event(in_free[b])
+            for k, v in pin.items():
+                dev_in[b][k].copy_(v, non_blocking=True)
+            in_ready[b].record(s_h2d)
+        stream.wait_event(in_ready[b])
+        stream.wait_event(out_free[b])
+        x, y = dev_in[b], dev_out[b]
         for (label, causal, _) in wl["variants"]:
-            k = kinds[label]
+            k, r = kinds[label], y[label]
             if k["mask"] is None:
-                o, lse = fa.forward(x["q"], x["k"], x["v"], causal=causal, scale=sc)
-                g = fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, scale=sc, workspace=ws,
-                                deterministic=not fused)
+                fa.forward(x["q"], x["k"], x["v"], causal=causal, scale=sc, out=r["o"], lse=r["lse"])
+                fa.backward(x["q"], x["k"], x["v"], r["o"], r["lse"], x["do"], causal=causal, scale=sc,
+                            workspace=ws, grads=(r["dq"], r["dk"], r["dv"]), deterministic=not fused)
             else:
-                o, lse = fa.forward_blocksparse(x["q"], x["k"], x["v"], k["mask"], scale=sc)
-                g = fa.backward_blocksparse(x["q"], x["k"], x["v"], o, lse, x["do"], k["mask"], scale=sc,
-                                            workspace=ws, deterministic=not fused)
-            for n, v in zip(("o", "lse", "dq", "dk", "dv"), (o, lse) + tuple(g)):
-                res_host[label][n].copy_(v, non_blocking=True)
+                fa.forward_blocksparse(x["q"], x["k"], x["v"], k["mask"], scale=sc, out=r["o"], lse=r["lse"])
+                fa.backward_blocksparse(x["q"], x["k"], x["v"], r["o"], r["lse"], x["do"], k["mask"], scale=sc,
+                                        workspace=ws, grads=(r["dq"], r["dk"], r["dv"]),
+                                        deterministic=not fused)
+        in_free[b].record(stream)
+        out_ready[b].record(stream)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(out_ready[b])
+            for label in labels:
+                for n in ("o", "lse", "dq", "dk", "dv"):
+                    res_host[b][label][n].copy_(y[label][n], non_blocking=True)
+            out_free[b].record(s_d2h)
 
-    for _ in range(2):
-        e2e_step()
+    for s_ in range(2):
+        e2e_step(s_)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_h2d.wait_event(e0)  # the first copy starts inside the timed region
+    for s_ in range(e2e_steps):
+        e2e_step(s_)
+    stream.wait_event(out_free[(e2e_steps - 1) & 1])  # the last results are on the host
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = job_throughput(world, step_flops, e2e_steps, e2e_ms)
+    # The device-side results of the last step are the ones the host copy holds.
+    last = res_host[(e2e_steps - 1) & 1][labels[0]]
+    if not torch.isfinite(last["dq"].float()).all():
+        raise SystemExit("end-to-end step produced non-finite gradients")
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOPs/s", "n_gpus": world, "steps": K,
@@ -515,7 +553,8 @@ def run_ours(args, wl_name, wl):
         "wall_s_timed_region": round(wall, 4),
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPs/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "api": "exact_tiled_attention_34_b200.forward/backward (C ABI), pinned host buffers"},
+                "api": "exact_tiled_attention_34_b200.forward/backward (C ABI), pinned host buffers; "
+                       "H2D, compute and D2H on three streams, next step's inputs copied during this step"},
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
