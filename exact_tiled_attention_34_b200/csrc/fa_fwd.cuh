@@ -393,7 +393,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t qa = sQa + i * Cfg::kTileBytes;
         const uint32_t ka = sKa + st * Cfg::kTileBytes;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < DS / 16; ++k) {  // head dim 96: columns 96..127 of the tiles are zeros
           const uint32_t off = (k >> 2) * Cfg::kBlockBytes + (k & 3) * 32;
           mma_ss(tmem + Cfg::tm_s(i), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS,
                  k > 0);
