@@ -257,9 +257,12 @@ __device__ __forceinline__ void mma_tile_nt(uint32_t tm, uint32_t a, uint32_t b)
 template <int D>
 __device__ __forceinline__ void mma_tile_tn(uint32_t tm, uint32_t a_tm, uint32_t b, bool acc) {
   constexpr uint32_t id = idesc_bf16_f32(128, D, 0, 1);
+  // Compute warpgroup h leaves its 64 queries' (or keys') packed values, 32 columns, at
+  // the start of its own 64-column half of the operand region: k-steps 0..3 read
+  // a_tm + 0..31, k-steps 4..7 read a_tm + 64..95.
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    mma_ts(tm, a_tm + k * 8, sdesc_sw128(b + k * 2048, BwdCfg<D>::kBlockBytes, 1024), id,
+    mma_ts(tm, a_tm + (k >> 2) * 64 + (k & 3) * 8, sdesc_sw128(b + k * 2048, BwdCfg<D>::kBlockBytes, 1024), id,
            (acc || k > 0) ? 1u : 0u);
 }
 
@@ -339,8 +342,6 @@ struct DkdvBars {
   uint64_t acc_done;
   uint64_t acc_empty;  // the epilogue has read dK and dV (the next item may overwrite them)
   uint64_t mma_done;
-  uint64_t rd_s;   // both compute warpgroups have read S^T of this tile
-  uint64_t rd_dp;  // ... and dP^T
   uint32_t tmem_base;
   int abort;
 };
@@ -382,8 +383,6 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
-    mbar_init(&bars->rd_s, 256);
-    mbar_init(&bars->rd_dp, 256);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -570,13 +569,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           uint32_t raw[64];
           tmem_ld64(trow + Cfg::kTmS + h * 64, raw);
           tmem_wait_ld();
-          // The packed P^T of query q goes to column q / 2: warpgroup 1 writes columns
-          // 32..63, which hold scores warpgroup 0 reads. Both finish reading first.
-          mbar_arrive(&bars->rd_s);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_s, it & 1, wc, kSiteBwdRead))) {
-            ok = false;
-            break;
-          }
+          // The packed P^T of this warpgroup's 64 queries goes to the first 32 of its own 64
+          // score columns: this thread has read its row of them, and no other thread reads
+          // this row.
           const uint64_t c2v = f2(c2, c2);
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
@@ -601,9 +596,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const float2 w = drop_pair(pp.x, pp.y, kb[t >> 4] >> ((2 * t) & 31), p.drop.rs);
             pd[t] = pack_bf16(w.x, w.y);
           }
-          tmem_st32(trow + Cfg::kTmS + h * 32, pd);
+          tmem_st32(trow + Cfg::kTmS + h * 64, pd);
         } else {
-          tmem_st32(trow + Cfg::kTmS + h * 32, pk);
+          tmem_st32(trow + Cfg::kTmS + h * 64, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -618,11 +613,6 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           uint32_t dpr[64];
           tmem_ld64(trow + Cfg::kTmDP + h * 64, dpr);
           tmem_wait_ld();
-          mbar_arrive(&bars->rd_dp);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
-            ok = false;
-            break;
-          }
           uint32_t ds[32];
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
@@ -639,7 +629,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
             ds[t] = pack_bf16(v.x, v.y);
           }
-          tmem_st32(trow + Cfg::kTmDP + h * 32, ds);
+          tmem_st32(trow + Cfg::kTmDP + h * 64, ds);  // over this warpgroup's own dP^T columns
         }
         tmem_wait_st();
         tc_fence_before();
@@ -692,7 +682,6 @@ struct DqBars {
   uint64_t acc_done;
   uint64_t acc_empty;  // the epilogue has read dQ (the next item may overwrite it)
   uint64_t mma_done;
-  uint64_t rd_dp;
   uint32_t tmem_base;
   int abort;
 };
@@ -732,7 +721,6 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
-    mbar_init(&bars->rd_dp, 256);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -944,11 +932,6 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           uint32_t dpr[64];
           tmem_ld64(trow + Cfg::kQTmDP + h * 64, dpr);
           tmem_wait_ld();
-          mbar_arrive(&bars->rd_dp);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_dp, it & 1, wc, kSiteBwdRead))) {
-            ok = false;
-            break;
-          }
           const uint64_t dv2 = f2(Dv, Dv);
           uint32_t ds[32];
 #pragma unroll
@@ -965,7 +948,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float2 v = f2_split(f2_mul(f2(pp.x, pp.y), diff));
             ds[t] = pack_bf16(v.x, v.y);
           }
-          tmem_st32(trow + Cfg::kQTmDP + h * 32, ds);
+          tmem_st32(trow + Cfg::kQTmDP + h * 64, ds);  // over this warpgroup's own dP columns
         }
         tmem_wait_st();
         tc_fence_before();
