@@ -48,7 +48,7 @@ struct Bwd256Bars {
   uint64_t q_full, q_empty;    // Q sub-tile + row arrays; empty: S^T and dK done with it
   uint64_t do_full, do_empty;  // empty: dP^T and dV done with it
   uint64_t s_full, dp_full, dq_full;
-  uint64_t p_ready, ds_ready, dq_taken, rd_s;  // 256 arrivals
+  uint64_t p_ready, ds_ready, dq_taken;  // 256 arrivals
   uint64_t acc_done, acc_empty;                // acc_empty: 256
   uint64_t pair[4];   // 64 arrivals: both warps of a lane quarter are done with their dQ staging
   uint64_t mma_done;
@@ -128,7 +128,6 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->dq_taken, 256);
-    mbar_init(&bars->rd_s, 256);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->acc_empty, 256);
     for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 64);
@@ -250,7 +249,7 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           // dV_c += P^T dO[:, c]   (P^T packed in X; dO column blocks 2c, 2c + 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_ts(tmem + Cfg::kTmDV, tmem + Cfg::kTmX + k * 8,
+            mma_ts(tmem + Cfg::kTmDV, tmem + Cfg::kTmX + (k >> 1) * 32 + (k & 1) * 8,  // P^T of warpgroup k / 2
                    sdesc_sw128(aDO + 2 * c * Cfg::kSubBlock + k * 2048, Cfg::kSubBlock, 1024), idTN,
                    (!first || k > 0) ? 1u : 0u);
           mma_commit(&bars->do_empty);
@@ -369,11 +368,6 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           uint32_t raw[32];
           tmem_ld32(trow + Cfg::kTmX + h * 32, raw);
           tmem_wait_ld();
-          mbar_arrive(&bars->rd_s);
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->rd_s, n & 1, wc, kSiteB256Read))) {
-            ok = false;
-            break;
-          }
           const uint64_t c2v = f2(c2, c2);
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
@@ -389,7 +383,9 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             pk[t] = kvalid ? pack_bf16(x.x, x.y) : 0u;
           }
         }
-        tmem_st16(trow + Cfg::kTmX + h * 16, pk);
+        // P^T over the first half of this warpgroup's own 32 score columns: this thread has
+        // read its row of them, and no other thread reads this row.
+        tmem_st16(trow + Cfg::kTmX + h * 32, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
