@@ -461,7 +461,7 @@ def run_ours(args, wl_name, wl):
     # -> host on a second copy stream while step s + 1 computes. Every step's copies are
     # inside the timed region; two sets of device buffers alternate between steps, and
     # events order each reuse after the copies that read or write the set.
-    e2e_steps = max(3, min(K, 30))  # enough steps that the pipeline's fill and drain matter little
+    e2e_steps = max(3, min(K, 30))
     pin = {k: v.pin_memory() for k, v in host.items()}
     labels = [label for (label, _, _) in wl["variants"]]
     res_host = [{label: {n: torch.empty(outs[label][n].shape, dtype=outs[label][n].dtype).pin_memory()
