@@ -1,0 +1,82 @@
+"""The persistent kernels' work schedules, restated in Python from their definitions
+(csrc/fa_ptx.cuh item_position, csrc/fa_bwd.cuh bwd_item, csrc/fa_bwd_fused.cuh FusedWalk,
+csrc/fa_api.cu launch_fused) and checked for the properties the kernels rely on: every
+(batch*head, tile) item is visited by exactly one CTA, paired causal items all cost the
+same, and the launcher pairs only when the pairs fill the last round of CTAs."""
+import itertools
+
+import pytest
+
+
+def item_position(n_items, k, grid, cta):
+    # round k deals positions k*G .. k*G + G - 1, in alternating direction
+    pos = k * grid + ((grid - 1 - cta) if (k & 1) else cta)
+    return pos if pos < n_items else -1
+
+
+def bwd_item(causal, n, bh_count, k, grid, cta):
+    pos = item_position(n * bh_count, k, grid, cta)
+    if pos < 0:
+        return None
+    if causal:  # costliest first across heads: tile 0 (the most query tiles) first
+        return (pos % bh_count, pos // bh_count)
+    return (pos // n, pos % n)  # head-major
+
+
+def paired_walk(n, bh_count, grid, cta):
+    """Items of one CTA when causal key tiles are dealt as pairs (j, n - 1 - j)."""
+    n_pairs = (n + 1) // 2
+    out, k = [], 0
+    while True:
+        pos = item_position(n_pairs * bh_count, k, grid, cta)
+        if pos < 0:
+            return out
+        bh, pr = pos // n_pairs, pos % n_pairs
+        out.append((bh, pr))
+        if n - 1 - pr != pr:
+            out.append((bh, n - 1 - pr))
+        k += 1
+
+
+def launcher_pairs(n, bh_count, sms):
+    """The fused launcher's rule: pair when the last round of CTAs is at least 95% full."""
+    pairs = (n + 1) // 2 * bh_count
+    slots = (pairs + sms - 1) // sms * sms
+    return 20 * (slots - pairs) <= slots
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_items_cover_every_tile_once(causal):
+    for n, bh_count, sms in itertools.product((1, 2, 5, 16, 64), (1, 3, 32), (7, 148)):
+        grid = min(n * bh_count, sms)
+        seen = []
+        for cta in range(grid):
+            k = 0
+            while (it := bwd_item(causal, n, bh_count, k, grid, cta)) is not None:
+                seen.append(it)
+                k += 1
+        assert sorted(seen) == sorted(itertools.product(range(bh_count), range(n))), (n, bh_count, sms)
+
+
+def test_paired_items_cover_every_tile_once_and_cost_the_same():
+    for n, bh_count, sms in itertools.product((1, 2, 3, 5, 16, 63, 64), (1, 3, 32), (7, 148)):
+        n_pairs = (n + 1) // 2
+        grid = min(n_pairs * bh_count, sms)
+        seen = []
+        for cta in range(grid):
+            items = paired_walk(n, bh_count, grid, cta)
+            seen += items
+        assert sorted(seen) == sorted(itertools.product(range(bh_count), range(n))), (n, bh_count, sms)
+    # with the causal mask key tile j has n - j query tiles: a pair (j, n - 1 - j) has n + 1
+    for n in (2, 16, 64):
+        assert {(n - j) + (n - (n - 1 - j)) for j in range(n // 2)} == {n + 1}
+
+
+def test_pairs_fill_the_rounds_at_the_bench_shape():
+    # B=2 H=16 N=8192: 64 key tiles, 32 pairs per head, 1024 pairs over 148 SMs (7 rounds,
+    # 12 empty slots in the last): paired. B=1 H=16 N=4096: 256 pairs, the second of two
+    # rounds 73% full: single items.
+    assert launcher_pairs(64, 32, 148)
+    assert not launcher_pairs(32, 16, 148)
+    # one head per SM always fills the rounds (the parity test that forces pairing)
+    assert launcher_pairs(3, 148, 148) and launcher_pairs(8, 148, 148)
