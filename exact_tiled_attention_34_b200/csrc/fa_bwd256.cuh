@@ -261,13 +261,13 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_ss(tmem + Cfg::kTmDK, sdesc_sw128(aDS + k * 32, 16, 1024),
                    sdesc_sw128(aQ + 2 * c * Cfg::kSubBlock + k * 2048, Cfg::kSubBlock, 1024), idTN,
                    (!first || k > 0) ? 1u : 0u);
+          mma_commit(&bars->q_empty);  // dK's product is the last to read this Q sub-tile
           // dQ^T = K[:, c]^T dS^T   (K read MN-major: head-dim rows; dS^T N-major: query columns)
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mma_ss(tmem + Cfg::kTmZ, sdesc_sw128(aK + 2 * c * Cfg::kKvBlock + k * 2048, Cfg::kKvBlock, 1024),
                    sdesc_sw128(aDS + k * 2048, 16, 1024), idQT, k > 0 ? 1u : 0u);
           mma_commit(&bars->dq_full);
-          mma_commit(&bars->q_empty);
           if (un < 0) mma_commit(&bars->kv_empty);
           if (un >= 0) {
             if (!mbar_wait(&bars->q_full, (n + 1) & 1, wc, kSiteB256QFull)) { ok = false; break; }
