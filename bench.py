@@ -220,6 +220,20 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+def use_host_cores() -> int:
+    """Let the oracle's BLAS use every core this process may run on. torch.distributed.run
+    sets OMP_NUM_THREADS=1 in each rank; the oracle runs on rank 0 alone, so without this it
+    would be timed on one core under the launcher and on all of them without it. Returns the
+    thread count BLAS reports afterwards."""
+    try:
+        from threadpoolctl import threadpool_limits
+        n = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+        threadpool_limits(limits=n, user_api="blas")
+    except Exception:
+        pass
+    return blas_threads()
+
+
 _HOST_INPUTS = {}
 
 
@@ -266,6 +280,7 @@ def run_reference(args, wl_name, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    use_host_cores()
     budget = 1.0  # seconds of oracle work per step
     for _ in range(args.warmup):
         cpu_oracle_sample(wl, budget)
@@ -558,6 +573,7 @@ def run_ours(args, wl_name, wl):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        use_host_cores()
         v, desc, el = cpu_oracle_sample(wl, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOPs/s", "cores": blas_threads(),
                                 "kind": "oracle", "sample": desc}

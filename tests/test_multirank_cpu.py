@@ -1,7 +1,12 @@
 """The N > 1 path of bench.py on CPU: two gloo ranks check the per-rank input seeds,
-the max-over-ranks reduction of the device time and the whole-job throughput."""
+the max-over-ranks reduction of the device time and the whole-job throughput; the
+reference arm is launched through torch.distributed.run with two ranks."""
+import json
 import os
+import signal
 import socket
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -56,3 +61,29 @@ def test_single_process_helpers():
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.job_throughput(1, 2e12, 4, 8.0) == pytest.approx(1000.0)
     assert bench.rank_seed(0) != bench.rank_seed(1)
+
+
+def test_reference_arm_under_the_launcher():
+    """bench.py --impl reference launched as for N > 1 GPUs (it needs none): rank 0 alone
+    prints one line, timed on all the cores it may use although the launcher sets
+    OMP_NUM_THREADS=1; the other rank exits 0 without work."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    proc = subprocess.Popen(cmd, cwd=root, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True,
+                            start_new_session=True)
+    try:
+        out, err = proc.communicate(timeout=240)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGKILL)
+        proc.communicate()
+        raise
+    assert proc.returncode == 0, err[-2000:]
+    lines = [json.loads(ln) for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    ncpu = len(os.sched_getaffinity(0))
+    assert line["cpu_baseline"]["cores"] > 1 or ncpu == 1, line["cpu_baseline"]
