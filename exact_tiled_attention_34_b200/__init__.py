@@ -157,6 +157,31 @@ def _check_qkv(q, k, v, *qlike, layout="bhnd"):
         raise ValueError("q and k must agree in batch, heads and head dim")
 
 
+def _check_buffer(t, shape, dtype, device, what):
+    """A caller-supplied output, row array or workspace: contiguous, of `dtype`, on
+    `device` and (unless shape is None) of `shape`. The C entry points receive only its
+    pointer, so a smaller tensor, or one on another device, would be written or read out
+    of bounds by the kernels."""
+    if t.dtype != dtype or not t.is_contiguous() or t.device != device:
+        raise ValueError(f"{what} must be a contiguous {dtype} tensor on {device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+
+
+def _check_outputs(q, out, lse, rows):
+    """out like q (bf16) and lse fp32 [B, H, Nq] (`rows`), where the caller supplies them."""
+    import torch
+    if out is not None:
+        _check_buffer(out, q.shape, torch.bfloat16, q.device, "out")
+    if lse is not None:
+        _check_buffer(lse, rows, torch.float32, q.device, "lse")
+
+
+def _check_equal_lengths(q, k, what):
+    if tuple(k.shape) != tuple(q.shape):
+        raise ValueError(f"{what} needs equal query and key lengths")
+
+
 def _scale(scale, d):
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
@@ -166,6 +191,7 @@ def forward(q, k, v, causal: bool = False, scale=None, out=None, lse=None, layou
     import torch
     _check_qkv(q, k, v, layout=layout)
     B, H, N, Nk, d = _dims(q, k, layout)
+    _check_outputs(q, out, lse, (B, H, N))
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     with torch.cuda.device(q.device):
@@ -196,8 +222,10 @@ def forward_blocksparse(q, k, v, tile_mask, scale=None, mask_block: int = 128, o
     """Block-sparse forward: attention restricted to the kept 128x128 tiles."""
     import torch
     _check_qkv(q, k, v)
+    _check_equal_lengths(q, k, "block-sparse attention")
     _check_mask(tile_mask, q, mask_block)
     B, H, N, d = q.shape
+    _check_outputs(q, out, lse, (B, H, N))
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     with torch.cuda.device(q.device):
@@ -226,6 +254,7 @@ def forward_dropout(q, k, v, p: float, seed: int, offset: int = 0, causal: bool 
         raise ValueError("dropout needs equal query and key lengths")
     p, seed, offset = _seed_args(p, seed, offset)
     B, H, N, d = q.shape
+    _check_outputs(q, out, lse, (B, H, N))
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     with torch.cuda.device(q.device):
@@ -252,8 +281,15 @@ def _bwd_prep(q, k, v, o, lse, do, workspace, grads, layout="bhnd", deterministi
     need = bwd_workspace_bytes(B, H, N, d, deterministic)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _check_buffer(workspace, None, torch.uint8, q.device, "workspace")  # its size is checked in C
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    else:
+        if len(grads) != 3:
+            raise ValueError("grads must be (dq, dk, dv)")
+        for g, like, name in zip(grads, (q, k, v), ("dq", "dk", "dv")):
+            _check_buffer(g, like.shape, torch.bfloat16, q.device, name)
     return workspace, grads
 
 
@@ -335,6 +371,8 @@ def backward_blocksparse(q, k, v, o, lse, do, tile_mask, scale=None, mask_block:
                          grads=None, deterministic=None):
     """Block-sparse backward (same mask as the forward); deterministic as for backward."""
     import torch
+    _check_qkv(q, k, v, o, do)
+    _check_equal_lengths(q, k, "block-sparse attention")
     _check_mask(tile_mask, q, mask_block)
     if not _deterministic(deterministic, q.shape[-1]):
         return _bwd_fused(q, k, v, o, lse, do, False, scale, workspace, grads, "bhnd", tile_mask, mask_block)
@@ -362,8 +400,23 @@ def device_status(device=None):
 # ---------------------------------------------------------------- staged backward
 # The three launches of ``backward`` as separate calls (same workspace for all three).
 
+def _check_stage(q, *like, lse=None, workspace=None, tile_mask=None, mask_block=128):
+    """Arguments of a staged call: q and every tensor in `like` contiguous bf16 CUDA
+    tensors of q's [B, H, N, d] shape on q's device (one length for queries and keys);
+    lse fp32 [B, H, N]; the workspace uint8 on that device (its size is checked in C);
+    the tile mask as for the block-sparse calls."""
+    import torch
+    _check_qkv(q, q, q, *like)
+    if lse is not None:
+        _check_buffer(lse, q.shape[:3], torch.float32, q.device, "lse")
+    if workspace is not None:
+        _check_buffer(workspace, None, torch.uint8, q.device, "workspace")
+    if tile_mask is not None:
+        _check_mask(tile_mask, q, mask_block)
+
 def bwd_preprocess(o, do, lse, workspace):
     import torch
+    _check_stage(o, do, lse=lse, workspace=workspace)
     B, H, N, d = o.shape
     with torch.cuda.device(o.device):
         st = lib().fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
@@ -373,6 +426,7 @@ def bwd_preprocess(o, do, lse, workspace):
 
 def bwd_dkdv(q, k, v, do, dk, dv, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
     import torch
+    _check_stage(q, k, v, do, dk, dv, workspace=workspace, tile_mask=tile_mask, mask_block=mask_block)
     B, H, N, d = q.shape
     with torch.cuda.device(q.device):
         st = lib().fa_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
@@ -384,6 +438,7 @@ def bwd_dkdv(q, k, v, do, dk, dv, workspace, causal=False, scale=None, tile_mask
 
 def bwd_dq(q, k, v, do, dq, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
     import torch
+    _check_stage(q, k, v, do, dq, workspace=workspace, tile_mask=tile_mask, mask_block=mask_block)
     B, H, N, d = q.shape
     with torch.cuda.device(q.device):
         st = lib().fa_bwd_dq(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dq.data_ptr(),
@@ -398,6 +453,7 @@ def bwd_dq(q, k, v, do, dq, workspace, causal=False, scale=None, tile_mask=None,
 
 def bwd_fused_preprocess(o, do, lse, workspace):
     import torch
+    _check_stage(o, do, lse=lse, workspace=workspace)
     B, H, N, d = o.shape
     with torch.cuda.device(o.device):
         st = lib().fa_bwd_fused_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
@@ -407,6 +463,7 @@ def bwd_fused_preprocess(o, do, lse, workspace):
 
 def bwd_fused_main(q, k, v, do, dk, dv, workspace, causal=False, scale=None, tile_mask=None, mask_block=128):
     import torch
+    _check_stage(q, k, v, do, dk, dv, workspace=workspace, tile_mask=tile_mask, mask_block=mask_block)
     B, H, N, d = q.shape
     with torch.cuda.device(q.device):
         st = lib().fa_bwd_fused_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
@@ -418,6 +475,7 @@ def bwd_fused_main(q, k, v, do, dk, dv, workspace, causal=False, scale=None, til
 
 def bwd_fused_dq(dq, workspace, scale=None):
     import torch
+    _check_stage(dq, workspace=workspace)
     B, H, N, d = dq.shape
     with torch.cuda.device(dq.device):
         st = lib().fa_bwd_fused_dq(dq.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, N, d,
@@ -502,10 +560,12 @@ def forward_merge(q, k, v, o_acc, lse_acc, causal: bool = False, scale=None):
     _check_qkv(q, k, v)
     if k.shape != q.shape:
         raise ValueError("query and key blocks must have the same shape")
-    if o_acc.dtype != torch.float32 or tuple(o_acc.shape) != tuple(q.shape) or not o_acc.is_contiguous():
-        raise ValueError("o_acc must be a contiguous fp32 tensor of q's shape")
-    if lse_acc.dtype != torch.float32 or tuple(lse_acc.shape) != tuple(q.shape[:3]) or not lse_acc.is_contiguous():
-        raise ValueError("lse_acc must be a contiguous fp32 [B, H, N] tensor")
+    if o_acc.dtype != torch.float32 or tuple(o_acc.shape) != tuple(q.shape) or not o_acc.is_contiguous() \
+            or o_acc.device != q.device:
+        raise ValueError("o_acc must be a contiguous fp32 tensor of q's shape on q's device")
+    if lse_acc.dtype != torch.float32 or tuple(lse_acc.shape) != tuple(q.shape[:3]) or not lse_acc.is_contiguous() \
+            or lse_acc.device != q.device:
+        raise ValueError("lse_acc must be a contiguous fp32 [B, H, N] tensor on q's device")
     B, H, N, d = q.shape
     with torch.cuda.device(q.device):
         st = lib().fa_fwd_merge(q.data_ptr(), k.data_ptr(), v.data_ptr(), o_acc.data_ptr(), lse_acc.data_ptr(), B, H, N,
@@ -517,10 +577,12 @@ def bwd_fused_main_f32(q, k, v, do, dk32, dv32, workspace, causal=False, scale=N
     """The fused backward's main kernel with fp32 dK, dV outputs (dQ's share added into the
     workspace's accumulator, as bwd_fused_main)."""
     import torch
+    _check_stage(q, k, v, do, workspace=workspace)
     B, H, N, d = q.shape
     for t in (dk32, dv32):
-        if t.dtype != torch.float32 or tuple(t.shape) != tuple(k.shape) or not t.is_contiguous():
-            raise ValueError("dk32 and dv32 must be contiguous fp32 tensors of k's shape")
+        if t.dtype != torch.float32 or tuple(t.shape) != tuple(k.shape) or not t.is_contiguous() \
+                or t.device != q.device:
+            raise ValueError("dk32 and dv32 must be contiguous fp32 tensors of k's shape on q's device")
     with torch.cuda.device(q.device):
         st = lib().fa_bwd_fused_main_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk32.data_ptr(),
                                          dv32.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, N, d,

@@ -92,3 +92,47 @@ def test_ring_rejects_blocks_of_different_shapes():
     q, k = _bf16(1, 1, 128, 64), _bf16(1, 1, 256, 64)
     with pytest.raises(ValueError):
         ring.ring_forward(q, k, k, ring=_RingThatMustNotExchange(), ops=ring.CudaBlockOps(0.1))
+
+
+def test_caller_buffers_are_checked_before_any_call():
+    """Outputs, row arrays and workspaces a caller supplies reach the C entry points as bare
+    pointers: shape, dtype, contiguity and device are checked in the binding."""
+    cpu = torch.device("cpu")
+    good = _bf16(1, 2, 128, 64)
+    fa._check_buffer(good, (1, 2, 128, 64), torch.bfloat16, cpu, "out")  # accepted
+    fa._check_buffer(torch.zeros(100, dtype=torch.uint8), None, torch.uint8, cpu, "workspace")
+    with pytest.raises(ValueError):  # one query row short: the kernel would write past it
+        fa._check_buffer(_bf16(1, 2, 127, 64), (1, 2, 128, 64), torch.bfloat16, cpu, "out")
+    with pytest.raises(ValueError):
+        fa._check_buffer(good.float(), (1, 2, 128, 64), torch.bfloat16, cpu, "out")
+    with pytest.raises(ValueError):
+        fa._check_buffer(_bf16(1, 2, 64, 128).transpose(2, 3), (1, 2, 128, 64), torch.bfloat16, cpu, "out")
+    with pytest.raises(ValueError):  # a workspace must be bytes (its size is counted in elements)
+        fa._check_buffer(torch.zeros(100), None, torch.uint8, cpu, "workspace")
+    with pytest.raises(ValueError):  # on another device than q
+        fa._check_buffer(good, (1, 2, 128, 64), torch.bfloat16, torch.device("cuda", 0), "out")
+    with pytest.raises(ValueError):
+        fa._check_outputs(good, None, torch.zeros(1, 2, 64), (1, 2, 128))
+    with pytest.raises(ValueError):
+        fa._check_equal_lengths(good, _bf16(1, 2, 256, 64), "block-sparse attention")
+    fa._check_equal_lengths(good, good, "block-sparse attention")
+
+
+def test_staged_calls_reject_cpu_tensors():
+    q = _bf16(1, 1, 128, 64)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    lse = torch.zeros(1, 1, 128)
+    with pytest.raises(ValueError):
+        fa.bwd_preprocess(q, q, lse, ws)
+    with pytest.raises(ValueError):
+        fa.bwd_fused_preprocess(q, q, lse, ws)
+    with pytest.raises(ValueError):
+        fa.bwd_dkdv(q, q, q, q, q, q, ws)
+    with pytest.raises(ValueError):
+        fa.bwd_dq(q, q, q, q, q, ws)
+    with pytest.raises(ValueError):
+        fa.bwd_fused_main(q, q, q, q, q, q, ws)
+    with pytest.raises(ValueError):
+        fa.bwd_fused_dq(q, ws)
+    with pytest.raises(ValueError):
+        fa.bwd_fused_main_f32(q, q, q, q, q.float(), q.float(), ws)
