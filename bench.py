@@ -165,13 +165,33 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- helpers
 
-def peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+def peaks(path=None):
+    """Roofline denominators: hbm_gbs, bf16_tflops (burst) and bf16_tflops_sustained from
+    MEASURED_PEAKS.json where the file gives them as positive numbers (at its top level or
+    one level down), each missing one from the machine's fallback figures. The kind says which:
+    "measured", "fallback", or "measured, partly fallback". A missing or unreadable file
+    means the fallback figures, never an error."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json") if path is None else path
+    out = dict(FALLBACK_PEAKS)
+    try:
         with open(p) as f:
             d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+    except (OSError, ValueError):
+        return out, "fallback"
+    if not isinstance(d, dict):
+        return out, "fallback"
+    scopes = [d] + [v for v in d.values() if isinstance(v, dict)]
+    found = 0
+    for key in FALLBACK_PEAKS:
+        for sc in scopes:
+            v = sc.get(key)
+            if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+                out[key] = float(v)
+                found += 1
+                break
+    if found == 0:
+        return out, "fallback"
+    return out, "measured" if found == len(FALLBACK_PEAKS) else "measured, partly fallback"
 
 
 # The files the profiled attention kernels and their launches are compiled from: a

@@ -49,10 +49,31 @@ def test_peaks_come_from_the_measured_file():
     import os
     p, kind = bench.peaks()
     if os.path.exists(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")):
-        assert kind == "measured"
+        assert kind.startswith("measured")
     else:
         assert kind == "fallback" and p == bench.FALLBACK_PEAKS
     assert p["bf16_tflops"] > 1000 and p["hbm_gbs"] > 1000
+
+
+def test_peaks_file_forms(tmp_path):
+    """Every figure the bench divides by is present whatever the file holds: flat or
+    nested keys are taken, missing or malformed ones fall back, and the label says so."""
+    import json
+    f = tmp_path / "peaks.json"
+    full = {"hbm_gbs": 6529.4, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1388.6, "clocks": "1965 MHz"}
+    f.write_text(json.dumps(full))
+    assert bench.peaks(str(f)) == ({k: full[k] for k in bench.FALLBACK_PEAKS}, "measured")
+    f.write_text(json.dumps({"gpu": "B200", "peaks": {k: full[k] for k in bench.FALLBACK_PEAKS}}))
+    assert bench.peaks(str(f))[1] == "measured"
+    f.write_text(json.dumps({"hbm_gbs": 6529.4, "bf16_tflops": "n/a", "bf16_tflops_sustained": True}))
+    p, kind = bench.peaks(str(f))
+    assert kind == "measured, partly fallback" and p["hbm_gbs"] == 6529.4
+    assert p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert p["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    for text in ("{not json", "[1, 2]", json.dumps({"other": 1})):
+        f.write_text(text)
+        assert bench.peaks(str(f)) == (bench.FALLBACK_PEAKS, "fallback")
+    assert bench.peaks(str(tmp_path / "absent.json")) == (bench.FALLBACK_PEAKS, "fallback")
 
 
 def test_traffic_only_while_sources_unchanged(tmp_path, monkeypatch):
