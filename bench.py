@@ -294,6 +294,17 @@ def cpu_oracle_sample(wl, budget_s: float, seed: int = 0):
     return flops / el / 1e12, desc, el
 
 
+def line_config(wl_name, wl, world: int) -> dict:
+    """The `config` object of both arms' JSON lines: the workload and the job's layout,
+    identical for the kernels and for the oracle so that the two lines describe the same
+    configuration (how each arm computes a step is stated outside it)."""
+    return {"workload": wl_name, "B": wl["B"], "H": wl["H"], "N": wl["N"], "d": wl["d"],
+            "variants": [v[0] for v in wl["variants"]],
+            "l2": "kernels: flushed before every timed step (256 MiB write, outside the step events); "
+                  "oracle: host memory",
+            "parallelism": f"replicas x{world} (independent (batch, head) shards, no collective)"}
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, wl_name, wl):
@@ -316,8 +327,8 @@ def run_reference(args, wl_name, wl):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * statistics.mean(times), 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded inputs)",
-        "config": {"workload": wl_name, "B": wl["B"], "H": wl["H"], "N": wl["N"], "d": wl["d"],
-                   "variants": [v[0] for v in wl["variants"]]},
+        "config": line_config(wl_name, wl, int(os.environ.get("WORLD_SIZE", args.gpus))),
+        "step": "per step: fp64 forward+backward of sampled (batch, head) pairs of the workload (all variants)",
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPs/s", "cores": cores, "kind": "oracle",
                          "sample": f"per step: {desc}"},
         "e2e": {"value": round(value, 6), "unit": "TFLOPs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -570,15 +581,12 @@ def run_ours(args, wl_name, wl):
         "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) inputs rounded to bf16; per-rank seeds)",
-        "config": {"workload": wl_name, "B": B, "H": H, "N": N, "d": d,
-                   "variants": [v[0] for v in wl["variants"]],
-                   "step": ("per variant: forward, backward pre-pass (D, lse rows, dQ accumulator zeroed), fused "
-                            "backward kernel (dK, dV, dQ shares reduced in fp32), dQ conversion" if fused else
-                            "per variant: forward, backward pre-pass, backward dK/dV kernel, backward dQ kernel"),
-                   "backward": ("fused: one kernel, dQ reduced in fp32 by TMA reduce-add (run-to-run order varies)"
-                                if fused else "deterministic: dK/dV kernel + dQ kernel (bit-reproducible)"),
-                   "l2": "flushed before every timed step (256 MiB write, outside the step events)",
-                   "parallelism": f"replicas x{world} (independent (batch, head) shards, no collective)"},
+        "config": line_config(wl_name, wl, world),
+        "step": ("per variant: forward, backward pre-pass (D, lse rows, dQ accumulator zeroed), fused "
+                 "backward kernel (dK, dV, dQ shares reduced in fp32), dQ conversion" if fused else
+                 "per variant: forward, backward pre-pass, backward dK/dV kernel, backward dQ kernel"),
+        "backward": ("fused: one kernel, dQ reduced in fp32 by TMA reduce-add (run-to-run order varies)"
+                     if fused else "deterministic: dK/dV kernel + dQ kernel (bit-reproducible)"),
         "pct_of_peak": round(100 * value / world / peak, 2),
         "pct_of_spec_peak": round(100 * value / world / SPEC_BF16_TFLOPS, 2),
         "peak_tflops": peak, "peak_kind": peak_label,

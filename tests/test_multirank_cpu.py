@@ -85,5 +85,9 @@ def test_reference_arm_under_the_launcher():
     line = lines[0]
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    # the same config object as the kernels' line, so the two arms compare
+    import bench
+    wl_name = line["config"]["workload"]
+    assert line["config"] == bench.line_config(wl_name, bench.workload(wl_name), 2)
     ncpu = len(os.sched_getaffinity(0))
     assert line["cpu_baseline"]["cores"] > 1 or ncpu == 1, line["cpu_baseline"]
