@@ -1,10 +1,13 @@
 """The persistent kernels' work schedules, restated in Python from their definitions
 (csrc/fa_ptx.cuh item_position, csrc/fa_bwd.cuh bwd_item, csrc/fa_bwd_fused.cuh FusedWalk,
-csrc/fa_api.cu launch_fused) and checked for the properties the kernels rely on: every
-(batch*head, tile) item is visited by exactly one CTA, paired causal items all cost the
-same, and the launcher pairs only when the pairs fill the last round of CTAs."""
+csrc/fa_api.cu launch_fused, csrc/fa_fwd.cuh fwd_item / causal_klast / FwdSched) and checked
+for the properties the kernels rely on: every (batch*head, tile) item is visited by exactly
+one CTA, paired causal items all cost the same, the launcher pairs only when the pairs fill
+the last round of CTAs, and the forward visits every key tile that holds a visible
+(query, key) pair."""
 import itertools
 
+import numpy as np
 import pytest
 
 
@@ -80,3 +83,71 @@ def test_pairs_fill_the_rounds_at_the_bench_shape():
     assert not launcher_pairs(32, 16, 148)
     # one head per SM always fills the rounds (the parity test that forces pairing)
     assert launcher_pairs(3, 148, 148) and launcher_pairs(8, 148, 148)
+
+
+# ------------------------------------------------------------------ forward
+
+
+def fwd_item(causal, n_qblocks, bh_count, k, grid, cta):
+    """(bh, qb) of a CTA's k-th forward item; an item is Q tiles 2 qb and 2 qb + 1."""
+    pos = item_position(n_qblocks * bh_count, k, grid, cta)
+    if pos < 0:
+        return None
+    if causal:  # block-major, the costliest (last) query block first
+        return (pos % bh_count, n_qblocks - 1 - pos // bh_count)
+    return (pos // n_qblocks, n_qblocks - 1 - pos % n_qblocks)  # head-major
+
+
+def causal_klast(t, off, n_ktiles):
+    """Last key tile Q tile t visits with the causal mask (bottom-right aligned, off = Nk - Nq)."""
+    x = 128 * t + 127 + off
+    last = -1 if x < 0 else x >> 7
+    return min(last, n_ktiles - 1)
+
+
+def fwd_visits(t, causal, n_ktiles, off):
+    last = causal_klast(t, off, n_ktiles) if causal else n_ktiles - 1
+    return set(range(last + 1))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_items_cover_every_query_tile_once(causal):
+    for n_tiles, bh_count, sms in itertools.product((1, 2, 3, 5, 16, 63, 64), (1, 3, 32), (7, 148)):
+        n_qblocks = (n_tiles + 1) // 2
+        grid = min(n_qblocks * bh_count, sms)
+        tiles = []
+        for cta in range(grid):
+            k, qbs = 0, []
+            while (it := fwd_item(causal, n_qblocks, bh_count, k, grid, cta)) is not None:
+                bh, qb = it
+                tiles += [(bh, t) for t in (2 * qb, 2 * qb + 1) if t < n_tiles]
+                qbs.append(qb)
+                k += 1
+            if causal:  # each CTA's items get no costlier: the deal stays balanced
+                assert qbs == sorted(qbs, reverse=True), (n_tiles, bh_count, sms, cta)
+        assert sorted(tiles) == sorted(itertools.product(range(bh_count), range(n_tiles)))
+
+
+@pytest.mark.parametrize("nq,nk", [(128, 128), (300, 300), (1000, 1000), (200, 700), (700, 200),
+                                   (129, 1), (1, 129), (384, 256), (256, 384)])
+def test_causal_forward_visits_every_visible_key_tile(nq, nk):
+    """Brute force over (query, key) pairs: key j is visible to query i iff j <= i + Nk - Nq.
+    Every key tile holding a visible pair of one of a Q tile's real rows is visited; a tile
+    whose rows see nothing visits nothing (those rows get O = 0, lse = -inf); a visited tile
+    that no real row sees occurs only in the last, partial Q tile (its element mask zeroes it)."""
+    off = nk - nq
+    n_tiles, n_ktiles = -(-nq // 128), -(-nk // 128)
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    vis = j <= i + off
+    for t in range(n_tiles):
+        rows = vis[128 * t:128 * (t + 1)]
+        needed = {jt for jt in range(n_ktiles) if rows[:, 128 * jt:128 * (jt + 1)].any()}
+        got = fwd_visits(t, True, n_ktiles, off)
+        assert needed <= got, (nq, nk, t, sorted(needed - got))
+        if not needed:
+            assert not got, (nq, nk, t)
+        if got - needed:
+            assert t == n_tiles - 1 and nq % 128, (nq, nk, t, sorted(got - needed))
+        if nq == nk:  # the square case: the diagonal tile is the last one
+            assert max(got) == t
