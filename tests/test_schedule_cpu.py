@@ -151,3 +151,31 @@ def test_causal_forward_visits_every_visible_key_tile(nq, nk):
             assert t == n_tiles - 1 and nq % 128, (nq, nk, t, sorted(got - needed))
         if nq == nk:  # the square case: the diagonal tile is the last one
             assert max(got) == t
+
+
+# ------------------------------------------------------------------ backward visibility
+
+
+def causal_qfirst(j, off):
+    """First query tile that sees key tile j (dK/dV and fused kernels)."""
+    x = 128 * j - 127 - off
+    return 0 if x <= 0 else (x + 127) >> 7
+
+
+@pytest.mark.parametrize("nq,nk", [(128, 128), (300, 300), (1000, 1000), (200, 700), (700, 200),
+                                   (129, 1), (1, 129), (384, 256), (256, 384), (640, 1000)])
+def test_causal_backward_pairs(nq, nk):
+    """The dK/dV side (query tiles t >= qfirst(j) of key tile j) and the dQ side (key tiles
+    j <= klast(t) of query tile t) visit the same (query tile, key tile) pairs, and these
+    hold every visible (query, key) pair of real rows and keys."""
+    off = nk - nq
+    n_tiles, n_ktiles = -(-nq // 128), -(-nk // 128)
+    by_key = {(t, j) for j in range(n_ktiles) for t in range(causal_qfirst(j, off), n_tiles)}
+    by_query = {(t, j) for t in range(n_tiles) for j in range(causal_klast(t, off, n_ktiles) + 1)}
+    assert by_key == by_query, (nq, nk, sorted(by_key ^ by_query))
+    vis = np.arange(nk)[None, :] <= np.arange(nq)[:, None] + off
+    needed = {(t, j) for t in range(n_tiles) for j in range(n_ktiles)
+              if vis[128 * t:128 * (t + 1), 128 * j:128 * (j + 1)].any()}
+    assert needed <= by_key, (nq, nk, sorted(needed - by_key))
+    extra = by_key - needed  # pairs no real row sees: only in the last, partial query tile
+    assert all(t == n_tiles - 1 and nq % 128 for t, _ in extra), (nq, nk, sorted(extra))
