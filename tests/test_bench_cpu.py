@@ -115,3 +115,21 @@ def test_source_hash_covers_the_kernel_files(tmp_path, monkeypatch):
     with open(csrc / "fa_bwd.cuh", "a") as f:
         f.write("\n")
     assert bench.kernel_source_hash() != h0
+
+
+def test_clock_samples_are_summarised():
+    """The clock record that decides whether a run is kept: median SM clock, the largest
+    maximum, and every throttle reason active in any sample."""
+    na = "Not Active"
+    rows = [f"0, 1965, 1965, 240.5, 0x0, {na}, {na}, {na}, {na}",
+            f"0, 1665, 1965, 998.0, 0x4, {na}, {na}, {na}, Active",
+            f"0, 1700, 1965, 990.1, 0x4, {na}, {na}, {na}, Active",
+            "0, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",
+            "garbage", ""]
+    c = bench.parse_clock_lines(rows)
+    assert c == {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c = bench.parse_clock_lines([f"0, 1200, 1965, 700.0, 0x8, Active, {na}, Active, {na}"])
+    assert c["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.parse_clock_lines(["[N/A]"]) is None and bench.parse_clock_lines([]) is None
+    # with no samples the line is rated against the burst peak (no clock evidence of a cap)
+    assert bench.ClockSampler(0).stop() is None
