@@ -41,6 +41,12 @@
  *    element is visible (the mask is not combined with causal).
  *  - Ownership: the caller owns every buffer. The library allocates and frees no
  *    device memory on these paths; scratch is caller-provided ("workspace").
+ *  - Buffer sizes: each buffer must hold the elements its documented shape implies
+ *    (q: B*H*N*d bf16, lse: B*H*N fp32, ...). The library receives only pointers and
+ *    cannot check this (it checks the workspace's byte count, which is passed): a
+ *    smaller buffer, or one on another device, is read or written out of bounds.
+ *    The Python binding checks every tensor's shape, dtype, contiguity and device
+ *    before it calls.
  *  - Asynchrony: each call only enqueues work on `stream` (a cudaStream_t, or
  *    NULL for the legacy default stream) and returns; no implicit synchronisation.
  *    Inputs must stay unmodified, and outputs unread, until the stream reaches
